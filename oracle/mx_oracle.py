@@ -1,0 +1,441 @@
+"""Plain CPU oracle of the MXFP8 training hot path (numpy, float64).
+
+TEST INFRASTRUCTURE ONLY: nothing in the product path imports it. It shares
+no code, table or constant generator with the CUDA library; the only module
+both sides use is the seeded input generator, which holds none of the
+arithmetic below.
+
+What it computes, and where each step comes from
+------------------------------------------------
+* MX block format: FP8 E4M3 elements that share one E8M0 power-of-two scale
+  per block of 32 values ("blocked E8M0 scales", torchtitan PR #5334,
+  description; "1x32" casts, ao PR "[moe training] Add backward_override to
+  the MXFP8 grouped GEMM", Design notes).
+* RCEIL scale rule ("shared RCEIL constant", "32x32 RCEIL weight-scale
+  policy", torchtitan PR #5334, description and review thread): the scale of a
+  block is the smallest power of two 2**e with 448 * 2**e >= amax, stored as
+  the E8M0 byte b = e + 127 clamped to [0, 254]. 448 is the largest finite
+  E4M3 value. A block whose amax is 0 gets b = 0.
+* Element cast: q = round-to-nearest-even, saturating E4M3 encoding of
+  x * 2**(127 - b), with the sign of zero kept.
+* Block geometry: rowwise "dim0" (1x32 along the contiguous axis), columnwise
+  "dim1" (32x1 down the columns, stored transposed), fused row+column (both
+  from one read; "fused dense rowwise/columnwise cast", torchtitan PR #5334),
+  and square 32x32 weight blocks ("32x32 RCEIL weight-scale policy", same
+  page), which let one quantized weight serve both the forward GEMM and the
+  dgrad GEMM.
+* Blocked ("swizzled") scale layout: the pages name it ("swizzled layouts are
+  directly output", torchtitan PR #5334) but do not define it. Reading taken:
+  the layout the Blackwell block-scaled MMA consumes -- 128-row x 4-column
+  tiles of 512 bytes, tile-major with the column tiles of a row band
+  contiguous, and inside a tile byte (r % 32) * 16 + (r // 32) * 4 + c.
+  Padding bytes are 0x00.
+* Grouped operands and the pad path ("pad_token_groups_for_grouped_mm" and
+  padded offsets, ao backward_override PR, Known follow-ups; "pad/unpad" and
+  "M-groups / K-groups scale rearrange" kernels, ao PR #4705 stack list): each
+  token group is placed at a row offset that is a multiple of 128, so that
+  every 128-row scale tile belongs to one group; pad rows are zero.
+* Scaled grouped GEMM over an offsets array (ao backward_override PR,
+  Summary): Y[rows of group g] = deq(X_g) @ deq(W_g)^T; dgrad
+  dX_g = dY_g @ W_g; wgrad dW_g = dY_g^T @ X_g, an empty group giving
+  dW_g = 0. Computed here in float64 over the dequantized operands.
+* MXFP8 linear forward / dgrad / wgrad ("MXFP8Linear training paths", ao PR
+  #4705) composed from the casts above at one group.
+
+Where the pages are silent, the readings taken are listed in the repository's
+design notes; each is restated beside the function that depends on it.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 32            # elements that share one scale
+E4M3_MAX = 448.0      # largest finite E4M3 value
+E8M0_BIAS = 127
+E8M0_MAX_FINITE = 254  # 255 is the E8M0 NaN encoding
+SCALE_TILE_ROWS = 128
+SCALE_TILE_COLS = 4
+GROUP_ALIGN = 128
+
+
+def ceil_to(x, a):
+    return ((x + a - 1) // a) * a
+
+
+# --------------------------------------------------------------------------
+# bf16 inputs are carried as their uint16 bit patterns
+# --------------------------------------------------------------------------
+def bf16_to_f64(bits) -> np.ndarray:
+    """Exact value of each bf16 bit pattern, as float64."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 ("fn" variant: bias 7, no infinities, NaN = S.1111.111)
+# --------------------------------------------------------------------------
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 code from the format definition (float64)."""
+    c = np.asarray(codes).astype(np.int64)
+    sign = c >> 7
+    exp = (c >> 3) & 0xF
+    man = c & 0x7
+    subnormal = man / 8.0 * 2.0 ** (1 - 7)
+    normal = (1.0 + man / 8.0) * np.exp2(exp - 7.0)
+    mag = np.where(exp == 0, subnormal, normal)
+    mag = np.where((exp == 0xF) & (man == 0x7), np.nan, mag)
+    return np.where(sign == 1, -mag, mag)
+
+
+# The 127 finite non-negative codes 0x00..0x7E; their values increase with the
+# code, so nearest-value search is a sorted search.
+_POS_CODES = np.arange(0x7F, dtype=np.int64)
+_POS_VALUES = e4m3_decode(_POS_CODES)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """Round-to-nearest-even E4M3 code of each float64 value.
+
+    Saturates to +-448 (the "satfinite" behaviour), keeps the sign of zero
+    (a negative value that rounds to zero gives 0x80) and breaks ties toward
+    the code whose mantissa is even. Inputs must be finite.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("e4m3_encode: non-finite input is outside the contract")
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    hi = np.searchsorted(_POS_VALUES, a, side="left")   # first value >= a
+    hi = np.minimum(hi, len(_POS_VALUES) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _POS_VALUES[lo]
+    d_hi = _POS_VALUES[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    sign = np.signbit(v).astype(np.int64)
+    return (code | (sign << 7)).astype(np.uint8)
+
+
+# --------------------------------------------------------------------------
+# E8M0 scale under RCEIL
+# --------------------------------------------------------------------------
+def rceil_e8m0(amax) -> np.ndarray:
+    """E8M0 byte of the RCEIL scale of blocks with the given amax.
+
+    b = clamp(e + 127, 0, 254) with e the smallest integer such that
+    448 * 2**e >= amax (i.e. e = ceil(log2(amax / 448)) in exact arithmetic).
+    amax == 0 gives b = 0 (the all-zero block; reading: the pages are silent,
+    the exact formula gives -inf before the clamp).
+
+    The search starts from a float64 log2 estimate and is then settled with
+    exact comparisons (448 * 2**e is exact in float64), so the result is the
+    exact minimum whatever the rounding of log2.
+    """
+    amax = np.asarray(amax, dtype=np.float64)
+    if np.any(~np.isfinite(amax)) or np.any(amax < 0):
+        raise ValueError("rceil_e8m0: amax must be finite and non-negative")
+    b = np.zeros(amax.shape, dtype=np.int64)
+    nz = amax > 0
+    if np.any(nz):
+        a = amax[nz]
+        e = np.ceil(np.log2(a / E4M3_MAX)).astype(np.int64)
+        for _ in range(4):   # each pass moves e by at most one step
+            too_big = np.ldexp(E4M3_MAX, e - 1) >= a
+            e = np.where(too_big, e - 1, e)
+            too_small = np.ldexp(E4M3_MAX, e) < a
+            e = np.where(too_small, e + 1, e)
+        assert np.all(np.ldexp(E4M3_MAX, e) >= a)
+        assert np.all(np.ldexp(E4M3_MAX, e - 1) < a)
+        b[nz] = np.clip(e + E8M0_BIAS, 0, E8M0_MAX_FINITE)
+    return b.astype(np.uint8)
+
+
+def e8m0_to_f64(b) -> np.ndarray:
+    """Value 2**(b - 127) of an E8M0 byte (b = 255, NaN, never produced here)."""
+    return np.exp2(np.asarray(b).astype(np.float64) - E8M0_BIAS)
+
+
+def quantize_blocks(xf, axis=-1):
+    """Quantize float64 blocks whose 32 elements lie along ``axis``.
+
+    Returns (q, b): q has the shape of xf (uint8 E4M3 codes), b has ``axis``
+    removed (uint8 E8M0 bytes).
+    """
+    xf = np.asarray(xf, dtype=np.float64)
+    if xf.shape[axis] != BLOCK:
+        raise ValueError("quantize_blocks: block axis must hold 32 elements")
+    amax = np.max(np.abs(xf), axis=axis)
+    b = rceil_e8m0(amax)
+    inv_scale = np.expand_dims(np.exp2(E8M0_BIAS - b.astype(np.float64)), axis)
+    q = e4m3_encode(xf * inv_scale)      # exact: scaling by a power of two
+    return q, b
+
+
+# --------------------------------------------------------------------------
+# The four casts (logical scales; the blocked layout is applied separately)
+# --------------------------------------------------------------------------
+def cast_dim0(x_bits):
+    """Rowwise 1x32 cast of bf16 X[R, C] -> (Q[R, C], S[R, C/32])."""
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    R, C = x_bits.shape
+    if C % BLOCK:
+        raise ValueError("cast_dim0: the row length must be a multiple of 32")
+    xf = bf16_to_f64(x_bits).reshape(R, C // BLOCK, BLOCK)
+    q, b = quantize_blocks(xf, axis=-1)
+    return q.reshape(R, C), b
+
+
+def cast_dim1(x_bits):
+    """Columnwise 32x1 cast of bf16 X[R, C] -> (Q^T[C, R], S[C, R/32]).
+
+    Blocks are X[32i:32i+32, c]; the output is stored transposed so that the
+    reduced axis is contiguous.
+    """
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    R, C = x_bits.shape
+    if R % BLOCK:
+        raise ValueError("cast_dim1: the column length must be a multiple of 32")
+    xf = bf16_to_f64(x_bits).reshape(R // BLOCK, BLOCK, C)   # [block, row-in-block, col]
+    q, b = quantize_blocks(xf, axis=1)                        # q [R/32, 32, C], b [R/32, C]
+    return np.ascontiguousarray(q.reshape(R, C).T), np.ascontiguousarray(b.T)
+
+
+def cast_2d(x_bits):
+    """Fused rowwise + columnwise cast: exactly the pair (dim0, dim1)."""
+    return cast_dim0(x_bits), cast_dim1(x_bits)
+
+
+def cast_32x32(w_bits):
+    """Square-block cast of bf16 W[..., N, K] -> (Q[..., N, K], S[..., N/32, K/32]).
+
+    One scale per 32x32 tile; stacks [G, N, K] are cast per expert (tiles
+    never cross experts).
+    """
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    *lead, N, K = w_bits.shape
+    if N % BLOCK or K % BLOCK:
+        raise ValueError("cast_32x32: both matrix dims must be multiples of 32")
+    xf = bf16_to_f64(w_bits).reshape(*lead, N // BLOCK, BLOCK, K // BLOCK, BLOCK)
+    amax = np.max(np.abs(xf), axis=(-3, -1))                  # [..., N/32, K/32]
+    b = rceil_e8m0(amax)
+    inv_scale = np.exp2(E8M0_BIAS - b.astype(np.float64))[..., :, None, :, None]
+    q = e4m3_encode(xf * inv_scale)
+    return q.reshape(*lead, N, K), b
+
+
+def w32_scale_views(s_tile):
+    """The two per-row scale views of 32x32 tile scales S[..., N/32, K/32].
+
+    S_fwd[n, kb] = S[n // 32, kb] scales W[N, K] along K (forward GEMM);
+    S_dgrad[k, nb] = S[nb, k // 32] scales W^T[K, N] along N (dgrad GEMM).
+    """
+    s_tile = np.asarray(s_tile)
+    s_fwd = np.repeat(s_tile, BLOCK, axis=-2)
+    s_dgrad = np.repeat(np.swapaxes(s_tile, -1, -2), BLOCK, axis=-2)
+    return s_fwd, s_dgrad
+
+
+# --------------------------------------------------------------------------
+# Blocked (swizzled) scale layout
+# --------------------------------------------------------------------------
+def blocked_scale_bytes(rows, cols):
+    """Size of the blocked layout of a logical scale matrix S[rows, cols]."""
+    return ceil_to(rows, SCALE_TILE_ROWS) * ceil_to(cols, SCALE_TILE_COLS)
+
+
+def blocked_offset(r, c, cols):
+    """Byte offset of logical scale S[r, c] in the blocked layout.
+
+    Tiles of 128 rows x 4 columns hold 512 bytes; tile (r//128, c//4) sits at
+    index (r//128) * ceil(cols/4) + c//4; inside a tile the byte is
+    (r % 32) * 16 + ((r % 128) // 32) * 4 + c % 4.
+    """
+    r = np.asarray(r, dtype=np.int64)
+    c = np.asarray(c, dtype=np.int64)
+    col_tiles = ceil_to(cols, SCALE_TILE_COLS) // SCALE_TILE_COLS
+    tile = (r // SCALE_TILE_ROWS) * col_tiles + (c // SCALE_TILE_COLS)
+    rr = r % SCALE_TILE_ROWS
+    return tile * 512 + (rr % 32) * 16 + (rr // 32) * 4 + (c % SCALE_TILE_COLS)
+
+
+def swizzle(s):
+    """Logical scales S[R, C] -> blocked byte buffer (pad bytes 0x00)."""
+    s = np.asarray(s, dtype=np.uint8)
+    R, C = s.shape
+    buf = np.zeros(blocked_scale_bytes(R, C), dtype=np.uint8)
+    rr, cc = np.indices((R, C))
+    buf[blocked_offset(rr, cc, C)] = s
+    return buf
+
+
+def unswizzle(buf, R, C):
+    """Blocked byte buffer -> logical scales S[R, C]."""
+    buf = np.asarray(buf, dtype=np.uint8)
+    rr, cc = np.indices((R, C))
+    return buf[blocked_offset(rr, cc, C)]
+
+
+def swizzle_stack(s):
+    """Per-expert blocked buffers of S[G, R, C], concatenated in expert order."""
+    return np.concatenate([swizzle(s[g]) for g in range(s.shape[0])])
+
+
+# --------------------------------------------------------------------------
+# Token groups and the pad path
+# --------------------------------------------------------------------------
+def group_bounds(offs):
+    """(starts, ends) of each group from cumulative end offsets."""
+    ends = np.asarray(offs, dtype=np.int64)
+    starts = np.concatenate([[0], ends[:-1]]).astype(np.int64)
+    if np.any(ends < starts):
+        raise ValueError("offsets must be non-decreasing and start at >= 0")
+    return starts, ends
+
+
+def padded_group_starts(offs):
+    """Row offset of each group in the padded layout, plus the total.
+
+    p[0] = 0, p[g+1] = p[g] + ceil_to(size_g, 128): each group starts on a
+    128-row boundary, so each 128-row scale tile holds one group only.
+    """
+    starts, ends = group_bounds(offs)
+    padded = ceil_to(ends - starts, GROUP_ALIGN)
+    return np.concatenate([[0], np.cumsum(padded)]).astype(np.int64)
+
+
+def padded_rows_capacity(m_total, groups):
+    """An upper bound of the padded row count that holds for any offsets."""
+    return ((m_total + (GROUP_ALIGN - 1) * groups) // GROUP_ALIGN) * GROUP_ALIGN
+
+
+def cast_dim0_grouped(x_bits, offs, m_cap):
+    """dim0 cast of X[M, K] into the padded row layout with m_cap rows.
+
+    Returns (Q[m_cap, K], S[m_cap, K/32]); pad rows hold q = 0 and b = 0.
+    """
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    M, K = x_bits.shape
+    starts, ends = group_bounds(offs)
+    p = padded_group_starts(offs)
+    if ends[-1] != M or p[-1] > m_cap:
+        raise ValueError("offsets do not cover X or the capacity is too small")
+    q = np.zeros((m_cap, K), dtype=np.uint8)
+    s = np.zeros((m_cap, K // BLOCK), dtype=np.uint8)
+    for g in range(len(starts)):
+        n = ends[g] - starts[g]
+        if n == 0:
+            continue
+        qg, sg = cast_dim0(x_bits[starts[g]:ends[g]])
+        q[p[g]:p[g] + n] = qg
+        s[p[g]:p[g] + n] = sg
+    return q, s
+
+
+def cast_dim1_grouped(x_bits, offs, m_cap):
+    """Per-group dim1 cast of X[M, K] into the padded token layout.
+
+    Blocks of 32 tokens start at each group's start; a group's last partial
+    block is completed with zeros (which leaves its amax unchanged). Returns
+    (Q^T[K, m_cap], S[K, m_cap/32]); pad tokens hold q = 0, pad blocks b = 0.
+    """
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    M, K = x_bits.shape
+    starts, ends = group_bounds(offs)
+    p = padded_group_starts(offs)
+    if ends[-1] != M or p[-1] > m_cap:
+        raise ValueError("offsets do not cover X or the capacity is too small")
+    qt = np.zeros((K, m_cap), dtype=np.uint8)
+    s = np.zeros((K, m_cap // BLOCK), dtype=np.uint8)
+    for g in range(len(starts)):
+        n = ends[g] - starts[g]
+        if n == 0:
+            continue
+        rows = ceil_to(n, BLOCK)
+        xg = np.zeros((rows, K), dtype=np.uint16)     # bf16 +0.0 padding
+        xg[:n] = x_bits[starts[g]:ends[g]]
+        qg, sg = cast_dim1(xg)
+        qt[:, p[g]:p[g] + rows] = qg
+        s[:, p[g] // BLOCK:(p[g] + rows) // BLOCK] = sg
+    return qt, s
+
+
+# --------------------------------------------------------------------------
+# Dequantization and the GEMMs (float64)
+# --------------------------------------------------------------------------
+def dequant(q, s):
+    """Value of Q[..., R, C] with logical scales S[..., R, C/32] along the last axis."""
+    vals = e4m3_decode(q)
+    return vals * np.repeat(e8m0_to_f64(s), BLOCK, axis=-1)
+
+
+def mm(a, b):
+    """Dense D = A @ B^T with both operands K-contiguous, float64."""
+    return np.asarray(a, np.float64) @ np.asarray(b, np.float64).T
+
+
+def grouped_mm_m(a, b, offs):
+    """M-groups GEMM: Y[start_g:end_g] = A[p_g : p_g + size_g] @ B[g]^T.
+
+    a: dequantized padded rows [m_cap, K]; b: dequantized experts [G, N, K];
+    offs: cumulative group ends. Returns Y[M, N] in the unpadded row order.
+    """
+    starts, ends = group_bounds(offs)
+    p = padded_group_starts(offs)
+    G, N, _ = b.shape
+    y = np.zeros((ends[-1] if len(ends) else 0, N), dtype=np.float64)
+    for g in range(G):
+        n = ends[g] - starts[g]
+        if n:
+            y[starts[g]:ends[g]] = mm(a[p[g]:p[g] + n], b[g])
+    return y
+
+
+def grouped_mm_k(a, b, offs):
+    """K-groups GEMM (wgrad): D[g] = A[:, tokens of g] @ B[:, tokens of g]^T.
+
+    a: dequantized [N, m_cap], b: dequantized [K, m_cap] (tokens in the padded
+    layout). An empty group gives D[g] = 0.
+    """
+    starts, ends = group_bounds(offs)
+    p = padded_group_starts(offs)
+    G = len(starts)
+    out = np.zeros((G, a.shape[0], b.shape[0]), dtype=np.float64)
+    for g in range(G):
+        n = ends[g] - starts[g]
+        if n:
+            out[g] = mm(a[:, p[g]:p[g] + n], b[:, p[g]:p[g] + n])
+    return out
+
+
+def gemm_bound(ref, abs_ref):
+    """Allowed |gpu - ref|: 2**-7 * |ref| + 1e-3 * (|A| @ |B|^T)."""
+    return 2.0 ** -7 * np.abs(ref) + 1e-3 * abs_ref
+
+
+# --------------------------------------------------------------------------
+# Composite paths: MXFP8 linear and MoE grouped layer (float64 results)
+# --------------------------------------------------------------------------
+def linear_fwd(x_bits, w_bits):
+    """Y = X W^T with X cast 1x32 (dim0) and W cast 32x32."""
+    qx, sx = cast_dim0(x_bits)
+    qw, st = cast_32x32(w_bits)
+    s_fwd, _ = w32_scale_views(st)
+    a, b = dequant(qx, sx), dequant(qw, s_fwd)
+    return mm(a, b), mm(np.abs(a), np.abs(b))
+
+
+def linear_dgrad(dy_bits, w_bits):
+    """dX = dY W: dY cast along N (dim0), W^T scaled by the same 32x32 tiles."""
+    qd, sd = cast_dim0(dy_bits)
+    qw, st = cast_32x32(w_bits)
+    _, s_dgrad = w32_scale_views(st)
+    a = dequant(qd, sd)
+    bt = dequant(np.ascontiguousarray(qw.T), s_dgrad)     # W^T [K, N]
+    return mm(a, bt), mm(np.abs(a), np.abs(bt))
+
+
+def linear_wgrad(dy_bits, x_bits):
+    """dW = dY^T X: both operands cast along the token axis (dim1)."""
+    qdt, sdt = cast_dim1(dy_bits)      # [N, M]
+    qxt, sxt = cast_dim1(x_bits)       # [K, M]
+    a, b = dequant(qdt, sdt), dequant(qxt, sxt)
+    return mm(a, b), mm(np.abs(a), np.abs(b))

@@ -1,0 +1,370 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle against a fact the pages or the mathematics fix:
+hand-worked golden values (tests/golden/, each file citing its source),
+closed forms derived independently of the oracle's search, a library routine
+(torch's CPU float8_e4m3fn conversion), invariants of RCEIL scaling, and brute
+force on tiny inputs. A plausible slip in the oracle (wrong tie rule, dropped
+clamp, transposed operand, wrong swizzle index) fails at least one of them;
+``test_planted_*`` shows that for two such slips.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mx_oracle as O
+from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append(line.split())
+    return rows
+
+
+def _all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    exp = (bits >> 7) & 0xFF
+    return bits[exp != 0xFF]
+
+
+# ----------------------------------------------------------------- E4M3 ----
+def test_e4m3_decode_golden():
+    for code, val in _golden_rows("e4m3_codes.txt"):
+        got = O.e4m3_decode(np.array([int(code, 16)]))[0]
+        assert got == float(val) and np.signbit(got) == np.signbit(float(val)), code
+    assert np.isnan(O.e4m3_decode(np.array([0x7F, 0xFF]))).all()
+
+
+def test_e4m3_encode_roundtrips_every_finite_code():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.int64)
+    vals = O.e4m3_decode(codes)
+    assert np.array_equal(O.e4m3_encode(vals), codes.astype(np.uint8))
+
+
+def _torch_e4m3(v):
+    t = torch.from_numpy(np.asarray(v, np.float64).astype(np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+@pytest.mark.parametrize("b", [0, 1, 120, 127, 134, 247, 3, 64, 190, 230])
+def test_e4m3_encode_matches_torch_exhaustive_bf16(b):
+    """All finite bf16 x at scale byte b: oracle code == torch's RNE cast of x/2^(b-127)."""
+    x = O.bf16_to_f64(_all_finite_bf16())
+    v = x * 2.0 ** (127 - b)
+    keep = np.abs(v) <= 448.0          # torch's cast does not saturate; RCEIL never exceeds 448
+    ours = O.e4m3_encode(v[keep])
+    ref = _torch_e4m3(v[keep])
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_saturates():
+    assert O.e4m3_encode(np.array([460.0, 1000.0, -1e6, 464.0]) ).tolist() == [0x7E, 0x7E, 0xFE, 0x7E]
+
+
+# ----------------------------------------------------------------- RCEIL ---
+def _closed_form_b(bits):
+    """b from the bf16 bit fields: E - 8 + [m > 96], clamped to [0, 254].
+
+    448 = 1.75 * 2^8 and 1.75 = 1 + 96/128, so for amax = (1 + m/128) * 2^(E-127)
+    the ratio amax / 448 exceeds the power of two 2^(E-135) exactly when m > 96.
+    """
+    E = (bits.astype(np.int64) >> 7) & 0xFF
+    m = bits.astype(np.int64) & 0x7F
+    return np.clip(E - 8 + (m > 96), 0, 254)
+
+
+def test_rceil_matches_closed_form_on_every_bf16_amax():
+    bits = _all_finite_bf16()
+    bits = bits[bits < 0x8000]             # non-negative patterns (amax >= 0)
+    amax = O.bf16_to_f64(bits)
+    assert np.array_equal(O.rceil_e8m0(amax).astype(np.int64), _closed_form_b(bits))
+
+
+def test_rceil_matches_float64_log2():
+    bits = _all_finite_bf16()
+    bits = bits[(bits < 0x8000) & (bits > 0)]
+    amax = O.bf16_to_f64(bits)
+    ref = np.clip(np.ceil(np.log2(amax / 448.0)) + 127, 0, 254)
+    assert np.array_equal(O.rceil_e8m0(amax).astype(np.int64), ref.astype(np.int64))
+
+
+def test_rceil_tiny_amax_reading_gives_zero():
+    # amax <= 448 * 2^-127 (about 2.63e-36): the exact rule clamps to b = 0 (a
+    # float32 quotient amax/448 would be subnormal there and could give 1; the
+    # exact reading is kept). Just above the threshold b = 1.
+    amax = np.array([9.2e-41, 1e-38, 2.6e-36, 448.0 * 2.0 ** -127, 2.7e-36, 5.0e-36])
+    assert O.rceil_e8m0(amax).tolist() == [0, 0, 0, 0, 1, 1]
+    assert O.rceil_e8m0(np.array([0.0]))[0] == 0
+
+
+def test_worked_examples_golden():
+    for amax, b, x, q in _golden_rows("rceil_worked_examples.txt"):
+        got_b = O.rceil_e8m0(np.array([float(amax)]))[0]
+        assert got_b == int(b), amax
+        blk = np.zeros(32)
+        blk[0] = float(amax)
+        blk[1] = float(x)
+        qq, bb = O.quantize_blocks(blk)
+        assert bb == int(b)
+        assert qq[1] == int(q, 16), (amax, x)
+
+
+def test_scale_invariants_random_blocks():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((4096, 32)) * np.exp2(rng.integers(-40, 40, (4096, 1)))
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    xf = O.bf16_to_f64(S.bf16_bits(xb))
+    q, b = O.quantize_blocks(xf)
+    amax = np.abs(xf).max(axis=1)
+    scale = O.e8m0_to_f64(b)
+    assert np.all(scale >= amax / 448.0)                       # large enough
+    assert np.all((b == 0) | (scale / 2 < amax / 448.0))       # and minimal
+    deq = O.e4m3_decode(q)
+    assert np.all(np.abs(deq) <= 448.0)
+    # dequantized error within half an E4M3 ulp of the scaled value
+    v = np.abs(xf) / scale[:, None]
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -6)))
+    half_ulp = 0.5 * np.exp2(e - 3)
+    assert np.all(np.abs(xf - deq * scale[:, None]) <= half_ulp * scale[:, None])
+
+
+def test_subnormal_block_keeps_nonzero_codes():
+    # bf16 subnormals (exponent field 0) get b = 0 and are scaled by 2^127 exactly.
+    bits = np.array([0x0001, 0x0040, 0x007F, 0x8003] + [0] * 28, dtype=np.uint16)
+    xf = O.bf16_to_f64(bits)
+    q, b = O.quantize_blocks(xf)
+    assert b == 0
+    vals = O.e4m3_decode(q[:4]) * 2.0 ** -127
+    assert np.all(vals != 0) and vals[3] < 0
+
+
+# ------------------------------------------------------------ geometry -----
+def test_dim1_equals_dim0_of_transpose():
+    x = S.bf16_bits(S.tiny_activation(0))
+    q1, s1 = O.cast_dim1(x)
+    q0, s0 = O.cast_dim0(np.ascontiguousarray(x.T))
+    assert np.array_equal(q1, q0) and np.array_equal(s1, s0)
+
+
+def test_fused_is_the_pair():
+    x = S.bf16_bits(S.normal_bf16((64, 96), seed=3))
+    (a, b), (c, d) = O.cast_2d(x)
+    ea, eb = O.cast_dim0(x)
+    ec, ed = O.cast_dim1(x)
+    for u, v in ((a, ea), (b, eb), (c, ec), (d, ed)):
+        assert np.array_equal(u, v)
+
+
+def test_tiny_config_worked_blocks():
+    x = S.bf16_bits(S.tiny_activation(0))
+    q, s = O.cast_dim0(x)
+    assert s[0, 0] == 0 and not q[0, :32].any()               # the zero block
+    assert S.bf16_bits(S.tiny_activation(0))[1, 0] == 0x476A  # bf16(6e4) = 59904
+    assert s[1, 0] == 135 and q[1, 0] == 0x77
+
+
+def test_32x32_brute_force():
+    w = S.bf16_bits(S.normal_bf16((64, 96), 0.02, seed=5))
+    q, st = O.cast_32x32(w)
+    wf = O.bf16_to_f64(w)
+    for i in range(2):
+        for j in range(3):
+            tile = wf[32 * i:32 * i + 32, 32 * j:32 * j + 32]
+            amax = float(np.abs(tile).max())
+            e = 0
+            while 448.0 * 2.0 ** e >= amax:      # walk down then up: smallest e
+                e -= 1
+            while 448.0 * 2.0 ** e < amax:
+                e += 1
+            assert st[i, j] == e + 127
+            for r in range(0, 32, 7):
+                for c in range(0, 32, 5):
+                    code = O.e4m3_encode(np.array([tile[r, c] / 2.0 ** e]))[0]
+                    assert q[32 * i + r, 32 * j + c] == code
+
+
+def test_32x32_scale_is_max_of_rowwise_scales():
+    w = S.bf16_bits(S.normal_bf16((128, 256), 1.0, seed=6))
+    _, st = O.cast_32x32(w)
+    _, s0 = O.cast_dim0(w)
+    assert np.array_equal(st, s0.reshape(4, 32, 8).max(axis=1))
+    s_fwd, s_dgrad = O.w32_scale_views(st)
+    assert s_fwd.shape == (128, 8) and s_dgrad.shape == (256, 4)
+    assert s_fwd[37, 5] == st[1, 5] and s_dgrad[200, 3] == st[3, 6]
+
+
+# ------------------------------------------------------------- swizzle -----
+def test_blocked_offsets_golden():
+    for r, c, C, off in _golden_rows("blocked_offsets.txt"):
+        assert O.blocked_offset(int(r), int(c), int(C)) == int(off)
+
+
+@pytest.mark.parametrize("R,C", [(128, 4), (256, 8), (300, 18), (16384 // 64, 18), (1, 1), (129, 5)])
+def test_swizzle_is_a_bijection_onto_non_pad_bytes(R, C):
+    rng = np.random.default_rng(R * 100 + C)
+    s = rng.integers(1, 255, (R, C), dtype=np.uint8)
+    buf = O.swizzle(s)
+    assert buf.size == O.ceil_to(R, 128) * O.ceil_to(C, 4)
+    assert np.array_equal(O.unswizzle(buf, R, C), s)
+    rr, cc = np.indices((R, C))
+    offs = O.blocked_offset(rr, cc, C).ravel()
+    assert len(np.unique(offs)) == R * C
+    assert np.count_nonzero(buf) == R * C               # pads stay 0x00
+
+
+# ----------------------------------------------------------- pad path ------
+def test_group_padding_offsets():
+    offs = np.array([100, 100, 356, 357])
+    p = O.padded_group_starts(offs)
+    assert p.tolist() == [0, 128, 128, 384, 512]
+    assert O.padded_rows_capacity(357, 4) >= p[-1]
+    sizes = S.zipf_group_sizes(32, 32768, 1.2, 3, 0)
+    cap = O.padded_rows_capacity(32768, 32)
+    assert O.padded_group_starts(np.cumsum(sizes))[-1] <= cap
+
+
+def test_grouped_dim0_places_rows_and_zero_pads():
+    x = S.bf16_bits(S.normal_bf16((300, 64), seed=7))
+    offs = np.array([100, 100, 250, 300])
+    cap = O.padded_rows_capacity(300, 4)
+    q, s = O.cast_dim0_grouped(x, offs, cap)
+    p = O.padded_group_starts(offs)
+    starts, ends = O.group_bounds(offs)
+    for g in range(4):
+        n = ends[g] - starts[g]
+        qg, sg = O.cast_dim0(x[starts[g]:ends[g]]) if n else (None, None)
+        if n:
+            assert np.array_equal(q[p[g]:p[g] + n], qg)
+            assert np.array_equal(s[p[g]:p[g] + n], sg)
+    mask = np.ones(cap, bool)
+    for g in range(4):
+        mask[p[g]:p[g] + ends[g] - starts[g]] = False
+    assert not q[mask].any() and not s[mask].any()
+
+
+def test_grouped_dim1_aligned_equals_global_dim1():
+    x = S.bf16_bits(S.normal_bf16((512, 64), seed=8))
+    offs = np.array([128, 384, 384, 512])
+    qt, st = O.cast_dim1_grouped(x, offs, 512)
+    q1, s1 = O.cast_dim1(x)
+    assert np.array_equal(qt, q1) and np.array_equal(st, s1)
+
+
+def test_grouped_dim1_blocks_restart_at_group_start():
+    x = S.bf16_bits(S.normal_bf16((70, 32), seed=9))
+    offs = np.array([40, 70])
+    qt, st = O.cast_dim1_grouped(x, offs, 256)
+    # group 0: tokens 0..39 at columns 0..39 -> blocks [0,32) and [32,40)+zeros
+    assert np.array_equal(qt[:, :32], O.cast_dim1(x[:32])[0])
+    xb = np.zeros((32, 32), np.uint16)
+    xb[:8] = x[32:40]
+    assert np.array_equal(qt[:, 32:64], O.cast_dim1(xb)[0])
+    # group 1 starts at padded column 128
+    xb = np.zeros((32, 32), np.uint16)
+    xb[:30] = x[40:70]
+    assert np.array_equal(qt[:, 128:160], O.cast_dim1(xb)[0])
+    assert not qt[:, 64:128].any() and not st[:, 2:4].any()
+
+
+# --------------------------------------------------------------- GEMMs -----
+def _loop_mm(a, b):
+    out = np.zeros((a.shape[0], b.shape[0]))
+    for i in range(a.shape[0]):
+        for j in range(b.shape[0]):
+            acc = 0.0
+            for k in range(a.shape[1]):
+                acc += a[i, k] * b[j, k]
+            out[i, j] = acc
+    return out
+
+
+def test_grouped_mm_m_equals_loop_of_dense():
+    rng = np.random.default_rng(11)
+    offs = np.array([3, 3, 9])
+    cap = O.padded_rows_capacity(9, 3)
+    a = np.zeros((cap, 4))
+    p = O.padded_group_starts(offs)
+    x = rng.standard_normal((9, 4))
+    a[p[0]:p[0] + 3] = x[0:3]
+    a[p[2]:p[2] + 6] = x[3:9]
+    b = rng.standard_normal((3, 5, 4))
+    y = O.grouped_mm_m(a, b, offs)
+    assert np.allclose(y[0:3], _loop_mm(x[0:3], b[0]))
+    assert np.allclose(y[3:9], _loop_mm(x[3:9], b[2]))
+
+
+def test_grouped_mm_k_equals_loop_and_empty_groups_are_zero():
+    rng = np.random.default_rng(12)
+    offs = np.array([5, 5, 12])
+    p = O.padded_group_starts(offs)
+    a = np.zeros((3, 384))
+    b = np.zeros((4, 384))
+    da = rng.standard_normal((3, 12))
+    db = rng.standard_normal((4, 12))
+    a[:, p[0]:p[0] + 5], b[:, p[0]:p[0] + 5] = da[:, :5], db[:, :5]
+    a[:, p[2]:p[2] + 7], b[:, p[2]:p[2] + 7] = da[:, 5:], db[:, 5:]
+    d = O.grouped_mm_k(a, b, offs)
+    assert np.allclose(d[0], _loop_mm(da[:, :5], db[:, :5]))
+    assert np.all(d[1] == 0.0)
+    assert np.allclose(d[2], _loop_mm(da[:, 5:], db[:, 5:]))
+
+
+def test_one_group_equals_dense_linear():
+    x, w, _ = S.linear_problem(128, 64, 96, seed=2)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    y, _ = O.linear_fwd(xb, wb)
+    qx, sx = O.cast_dim0_grouped(xb, np.array([128]), 128)
+    qw, st = O.cast_32x32(wb[None])
+    s_fwd, _ = O.w32_scale_views(st)
+    yg = O.grouped_mm_m(O.dequant(qx, sx), O.dequant(qw, s_fwd), np.array([128]))
+    assert np.array_equal(y, yg)
+
+
+def test_linear_grads_match_float64_definition_within_mx_error():
+    x, w, dy = S.linear_problem(64, 64, 96, seed=4)
+    xb, wb, db = (S.bf16_bits(t) for t in (x, w, dy))
+    xf, wf, df = (O.bf16_to_f64(t) for t in (xb, wb, db))
+    for (got, _), ref in ((O.linear_fwd(xb, wb), xf @ wf.T),
+                          (O.linear_dgrad(db, wb), df @ wf),
+                          (O.linear_wgrad(db, xb), df.T @ xf)):
+        # E4M3 keeps 3 mantissa bits: each operand is within 2^-4 relative per
+        # element, so the product's relative Frobenius error stays well below 5%.
+        assert got.shape == ref.shape and np.all(np.isfinite(got))
+        rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert rel < 0.05, rel
+
+
+# ---------------------------------------------------- planted mistakes -----
+def test_planted_tie_rule_is_caught(monkeypatch):
+    """A round-half-away encoder (a plausible slip) fails the torch pin."""
+    def half_away(v):
+        v = np.asarray(v, np.float64)
+        a = np.minimum(np.abs(v), 448.0)
+        d = np.abs(O._POS_VALUES[None, :] - a[:, None])
+        code = len(O._POS_VALUES) - 1 - np.argmin(d[:, ::-1], axis=1)   # ties -> larger
+        return (code | (np.signbit(v).astype(np.int64) << 7)).astype(np.uint8)
+    monkeypatch.setattr(O, "e4m3_encode", half_away)
+    with pytest.raises(AssertionError):
+        test_e4m3_encode_matches_torch_exhaustive_bf16(127)
+
+
+def test_planted_swizzle_slip_is_caught(monkeypatch):
+    """Swapping the two in-tile strides (16 and 4) fails the golden offsets."""
+    real = O.blocked_offset
+
+    def wrong(r, c, cols):
+        r = np.asarray(r)
+        rr = r % 128
+        return real(r, c, cols) - (rr % 32) * 16 - (rr // 32) * 4 + (rr % 32) * 4 + (rr // 32) * 16
+    monkeypatch.setattr(O, "blocked_offset", wrong)
+    with pytest.raises(AssertionError):
+        test_blocked_offsets_golden()
