@@ -1,0 +1,152 @@
+/*
+ * mx.h -- C ABI of libmx, the sm_100a (B200) MXFP8 training hot path.
+ *
+ * Operations (sources: five public pull-request pages on MXFP8 training):
+ *   - block-32 casts of bf16 tensors to FP8 E4M3 elements with one E8M0
+ *     power-of-two scale per 32 elements under the RCEIL rule ("shared RCEIL
+ *     constant", torchtitan PR #5334, description): rowwise 1x32 ("dim0"),
+ *     columnwise 32x1 ("dim1", ao "[moe training] Add backward_override to
+ *     the MXFP8 grouped GEMM", Summary and Design notes), the fused
+ *     rowwise+columnwise cast and 32x32 weight blocks (torchtitan PR #5334,
+ *     description); scales are written straight into the blocked layout the
+ *     block-scaled MMA reads ("no need for scale rearrangements since swizzled
+ *     layouts are directly output", same page);
+ *   - the group pad path ("pad_token_groups_for_grouped_mm", ao
+ *     backward_override PR, Known follow-ups; "pad/unpad" and "M-groups /
+ *     K-groups scale rearrange" kernels, ao PR #4705 stack list);
+ *   - the MXFP8 scaled grouped GEMM over an offsets array and its dgrad and
+ *     wgrad (ao backward_override PR, Summary; ao PR #4705, description);
+ *   - the MXFP8 linear forward / dgrad / wgrad (ao PR #4705, "MXFP8Linear
+ *     training paths") and a per-weight quantization cache keyed by the
+ *     weight's version counter ("Cache quantized weights for full AC",
+ *     prime-rl PR #3388, Overview).
+ *
+ * Conventions shared by every entry point
+ *   - All pointers except host-side handles are DEVICE pointers owned by the
+ *     caller; they must be 16-byte aligned (MX_ERR_ALIGN otherwise). Tensors
+ *     are dense row-major with the last dimension contiguous; a strided or
+ *     stride-0 view must be made contiguous by the caller first.
+ *   - bf16 inputs are raw 16-bit bf16 values; E4M3 outputs are one byte per
+ *     element ("fn" encoding: bias 7, max 448, no infinities); E8M0 scale
+ *     bytes are b with value 2^(b-127).
+ *   - Scale buffers use the blocked layout: a logical scale matrix S[R, C] is
+ *     padded to R' = ceil(R/128)*128 rows and C' = ceil(C/4)*4 columns and
+ *     stored as 128x4 tiles of 512 bytes, tile (r/128, c/4) at index
+ *     (r/128)*(C'/4) + c/4, byte (r%32)*16 + ((r%128)/32)*4 + c%4 inside the
+ *     tile. Pad bytes are written as 0x00. mx_scale_bytes() gives the size.
+ *   - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream). Argument errors are detected on the host
+ *     before any launch and leave every buffer untouched. Errors found on the
+ *     device (bad offsets, a pipeline wait that timed out) set a sticky device
+ *     flag that mx_device_error() reads.
+ *   - Nothing here allocates device memory except the weight cache, which owns
+ *     the buffers it creates and frees them in mx_wcache_clear/destroy.
+ *   - Non-finite inputs are outside the contract (their outputs are
+ *     unspecified but the kernels stay in bounds).
+ */
+#ifndef MX_H_
+#define MX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MX_API __attribute__((visibility("default")))
+#else
+#define MX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MX_OK = 0,
+  MX_ERR_ARG = 1,          /* a size, count or pointer is invalid             */
+  MX_ERR_ALIGN = 2,        /* a pointer is not 16-byte aligned                */
+  MX_ERR_UNSUPPORTED = 3,  /* a geometry this library does not handle         */
+  MX_ERR_CUDA = 4,         /* a CUDA runtime call failed                      */
+  MX_ERR_TIMEOUT = 5,      /* a device-side pipeline wait gave up             */
+  MX_ERR_DEVICE = 6        /* the device flagged invalid data (e.g. offsets)  */
+} mx_status;
+
+/* Human-readable reason of the last non-MX_OK status returned on this host
+ * thread (empty string if none). The pointer stays valid until the next call. */
+MX_API const char* mx_last_error(void);
+
+/* Bytes of the blocked layout of a logical scale matrix S[rows, cols]:
+ * ceil(rows/128)*128 * ceil(cols/4)*4. */
+MX_API size_t mx_scale_bytes(int64_t rows, int64_t cols);
+
+/* Upper bound of the padded row count of M tokens in `groups` groups when
+ * every group is rounded up to a multiple of 128 rows:
+ * floor((M + 127*groups) / 128) * 128. */
+MX_API int64_t mx_padded_rows_capacity(int64_t m_total, int32_t groups);
+
+/* Synchronizes `stream`, then returns MX_OK, MX_ERR_TIMEOUT or MX_ERR_DEVICE
+ * according to the sticky device flag, and clears the flag. */
+MX_API mx_status mx_device_error(void* stream);
+
+/* ---------------------------------------------------------------- casts --
+ * dim0 (rowwise, 1x32 along the contiguous axis; ao backward_override PR,
+ * Design notes, "CuTe DSL 1x32 kernel"):
+ *   x  bf16 [R, C]          q  E4M3 [R, C]          s  blocked(R, C/32)
+ * R >= 0, C a positive multiple of 32. */
+MX_API mx_status mx_cast_dim0(const void* x, int64_t R, int64_t C,
+                       void* q, void* s, void* stream);
+
+/* dim1 (columnwise, 32x1 down each column, stored transposed so that the
+ * reduced axis is contiguous; ao backward_override PR, Summary, "dim1 cast"):
+ *   x  bf16 [R, C]          qt E4M3 [C, R]          st blocked(C, R/32)
+ * R a multiple of 32, C a positive multiple of 32. */
+MX_API mx_status mx_cast_dim1(const void* x, int64_t R, int64_t C,
+                       void* qt, void* st, void* stream);
+
+/* Fused rowwise + columnwise cast from one read of x (torchtitan PR #5334,
+ * description, "fused dense rowwise/columnwise cast"). Outputs are bitwise
+ * those of mx_cast_dim0 and mx_cast_dim1. Same size rules as mx_cast_dim1. */
+MX_API mx_status mx_cast_2d(const void* x, int64_t R, int64_t C,
+                     void* q, void* s, void* qt, void* st, void* stream);
+
+/* 32x32 weight cast (one scale per 32x32 tile; torchtitan PR #5334,
+ * description and review thread, "32x32 RCEIL weight-scale policy"), for a
+ * stack of G weights w bf16 [G, N, K] (G = 1 for a dense weight):
+ *   q        E4M3 [G, N, K]
+ *   s_fwd    G concatenated blocked(N, K/32) buffers, S_fwd[n, kb] = S[n/32, kb]
+ *   qt       E4M3 [G, K, N] (the same codes transposed) or NULL
+ *   s_dgrad  G concatenated blocked(K, N/32) buffers, S_dgrad[k, nb] = S[nb, k/32],
+ *            or NULL
+ * N and K positive multiples of 32. */
+MX_API mx_status mx_cast_w32x32(const void* w, int64_t G, int64_t N, int64_t K,
+                         void* q, void* s_fwd, void* qt, void* s_dgrad,
+                         void* stream);
+
+/* ------------------------------------------------------- group pad path --
+ * offs: device int32 [G] cumulative group ends (non-decreasing, offs[G-1] ==
+ * M). Group g occupies rows offs[g-1]..offs[g] of x (offs[-1] = 0) and is
+ * placed at padded row p_g = sum_{h<g} ceil(size_h/128)*128. m_cap is the
+ * row capacity of the padded outputs: a multiple of 128 that is at least the
+ * padded total (mx_padded_rows_capacity() always is). Pad rows/tokens are
+ * written as code 0 with scale byte 0. Offsets are read on the device only;
+ * invalid ones set the device flag (MX_ERR_DEVICE). 1 <= G <= 1024.
+ *
+ * dim0 into padded rows:   x bf16 [M, K] -> q [m_cap, K], s blocked(m_cap, K/32)
+ * dim1 per group (32-token blocks start at each group start, a group's last
+ * partial block is completed with zeros):
+ *                          x bf16 [M, K] -> qt [K, m_cap], st blocked(K, m_cap/32)
+ * 2d: both from one read.  K a positive multiple of 32. */
+MX_API mx_status mx_cast_dim0_grouped(const void* x, int64_t M, int64_t K,
+                               const int32_t* offs, int32_t G, int64_t m_cap,
+                               void* q, void* s, void* stream);
+MX_API mx_status mx_cast_dim1_grouped(const void* x, int64_t M, int64_t K,
+                               const int32_t* offs, int32_t G, int64_t m_cap,
+                               void* qt, void* st, void* stream);
+MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
+                             const int32_t* offs, int32_t G, int64_t m_cap,
+                             void* q, void* s, void* qt, void* st, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MX_H_ */

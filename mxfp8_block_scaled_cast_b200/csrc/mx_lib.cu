@@ -1,0 +1,246 @@
+// libmx: the C ABI declared in include/mx.h.
+//
+// This single translation unit holds every kernel of the library (casts,
+// the tcgen05 grouped GEMM, the linear and its weight cache) so that they
+// share the sticky device error flag without relocatable device code.
+// Host functions validate every argument before any launch and report the
+// reason of a failure through mx_last_error().
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "mx_common.cuh"
+#include "mx_cast.cuh"
+
+namespace mx {
+namespace {
+
+thread_local char g_err[512] = "";
+
+mx_status fail(mx_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mx_status cuda_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MX_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MX_OK;
+}
+
+#define MX_REQUIRE(cond, st, ...) \
+  do {                            \
+    if (!(cond)) return fail(st, __VA_ARGS__); \
+  } while (0)
+
+template <int kMode, bool kGrouped>
+mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
+                      cudaStream_t stream) {
+  if (col_tiles == 0 || row_tiles == 0 || depth == 0) return MX_OK;
+  MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth <= 65535, MX_ERR_UNSUPPORTED,
+             "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles,
+             (long long)row_tiles, (long long)depth);
+  const bool colpass = (kMode & kModeCol) || ((kMode & kModeSquare) && a.qt != nullptr);
+  const size_t smem = colpass ? size_t(kXsBytes + kQsBytes) : 0;
+  if (smem > 0) {
+    cudaError_t e = cudaFuncSetAttribute(cast_tile_kernel<kMode, kGrouped>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return fail(MX_ERR_CUDA, "cast smem attribute: %s", cudaGetErrorString(e));
+  }
+  cast_tile_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)),
+                                       kCastThreads, smem, stream>>>(a);
+  return cuda_check("cast launch");
+}
+
+CastArgs make_args(const void* x, int64_t rows_src, int64_t C, int64_t rows_out) {
+  CastArgs a;
+  memset(&a, 0, sizeof(a));
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows_src = rows_src;
+  a.C = C;
+  a.rows_out = rows_out;
+  return a;
+}
+
+mx_status check_cast_geometry(const void* x, int64_t R, int64_t C, bool rows_blocked) {
+  MX_REQUIRE(R >= 0 && C > 0, MX_ERR_ARG, "sizes must be R >= 0, C > 0 (got %lld, %lld)", (long long)R,
+             (long long)C);
+  MX_REQUIRE(C % kBlock == 0, MX_ERR_UNSUPPORTED, "C = %lld is not a multiple of 32", (long long)C);
+  MX_REQUIRE(!rows_blocked || R % kBlock == 0, MX_ERR_UNSUPPORTED,
+             "R = %lld is not a multiple of 32 (columnwise blocks)", (long long)R);
+  MX_REQUIRE(R == 0 || x != nullptr, MX_ERR_ARG, "null input");
+  MX_REQUIRE(aligned16(x), MX_ERR_ALIGN, "input not 16-byte aligned");
+  return MX_OK;
+}
+
+mx_status check_out(const void* p, bool needed, const char* name) {
+  MX_REQUIRE(!needed || p != nullptr, MX_ERR_ARG, "null output %s", name);
+  MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "output %s not 16-byte aligned", name);
+  return MX_OK;
+}
+
+#define MX_TRY(expr)              \
+  do {                            \
+    mx_status st_ = (expr);       \
+    if (st_ != MX_OK) return st_; \
+  } while (0)
+
+mx_status check_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                        int64_t m_cap) {
+  MX_REQUIRE(M >= 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, K > 0");
+  MX_REQUIRE(K % kBlock == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 32", (long long)K);
+  MX_REQUIRE(G >= 1 && G <= kMaxGroups, MX_ERR_ARG, "G = %d outside [1, %d]", G, kMaxGroups);
+  MX_REQUIRE(offs != nullptr, MX_ERR_ARG, "null offsets");
+  MX_REQUIRE((reinterpret_cast<uintptr_t>(offs) & 3u) == 0, MX_ERR_ALIGN, "offsets not 4-byte aligned");
+  MX_REQUIRE(m_cap >= M && m_cap % 128 == 0, MX_ERR_ARG,
+             "m_cap = %lld must be a multiple of 128 and >= M = %lld", (long long)m_cap, (long long)M);
+  MX_REQUIRE(M == 0 || x != nullptr, MX_ERR_ARG, "null input");
+  MX_REQUIRE(aligned16(x), MX_ERR_ALIGN, "input not 16-byte aligned");
+  return MX_OK;
+}
+
+}  // namespace
+}  // namespace mx
+
+using namespace mx;
+
+extern "C" {
+
+const char* mx_last_error(void) { return g_err; }
+
+size_t mx_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return size_t(scale_bytes(rows, cols));
+}
+
+int64_t mx_padded_rows_capacity(int64_t m_total, int32_t groups) {
+  if (m_total < 0 || groups < 0) return -1;
+  return ((m_total + 127ll * groups) / 128) * 128;
+}
+
+mx_status mx_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MX_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  unsigned v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(MX_ERR_CUDA, "device flag: %s", cudaGetErrorString(e));
+  if (v & kErrTimeout) return fail(MX_ERR_TIMEOUT, "a device pipeline wait timed out");
+  if (v & kErrOffsets) return fail(MX_ERR_DEVICE, "invalid group offsets seen on the device");
+  g_err[0] = '\0';
+  return MX_OK;
+}
+
+mx_status mx_cast_dim0(const void* x, int64_t R, int64_t C, void* q, void* s, void* stream) {
+  MX_TRY(check_cast_geometry(x, R, C, false));
+  MX_TRY(check_out(q, R > 0, "q"));
+  MX_TRY(check_out(s, R > 0, "s"));
+  CastArgs a = make_args(x, R, C, R);
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s);
+  return launch_cast<kModeRow, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_dim1(const void* x, int64_t R, int64_t C, void* qt, void* st, void* stream) {
+  MX_TRY(check_cast_geometry(x, R, C, true));
+  MX_TRY(check_out(qt, R > 0, "qt"));
+  MX_TRY(check_out(st, R > 0, "st"));
+  CastArgs a = make_args(x, R, C, R);
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(st);
+  return launch_cast<kModeCol, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_2d(const void* x, int64_t R, int64_t C, void* q, void* s, void* qt, void* st,
+                     void* stream) {
+  MX_TRY(check_cast_geometry(x, R, C, true));
+  MX_TRY(check_out(q, R > 0, "q"));
+  MX_TRY(check_out(s, R > 0, "s"));
+  MX_TRY(check_out(qt, R > 0, "qt"));
+  MX_TRY(check_out(st, R > 0, "st"));
+  CastArgs a = make_args(x, R, C, R);
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s);
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(st);
+  return launch_cast<kModeRowCol, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
+                                         static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_w32x32(const void* w, int64_t G, int64_t N, int64_t K, void* q, void* s_fwd, void* qt,
+                         void* s_dgrad, void* stream) {
+  MX_REQUIRE(G >= 0, MX_ERR_ARG, "G must be >= 0");
+  MX_TRY(check_cast_geometry(w, N, K, true));
+  MX_REQUIRE(N > 0, MX_ERR_ARG, "N must be > 0");
+  MX_TRY(check_out(q, G > 0, "q"));
+  MX_TRY(check_out(s_fwd, G > 0, "s_fwd"));
+  MX_TRY(check_out(qt, false, "qt"));
+  MX_TRY(check_out(s_dgrad, false, "s_dgrad"));
+  CastArgs a = make_args(w, N, K, N);
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s_fwd);
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(s_dgrad);
+  a.x_stride = N * K;
+  a.q_stride = N * K;
+  a.qt_stride = N * K;
+  a.s_stride = scale_bytes(N, K / kBlock);
+  a.st_stride = scale_bytes(K, N / kBlock);
+  return launch_cast<kModeSquare, false>(a, ceil_div(K, kCastTile), ceil_div(N, kCastTile), G,
+                                         static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_dim0_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                               int64_t m_cap, void* q, void* s, void* stream) {
+  MX_TRY(check_grouped(x, M, K, offs, G, m_cap));
+  MX_TRY(check_out(q, m_cap > 0, "q"));
+  MX_TRY(check_out(s, m_cap > 0, "s"));
+  CastArgs a = make_args(x, M, K, m_cap);
+  a.offs = offs;
+  a.G = G;
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s);
+  return launch_cast<kModeRow, true>(a, ceil_div(K, kCastTile), m_cap / kCastTile, 1,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_dim1_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                               int64_t m_cap, void* qt, void* st, void* stream) {
+  MX_TRY(check_grouped(x, M, K, offs, G, m_cap));
+  MX_TRY(check_out(qt, m_cap > 0, "qt"));
+  MX_TRY(check_out(st, m_cap > 0, "st"));
+  CastArgs a = make_args(x, M, K, m_cap);
+  a.offs = offs;
+  a.G = G;
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(st);
+  return launch_cast<kModeCol, true>(a, ceil_div(K, kCastTile), m_cap / kCastTile, 1,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                             int64_t m_cap, void* q, void* s, void* qt, void* st, void* stream) {
+  MX_TRY(check_grouped(x, M, K, offs, G, m_cap));
+  MX_TRY(check_out(q, m_cap > 0, "q"));
+  MX_TRY(check_out(s, m_cap > 0, "s"));
+  MX_TRY(check_out(qt, m_cap > 0, "qt"));
+  MX_TRY(check_out(st, m_cap > 0, "st"));
+  CastArgs a = make_args(x, M, K, m_cap);
+  a.offs = offs;
+  a.G = G;
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s);
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(st);
+  return launch_cast<kModeRowCol, true>(a, ceil_div(K, kCastTile), m_cap / kCastTile, 1,
+                                        static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

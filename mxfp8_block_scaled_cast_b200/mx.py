@@ -1,0 +1,212 @@
+"""Thin ctypes binding of libmx (include/mx.h).
+
+Argument marshalling only: every function named ``mx_*`` here passes device
+pointers of caller-owned torch tensors, sizes and the current CUDA stream to
+the C entry point of the same name and raises ``MXError`` on a non-zero
+status. The convenience wrappers (``cast_dim0`` ...) only allocate the output
+tensors with torch and call those. No computation happens in Python and there
+is no fallback: if libmx.so is missing or no GPU is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmx.so")
+
+_vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+
+# name -> (restype, argtypes); the table mirrors include/mx.h
+_SIGNATURES = {
+    "mx_last_error": (ctypes.c_char_p, []),
+    "mx_scale_bytes": (_sz, [_i64, _i64]),
+    "mx_padded_rows_capacity": (_i64, [_i64, _i32]),
+    "mx_device_error": (ctypes.c_int, [_vp]),
+    "mx_cast_dim0": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "mx_cast_dim1": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "mx_cast_2d": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "mx_cast_w32x32": (ctypes.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "mx_cast_dim0_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
+    "mx_cast_dim1_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
+    "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
+}
+
+_lib = None
+
+
+class MXError(RuntimeError):
+    def __init__(self, name, status, detail):
+        super().__init__(f"{name} failed with status {status}: {detail}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmx (loaded once; raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mxfp8_block_scaled_cast_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def exported_names():
+    return list(_SIGNATURES)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmx takes device tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libmx takes contiguous tensors only (call .contiguous() first)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _call(name, *args):
+    status = getattr(lib(), name)(*args)
+    if status != 0:
+        raise MXError(name, status, lib().mx_last_error().decode())
+
+
+# ------------------------------------------------------------ raw entries --
+def mx_scale_bytes(rows, cols) -> int:
+    return int(lib().mx_scale_bytes(rows, cols))
+
+
+def mx_padded_rows_capacity(m_total, groups) -> int:
+    return int(lib().mx_padded_rows_capacity(m_total, groups))
+
+
+def mx_device_error(stream=None):
+    _call("mx_device_error", _stream(stream))
+
+
+def mx_cast_dim0(x, q, s, stream=None):
+    R, C = x.shape
+    _call("mx_cast_dim0", _p(x), R, C, _p(q), _p(s), _stream(stream))
+
+
+def mx_cast_dim1(x, qt, st, stream=None):
+    R, C = x.shape
+    _call("mx_cast_dim1", _p(x), R, C, _p(qt), _p(st), _stream(stream))
+
+
+def mx_cast_2d(x, q, s, qt, st, stream=None):
+    R, C = x.shape
+    _call("mx_cast_2d", _p(x), R, C, _p(q), _p(s), _p(qt), _p(st), _stream(stream))
+
+
+def mx_cast_w32x32(w, q, s_fwd, qt=None, s_dgrad=None, stream=None):
+    G, N, K = w.shape if w.dim() == 3 else (1, *w.shape)
+    _call("mx_cast_w32x32", _p(w), G, N, K, _p(q), _p(s_fwd), _p(qt), _p(s_dgrad), _stream(stream))
+
+
+def mx_cast_dim0_grouped(x, offs, m_cap, q, s, stream=None):
+    M, K = x.shape
+    _call("mx_cast_dim0_grouped", _p(x), M, K, _p(offs), offs.numel(), m_cap, _p(q), _p(s),
+          _stream(stream))
+
+
+def mx_cast_dim1_grouped(x, offs, m_cap, qt, st, stream=None):
+    M, K = x.shape
+    _call("mx_cast_dim1_grouped", _p(x), M, K, _p(offs), offs.numel(), m_cap, _p(qt), _p(st),
+          _stream(stream))
+
+
+def mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st, stream=None):
+    M, K = x.shape
+    _call("mx_cast_2d_grouped", _p(x), M, K, _p(offs), offs.numel(), m_cap, _p(q), _p(s), _p(qt),
+          _p(st), _stream(stream))
+
+
+# --------------------------------------------------- allocating wrappers --
+def _u8(*shape, device):
+    return torch.empty(*shape, dtype=torch.uint8, device=device)
+
+
+def _check_bf16(x):
+    if x.dtype != torch.bfloat16:
+        raise TypeError("libmx casts take bf16 input")
+    return x.contiguous()
+
+
+def cast_dim0(x):
+    x = _check_bf16(x)
+    R, C = x.shape
+    q, s = _u8(R, C, device=x.device), _u8(mx_scale_bytes(R, C // 32), device=x.device)
+    mx_cast_dim0(x, q, s)
+    return q, s
+
+
+def cast_dim1(x):
+    x = _check_bf16(x)
+    R, C = x.shape
+    qt, st = _u8(C, R, device=x.device), _u8(mx_scale_bytes(C, R // 32), device=x.device)
+    mx_cast_dim1(x, qt, st)
+    return qt, st
+
+
+def cast_2d(x):
+    x = _check_bf16(x)
+    R, C = x.shape
+    q, s = _u8(R, C, device=x.device), _u8(mx_scale_bytes(R, C // 32), device=x.device)
+    qt, st = _u8(C, R, device=x.device), _u8(mx_scale_bytes(C, R // 32), device=x.device)
+    mx_cast_2d(x, q, s, qt, st)
+    return q, s, qt, st
+
+
+def cast_w32x32(w, transposed=True):
+    w = _check_bf16(w)
+    G, N, K = w.shape if w.dim() == 3 else (1, *w.shape)
+    dev = w.device
+    q = _u8(*w.shape, device=dev)
+    s_fwd = _u8(G * mx_scale_bytes(N, K // 32), device=dev)
+    qt = _u8(*((G, K, N) if w.dim() == 3 else (K, N)), device=dev) if transposed else None
+    s_dgrad = _u8(G * mx_scale_bytes(K, N // 32), device=dev) if transposed else None
+    mx_cast_w32x32(w, q, s_fwd, qt, s_dgrad)
+    return q, s_fwd, qt, s_dgrad
+
+
+def cast_dim0_grouped(x, offs, m_cap=None):
+    x = _check_bf16(x)
+    M, K = x.shape
+    m_cap = mx_padded_rows_capacity(M, offs.numel()) if m_cap is None else m_cap
+    q, s = _u8(m_cap, K, device=x.device), _u8(mx_scale_bytes(m_cap, K // 32), device=x.device)
+    mx_cast_dim0_grouped(x, offs, m_cap, q, s)
+    return q, s
+
+
+def cast_dim1_grouped(x, offs, m_cap=None):
+    x = _check_bf16(x)
+    M, K = x.shape
+    m_cap = mx_padded_rows_capacity(M, offs.numel()) if m_cap is None else m_cap
+    qt, st = _u8(K, m_cap, device=x.device), _u8(mx_scale_bytes(K, m_cap // 32), device=x.device)
+    mx_cast_dim1_grouped(x, offs, m_cap, qt, st)
+    return qt, st
+
+
+def cast_2d_grouped(x, offs, m_cap=None):
+    x = _check_bf16(x)
+    M, K = x.shape
+    m_cap = mx_padded_rows_capacity(M, offs.numel()) if m_cap is None else m_cap
+    dev = x.device
+    q, s = _u8(m_cap, K, device=dev), _u8(mx_scale_bytes(m_cap, K // 32), device=dev)
+    qt, st = _u8(K, m_cap, device=dev), _u8(mx_scale_bytes(K, m_cap // 32), device=dev)
+    mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st)
+    return q, s, qt, st
