@@ -145,6 +145,38 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
                              const int32_t* offs, int32_t G, int64_t m_cap,
                              void* q, void* s, void* qt, void* st, void* stream);
 
+/* -------------------------------------------------- scaled grouped GEMM --
+ * The MXFP8 scaled grouped GEMM over an offsets array (ao "[moe training]
+ * Add backward_override to the MXFP8 grouped GEMM", Summary: forward, dgrad
+ * and wgrad of the grouped GEMM; ao PR #4705, "MXFP8 MoE grouped-mm").
+ * Operands are E4M3 codes with blocked E8M0 scales, both K-major (the
+ * contraction axis contiguous), as the casts above produce them. fp32
+ * accumulation on the tensor cores, bf16 output (round to nearest even).
+ * Deterministic: no split-K, no atomics.
+ *
+ * mode MX_GROUPS_M (forward and dgrad; groups split the rows):
+ *   out[start_g + i, :] = sum_k A[p_g + i, k] B[g, :, k]   for i < size_g
+ *   a_q [rows_a, K], a_s blocked(rows_a, K/32)   rows_a = m_cap (padded rows
+ *       from mx_cast_dim0_grouped) or M when offs == NULL (dense, G = 1)
+ *   b_q [G, N, K],   b_s G concatenated blocked(N, K/32) buffers
+ *   out bf16 [M, N]; rows of the padded layout that are padding are not read
+ *       into the output (the unpad is fused into the store).
+ *   N a multiple of 256, K a multiple of 128.
+ * mode MX_GROUPS_K (wgrad; groups split the contraction, "K groups"):
+ *   out[g, n, k] = sum over the tokens t of group g of A[n, t] B[k, t]
+ *   a_q [N, L], a_s blocked(N, L/32); b_q [K, L], b_s blocked(K, L/32) with
+ *       L = m_cap (padded token columns from mx_cast_dim1_grouped) or M when
+ *       offs == NULL (dense, G = 1, M a multiple of 32)
+ *   out bf16 [G, N, K]; an empty group gives exact zeros.
+ *   N a multiple of 128, K a multiple of 256.
+ * offs: device int32 [G] cumulative ends (see the pad path above) or NULL.
+ * Invalid offsets set the device flag and leave the output unwritten. */
+#define MX_GROUPS_M 0
+#define MX_GROUPS_K 1
+MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                               const int32_t* offs, int32_t G, int32_t mode, void* out,
+                               int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,8 +9,11 @@
 #include <cstdio>
 #include <cstring>
 
+#include <cudaTypedefs.h>
+
 #include "mx_common.cuh"
 #include "mx_cast.cuh"
+#include "mx_gemm.cuh"
 
 namespace mx {
 namespace {
@@ -102,6 +105,41 @@ mx_status check_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs
   MX_REQUIRE(M == 0 || x != nullptr, MX_ERR_ARG, "null input");
   MX_REQUIRE(aligned16(x), MX_ERR_ALIGN, "input not 16-byte aligned");
   return MX_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D uint8 tensor map over a row-major [outer, inner] byte matrix, box
+// {128, box_outer}, 128-byte swizzle, zero fill outside the tensor.
+mx_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  auto fn = encode_fn();
+  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128u, box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MX_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
 }
 
 }  // namespace
@@ -241,6 +279,83 @@ mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K, const int32_t*
   a.st = static_cast<uint8_t*>(st);
   return launch_cast<kModeRowCol, true>(a, ceil_div(K, kCastTile), m_cap / kCastTile, 1,
                                         static_cast<cudaStream_t>(stream));
+}
+
+mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                        const int32_t* offs, int32_t G, int32_t mode, void* out, int64_t M, int64_t N,
+                        int64_t K, int64_t m_cap, void* stream) {
+  MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K, MX_ERR_ARG, "unknown mode %d", mode);
+  MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
+  if (offs != nullptr) {
+    MX_REQUIRE(G >= 1 && G <= kMaxGroups, MX_ERR_ARG, "G = %d outside [1, %d]", G, kMaxGroups);
+    MX_REQUIRE(m_cap >= M && m_cap % 128 == 0 && m_cap < (1ll << 31), MX_ERR_ARG,
+               "m_cap = %lld must be a multiple of 128, >= M and < 2^31", (long long)m_cap);
+    MX_REQUIRE((reinterpret_cast<uintptr_t>(offs) & 3u) == 0, MX_ERR_ALIGN, "offsets not 4-byte aligned");
+  } else {
+    MX_REQUIRE(G == 1, MX_ERR_ARG, "without offsets G must be 1 (dense)");
+    MX_REQUIRE(M < (1ll << 31), MX_ERR_ARG, "M too large");
+  }
+  const void* ptrs[5] = {a_q, a_s, b_q, b_s, out};
+  for (const void* p : ptrs) MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "operand not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemmArgs ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.a_s = static_cast<const uint8_t*>(a_s);
+  ga.b_s = static_cast<const uint8_t*>(b_s);
+  ga.offs = offs;
+  ga.out = static_cast<__nv_bfloat16*>(out);
+  ga.G = G;
+  ga.M = M;
+  ga.N = N;
+  ga.K = K;
+  CUtensorMap map_a, map_b;
+  int64_t tiles_ub = 0;
+  if (mode == MX_GROUPS_M) {
+    MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
+    MX_REQUIRE(K % kBK == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 128", (long long)K);
+    const int64_t rows_a = offs ? m_cap : M;
+    ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
+    if (rows_a == 0 || M == 0) return MX_OK;
+    MX_REQUIRE(a_q && a_s && b_q && b_s && out, MX_ERR_ARG, "null operand");
+    ga.a_sc_tiles = K / kBK;
+    ga.b_sc_tiles = K / kBK;
+    ga.b_sc_group_stride = scale_bytes(N, K / kBlock);
+    MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kBM));
+    MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN));
+    tiles_ub = ceil_div(rows_a, kBM) * (N / kBN);
+  } else {
+    MX_REQUIRE(N % kBM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 128", (long long)N);
+    MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
+    MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
+    const int64_t len = offs ? m_cap : M;
+    MX_REQUIRE(offs || M % kBlock == 0, MX_ERR_UNSUPPORTED, "dense K-groups needs M %% 32 == 0");
+    ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
+    if (len == 0) {
+      cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
+      MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+      return MX_OK;
+    }
+    MX_REQUIRE(a_q && a_s && b_q && b_s, MX_ERR_ARG, "null operand");
+    ga.a_sc_tiles = ceil_div(ceil_div(len, kBlock), 4);
+    ga.b_sc_tiles = ga.a_sc_tiles;
+    ga.b_sc_group_stride = 0;
+    MX_TRY(make_map(&map_a, a_q, uint64_t(len), uint64_t(N), kBM));
+    MX_TRY(make_map(&map_b, b_q, uint64_t(len), uint64_t(K), kBN));
+    tiles_ub = int64_t(G) * (N / kBM) * (K / kBN);
+  }
+  const int sms = sm_count();
+  MX_REQUIRE(sms > 0, MX_ERR_CUDA, "no CUDA device");
+  const unsigned grid = unsigned(tiles_ub < sms ? tiles_ub : sms);
+  cudaError_t e;
+  if (mode == MX_GROUPS_M) {
+    e = cudaFuncSetAttribute(mx_gemm_kernel<kGroupsM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+    if (e == cudaSuccess) mx_gemm_kernel<kGroupsM><<<grid, kGemmThreads, kGemmSmem, st>>>(map_a, map_b, ga);
+  } else {
+    e = cudaFuncSetAttribute(mx_gemm_kernel<kGroupsK>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+    if (e == cudaSuccess) mx_gemm_kernel<kGroupsK><<<grid, kGemmThreads, kGemmSmem, st>>>(map_a, map_b, ga);
+  }
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
+  return cuda_check("gemm launch");
 }
 
 }  // extern "C"

@@ -32,7 +32,11 @@ _SIGNATURES = {
     "mx_cast_dim0_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_dim1_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
 }
+
+MX_GROUPS_M = 0
+MX_GROUPS_K = 1
 
 _lib = None
 
@@ -135,6 +139,11 @@ def mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st, stream=None):
           _p(st), _stream(stream))
 
 
+def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream=None):
+    _call("mx_grouped_mm", _p(a_q), _p(a_s), _p(b_q), _p(b_s), _p(offs), G, mode, _p(out), M, N, K,
+          m_cap, _stream(stream))
+
+
 # --------------------------------------------------- allocating wrappers --
 def _u8(*shape, device):
     return torch.empty(*shape, dtype=torch.uint8, device=device)
@@ -210,3 +219,24 @@ def cast_2d_grouped(x, offs, m_cap=None):
     qt, st = _u8(K, m_cap, device=dev), _u8(mx_scale_bytes(K, m_cap // 32), device=dev)
     mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st)
     return q, s, qt, st
+
+
+def grouped_mm(a_q, a_s, b_q, b_s, offs, M, m_cap=None):
+    """M-groups GEMM: out[M, N] bf16 from padded A [rows, K] and experts B [G, N, K]."""
+    G = b_q.shape[0] if b_q.dim() == 3 else 1
+    N, K = b_q.shape[-2], b_q.shape[-1]
+    if offs is not None and m_cap is None:
+        m_cap = a_q.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=a_q.device)
+    mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, MX_GROUPS_M, out, M, N, K, m_cap or 0)
+    return out
+
+
+def grouped_mm_wgrad(a_q, a_s, b_q, b_s, offs, M, G=None):
+    """K-groups GEMM: out[G, N, K] bf16 from A [N, L] and B [K, L] over token groups."""
+    N, L = a_q.shape
+    K = b_q.shape[0]
+    G = (offs.numel() if offs is not None else 1) if G is None else G
+    out = torch.empty(G, N, K, dtype=torch.bfloat16, device=a_q.device)
+    mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, MX_GROUPS_K, out, M, N, K, L if offs is not None else 0)
+    return out
