@@ -177,6 +177,41 @@ MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q
                                const int32_t* offs, int32_t G, int32_t mode, void* out,
                                int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
 
+/* ------------------------------------------------------ MXFP8 linear -----
+ * Dense MXFP8 linear (ao PR #4705, "MXFP8Linear training paths"; torchtitan
+ * PR #5334, "a single API for dense and grouped mxfp8 linears"):
+ *   forward  y  [M, N] = x [M, K] w [N, K]^T   x cast 1x32 (dim0), w 32x32
+ *   backward dx [M, K] = dy [M, N] w           dy cast 1x32 along N
+ *            dw [N, K] = dy^T x                dy and x cast 32x1 along M
+ * dy is cast once by the fused rowwise+columnwise cast. All tensors bf16,
+ * row-major. M a multiple of 32; N and K multiples of 256.
+ * ws: caller-owned device workspace of at least mx_linear_ws_bytes(M, N, K)
+ * bytes (holds the quantized activations and gradients and, without a
+ * cache, the quantized weight); it must stay untouched until the call's
+ * work on `stream` completes.
+ *
+ * Weight cache ("Cache quantized weights for full AC", prime-rl PR #3388,
+ * Overview): with cache != NULL the 32x32 quantization of w is kept in
+ * device memory owned by the cache, keyed by (w address, N, K) and reused
+ * while w_version (the caller's in-place update counter of w) is unchanged;
+ * a changed version re-quantizes in place. Results are bitwise identical
+ * with and without a hit. mx_wcache_clear() frees every entry (call it
+ * after backward; it synchronizes the device). The cache is thread-safe;
+ * an entry must not be cleared while work that reads it is in flight. */
+typedef struct mx_wcache mx_wcache;
+MX_API mx_wcache* mx_wcache_create(void);
+MX_API void mx_wcache_clear(mx_wcache* cache);
+MX_API void mx_wcache_destroy(mx_wcache* cache);
+MX_API mx_status mx_wcache_stats(mx_wcache* cache, int64_t* hits, int64_t* misses, int64_t* entries);
+MX_API size_t mx_linear_ws_bytes(int64_t M, int64_t N, int64_t K);
+MX_API mx_status mx_linear_fwd(const void* x, const void* w, int64_t M, int64_t N, int64_t K,
+                               mx_wcache* cache, uint64_t w_version, void* y,
+                               void* ws, size_t ws_bytes, void* stream);
+MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
+                               int64_t M, int64_t N, int64_t K,
+                               mx_wcache* cache, uint64_t w_version, void* dx, void* dw,
+                               void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,12 +8,14 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <new>
 
 #include <cudaTypedefs.h>
 
 #include "mx_common.cuh"
 #include "mx_cast.cuh"
 #include "mx_gemm.cuh"
+#include "mx_linear.cuh"
 
 namespace mx {
 namespace {
@@ -356,6 +358,136 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
   }
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
   return cuda_check("gemm launch");
+}
+
+mx_wcache* mx_wcache_create(void) { return new (std::nothrow) mx_wcache(); }
+
+void mx_wcache_clear(mx_wcache* c) {
+  if (c == nullptr) return;
+  std::lock_guard<std::mutex> lk(c->mu);
+  for (auto& e : c->entries) cudaFree(e.q);
+  c->entries.clear();
+}
+
+void mx_wcache_destroy(mx_wcache* c) {
+  mx_wcache_clear(c);
+  delete c;
+}
+
+mx_status mx_wcache_stats(mx_wcache* c, int64_t* hits, int64_t* misses, int64_t* entries) {
+  MX_REQUIRE(c != nullptr, MX_ERR_ARG, "null cache");
+  std::lock_guard<std::mutex> lk(c->mu);
+  if (hits) *hits = c->hits;
+  if (misses) *misses = c->misses;
+  if (entries) *entries = int64_t(c->entries.size());
+  return MX_OK;
+}
+
+size_t mx_linear_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N <= 0 || K <= 0) return 0;
+  const int64_t fwd = ceil_to(M * K, 256) + ceil_to(scale_bytes(M, K / kBlock), 256);
+  const int64_t bwd = 2 * ceil_to(M * N, 256) + ceil_to(scale_bytes(M, N / kBlock), 256) +
+                      ceil_to(scale_bytes(N, M / kBlock), 256) + ceil_to(K * M, 256) +
+                      ceil_to(scale_bytes(K, M / kBlock), 256);
+  return size_t((fwd > bwd ? fwd : bwd) + wq_bytes(N, K));
+}
+
+}  // extern "C"
+
+namespace mx {
+namespace {
+
+mx_status check_linear(int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes) {
+  MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
+  MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
+  MX_REQUIRE(N % kBN == 0 && K % kBN == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 256");
+  MX_REQUIRE(ws_bytes >= mx_linear_ws_bytes(M, N, K), MX_ERR_ARG, "workspace too small (%zu < %zu bytes)",
+             ws_bytes, mx_linear_ws_bytes(M, N, K));
+  MX_REQUIRE(ws != nullptr && aligned16(ws), MX_ERR_ALIGN, "workspace null or not 16-byte aligned");
+  return MX_OK;
+}
+
+// The 32x32 quantization of W: from the cache (hit), re-cast into the cache
+// (miss or stale version), or cast into the workspace tail (no cache).
+mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, uint64_t version, uint8_t* ws_tail,
+                       WeightView* out, cudaStream_t st) {
+  if (cache == nullptr) {
+    *out = carve_weight(ws_tail, N, K);
+    return mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, out->qt, out->s_dgrad, st);
+  }
+  std::lock_guard<std::mutex> lk(cache->mu);
+  mx_wcache::Entry* e = nullptr;
+  for (auto& x : cache->entries)
+    if (x.w == w && x.N == N && x.K == K) e = &x;
+  if (e != nullptr && e->valid && e->version == version) {
+    ++cache->hits;
+    *out = carve_weight(e->q, N, K);
+    return MX_OK;
+  }
+  ++cache->misses;
+  if (e == nullptr) {
+    uint8_t* buf = nullptr;
+    cudaError_t err = cudaMalloc(&buf, size_t(wq_bytes(N, K)));
+    MX_REQUIRE(err == cudaSuccess, MX_ERR_CUDA, "weight cache allocation: %s", cudaGetErrorString(err));
+    cache->entries.push_back(mx_wcache::Entry());
+    e = &cache->entries.back();
+    e->w = w;
+    e->N = N;
+    e->K = K;
+    e->q = buf;
+  }
+  *out = carve_weight(e->q, N, K);
+  e->valid = false;
+  MX_TRY(mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, out->qt, out->s_dgrad, st));
+  e->version = version;
+  e->valid = true;
+  return MX_OK;
+}
+
+}  // namespace
+}  // namespace mx
+
+extern "C" {
+
+mx_status mx_linear_fwd(const void* x, const void* w, int64_t M, int64_t N, int64_t K, mx_wcache* cache,
+                        uint64_t w_version, void* y, void* ws, size_t ws_bytes, void* stream) {
+  MX_TRY(check_linear(M, N, K, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint8_t* xq = p;
+  uint8_t* xs = xq + ceil_to(M * K, 256);
+  uint8_t* tail = p + (mx_linear_ws_bytes(M, N, K) - wq_bytes(N, K));
+  WeightView wv;
+  MX_TRY(weight_codes(w, N, K, cache, w_version, tail, &wv, st));
+  if (M == 0) return MX_OK;
+  MX_TRY(mx_cast_dim0(x, M, K, xq, xs, stream));
+  return mx_grouped_mm(xq, xs, wv.q, wv.s_fwd, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
+}
+
+mx_status mx_linear_bwd(const void* dy, const void* x, const void* w, int64_t M, int64_t N, int64_t K,
+                        mx_wcache* cache, uint64_t w_version, void* dx, void* dw, void* ws, size_t ws_bytes,
+                        void* stream) {
+  MX_TRY(check_linear(M, N, K, ws, ws_bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint8_t* dyq = p;                                              // [M, N]
+  uint8_t* dys = dyq + ceil_to(M * N, 256);                      // blocked(M, N/32)
+  uint8_t* dyqt = dys + ceil_to(scale_bytes(M, N / kBlock), 256);  // [N, M]
+  uint8_t* dyst = dyqt + ceil_to(M * N, 256);                    // blocked(N, M/32)
+  uint8_t* xqt = dyst + ceil_to(scale_bytes(N, M / kBlock), 256);  // [K, M]
+  uint8_t* xst = xqt + ceil_to(K * M, 256);                      // blocked(K, M/32)
+  uint8_t* tail = p + (mx_linear_ws_bytes(M, N, K) - wq_bytes(N, K));
+  WeightView wv;
+  MX_TRY(weight_codes(w, N, K, cache, w_version, tail, &wv, st));
+  if (M == 0) {
+    cudaError_t e = cudaMemsetAsync(dw, 0, size_t(N) * K * 2, st);
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MX_OK;
+  }
+  MX_TRY(mx_cast_2d(dy, M, N, dyq, dys, dyqt, dyst, stream));
+  MX_TRY(mx_cast_dim1(x, M, K, xqt, xst, stream));
+  MX_TRY(mx_grouped_mm(dyq, dys, wv.qt, wv.s_dgrad, nullptr, 1, MX_GROUPS_M, dx, M, K, N, 0, stream));
+  return mx_grouped_mm(dyqt, dyst, xqt, xst, nullptr, 1, MX_GROUPS_K, dw, M, N, K, 0, stream);
 }
 
 }  // extern "C"

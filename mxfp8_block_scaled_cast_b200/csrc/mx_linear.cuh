@@ -1,0 +1,63 @@
+// MXFP8 linear forward / dgrad / wgrad and the per-weight quantization cache.
+//
+// The linear composes the casts and the grouped GEMM at one dense group
+// (ao PR #4705, "MXFP8Linear training paths"; torchtitan PR #5334, "a single
+// API for dense and grouped mxfp8 linears"):
+//   forward  Y  = X W^T   X cast 1x32 along K, W cast with 32x32 blocks
+//   dgrad    dX = dY W    dY cast 1x32 along N, W^T codes of the same 32x32 cast
+//   wgrad    dW = dY^T X  dY and X cast 32x1 along the token axis
+// dY is cast once with the fused rowwise+columnwise kernel.
+//
+// Weight cache ("Cache quantized weights for full AC", prime-rl PR #3388,
+// Overview): with full activation checkpointing every checkpoint segment
+// re-runs the forward, which used to re-quantize the weight each time. The
+// cache keeps the 32x32 quantization of each weight, keyed by the weight's
+// device address and shape and invalidated when the caller's version counter
+// (the tensor's in-place update count) changes; it is cleared after
+// backward. Quantization is a pure function of the weight bits, so a hit is
+// bitwise identical to a miss.
+#pragma once
+
+#include <mutex>
+#include <vector>
+
+#include "mx_common.cuh"
+
+struct mx_wcache {
+  struct Entry {
+    const void* w = nullptr;
+    int64_t N = 0, K = 0;
+    uint64_t version = 0;
+    bool valid = false;
+    uint8_t* q = nullptr;        // [N, K]
+    uint8_t* s_fwd = nullptr;    // blocked(N, K/32)
+    uint8_t* qt = nullptr;       // [K, N]
+    uint8_t* s_dgrad = nullptr;  // blocked(K, N/32)
+  };
+  std::vector<Entry> entries;
+  int64_t hits = 0, misses = 0;
+  std::mutex mu;
+};
+
+namespace mx {
+
+// Device bytes of one 32x32-quantized weight (codes, both scale views and the
+// transposed codes), each piece rounded up to 256 bytes.
+inline int64_t wq_bytes(int64_t N, int64_t K) {
+  return ceil_to(N * K, 256) * 2 + ceil_to(scale_bytes(N, K / kBlock), 256) + ceil_to(scale_bytes(K, N / kBlock), 256);
+}
+
+struct WeightView {
+  uint8_t *q, *s_fwd, *qt, *s_dgrad;
+};
+
+inline WeightView carve_weight(uint8_t* base, int64_t N, int64_t K) {
+  WeightView v;
+  v.q = base;
+  v.qt = v.q + ceil_to(N * K, 256);
+  v.s_fwd = v.qt + ceil_to(N * K, 256);
+  v.s_dgrad = v.s_fwd + ceil_to(scale_bytes(N, K / kBlock), 256);
+  return v;
+}
+
+}  // namespace mx

@@ -33,6 +33,14 @@ _SIGNATURES = {
     "mx_cast_dim1_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
+    "mx_wcache_create": (_vp, []),
+    "mx_wcache_clear": (None, [_vp]),
+    "mx_wcache_destroy": (None, [_vp]),
+    "mx_wcache_stats": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "mx_linear_ws_bytes": (_sz, [_i64, _i64, _i64]),
+    "mx_linear_fwd": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _sz, _vp]),
+    "mx_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _vp, _sz,
+                                     _vp]),
 }
 
 MX_GROUPS_M = 0
@@ -144,6 +152,52 @@ def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream
           m_cap, _stream(stream))
 
 
+def mx_linear_ws_bytes(M, N, K) -> int:
+    return int(lib().mx_linear_ws_bytes(M, N, K))
+
+
+def mx_linear_fwd(x, w, cache, w_version, y, ws, stream=None):
+    M, K = x.shape
+    N = w.shape[0]
+    _call("mx_linear_fwd", _p(x), _p(w), M, N, K, cache.handle if cache is not None else None,
+          int(w_version), _p(y), _p(ws), ws.numel(), _stream(stream))
+
+
+def mx_linear_bwd(dy, x, w, cache, w_version, dx, dw, ws, stream=None):
+    M, K = x.shape
+    N = w.shape[0]
+    _call("mx_linear_bwd", _p(dy), _p(x), _p(w), M, N, K, cache.handle if cache is not None else None,
+          int(w_version), _p(dx), _p(dw), _p(ws), ws.numel(), _stream(stream))
+
+
+class WeightCache:
+    """Owner of an mx_wcache: quantized weights reused while their version is unchanged."""
+
+    def __init__(self):
+        self.handle = ctypes.c_void_p(lib().mx_wcache_create())
+        if not self.handle:
+            raise MemoryError("mx_wcache_create failed")
+
+    def clear(self):
+        lib().mx_wcache_clear(self.handle)
+
+    def stats(self):
+        h, m, e = _i64(), _i64(), _i64()
+        _call("mx_wcache_stats", self.handle, ctypes.byref(h), ctypes.byref(m), ctypes.byref(e))
+        return {"hits": h.value, "misses": m.value, "entries": e.value}
+
+    def close(self):
+        if self.handle:
+            lib().mx_wcache_destroy(self.handle)
+            self.handle = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 # --------------------------------------------------- allocating wrappers --
 def _u8(*shape, device):
     return torch.empty(*shape, dtype=torch.uint8, device=device)
@@ -240,3 +294,30 @@ def grouped_mm_wgrad(a_q, a_s, b_q, b_s, offs, M, G=None):
     out = torch.empty(G, N, K, dtype=torch.bfloat16, device=a_q.device)
     mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, MX_GROUPS_K, out, M, N, K, L if offs is not None else 0)
     return out
+
+
+def linear_workspace(M, N, K, device="cuda"):
+    return torch.empty(mx_linear_ws_bytes(M, N, K), dtype=torch.uint8, device=device)
+
+
+def linear_fwd(x, w, cache=None, version=None, ws=None):
+    """y = x w^T through the MXFP8 path; version defaults to w._version."""
+    x, w = _check_bf16(x), _check_bf16(w)
+    M, K = x.shape
+    N = w.shape[0]
+    ws = linear_workspace(M, N, K, x.device) if ws is None else ws
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    mx_linear_fwd(x, w, cache, w._version if version is None else version, y, ws)
+    return y
+
+
+def linear_bwd(dy, x, w, cache=None, version=None, ws=None):
+    """(dx, dw) of y = x w^T; a strided or stride-0 dy is materialised first."""
+    dy, x, w = _check_bf16(dy), _check_bf16(x), _check_bf16(w)
+    M, K = x.shape
+    N = w.shape[0]
+    ws = linear_workspace(M, N, K, x.device) if ws is None else ws
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
+    dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
+    mx_linear_bwd(dy, x, w, cache, w._version if version is None else version, dx, dw, ws)
+    return dx, dw

@@ -1,0 +1,135 @@
+"""MXFP8 linear forward / dgrad / wgrad and the weight cache on the GPU.
+
+Parity against the float64 oracle within 2^-7 |ref| + 1e-3 (|A| |B|^T); the
+cache tests follow the cases named by "Cache quantized weights for full AC"
+(prime-rl PR #3388, Overview): hit/miss, in-place weight update, per-tensor
+isolation, and bit-identical results with and without a hit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mx_oracle as O
+from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from mxfp8_block_scaled_cast_b200 import mx as _mx
+    _mx.lib()
+    return _mx
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, absref, what):
+    bad = np.abs(got - ref) > O.gemm_bound(ref, absref)
+    assert not bad.any(), f"{what}: {bad.sum()} entries outside tolerance"
+
+
+def test_linear_reduced_full_compare(mx):
+    x, w, dy = S.linear_problem(M=512, N=512, K=256, seed=3)
+    y = mx.linear_fwd(x.cuda(), w.cuda())
+    dx, dw = mx.linear_bwd(dy.cuda(), x.cuda(), w.cuda())
+    xb, wb, db = (S.bf16_bits(t) for t in (x, w, dy))
+    _close(_f64(y), *O.linear_fwd(xb, wb), "fwd")
+    _close(_f64(dx), *O.linear_dgrad(db, wb), "dgrad")
+    _close(_f64(dw), *O.linear_wgrad(db, xb), "wgrad")
+
+
+def _sqnr_db(ref, got):
+    ref, got = ref.double(), got.double()
+    return float(10 * torch.log10(ref.pow(2).sum() / (ref - got).pow(2).sum()))
+
+
+def test_linear_full_size_sampled_and_sqnr(mx):
+    """X[4096, 2048], W[4096, 2048], dY[4096, 4096]; sampled entries vs the oracle."""
+    x, w, dy = S.linear_problem(seed=0, device="cuda")
+    cache = mx.WeightCache()
+    y = mx.linear_fwd(x, w, cache)
+    dx, dw = mx.linear_bwd(dy, x, w, cache)
+    mx.mx_device_error()
+    rng = np.random.default_rng(0)
+    yc, dxc, dwc = y.float().cpu().numpy(), dx.float().cpu().numpy(), dw.float().cpu().numpy()
+    for _ in range(48):
+        i, n, k = int(rng.integers(4096)), int(rng.integers(4096)), int(rng.integers(2048))
+        n0, k0, i0 = n // 32 * 32, k // 32 * 32, i // 32 * 32
+        # forward entry (i, n): row i of X (dim0) against row n of W (32x32 scales)
+        qx, sx = O.cast_dim0(S.bf16_bits(x[i:i + 1]))
+        qw, st = O.cast_32x32(S.bf16_bits(w[n0:n0 + 32]))
+        a, b = O.dequant(qx, sx)[0], O.dequant(qw, O.w32_scale_views(st)[0])[n - n0]
+        ref = a @ b
+        assert abs(yc[i, n] - ref) <= 2 ** -7 * abs(ref) + 1e-3 * (np.abs(a) @ np.abs(b))
+        # dgrad entry (i, k): row i of dY (dim0 along N) against column k of W
+        qd, sd = O.cast_dim0(S.bf16_bits(dy[i:i + 1]))
+        qw, st = O.cast_32x32(S.bf16_bits(w[:, k0:k0 + 32]))
+        a = O.dequant(qd, sd)[0]
+        b = O.dequant(np.ascontiguousarray(qw.T), O.w32_scale_views(st)[1])[k - k0]
+        ref = a @ b
+        assert abs(dxc[i, k] - ref) <= 2 ** -7 * abs(ref) + 1e-3 * (np.abs(a) @ np.abs(b))
+        # wgrad entry (n, k): column n of dY and column k of X, cast down the tokens
+        qa, sa = O.cast_dim1(S.bf16_bits(dy[:, n0:n0 + 32]))
+        qb, sb = O.cast_dim1(S.bf16_bits(x[:, k0:k0 + 32]))
+        a, b = O.dequant(qa, sa)[n - n0], O.dequant(qb, sb)[k - k0]
+        ref = a @ b
+        assert abs(dwc[n, k] - ref) <= 2 ** -7 * abs(ref) + 1e-3 * (np.abs(a) @ np.abs(b))
+    # numerics versus the bf16 reference products (reported metric of the linear tests)
+    y_ref = x.float() @ w.float().t()
+    dx_ref = dy.float() @ w.float()
+    dw_ref = dy.float().t() @ x.float()
+    for got, ref in ((y, y_ref), (dx, dx_ref), (dw, dw_ref)):
+        assert _sqnr_db(ref, got.float()) > 20.0
+    cache.close()
+
+
+def test_cache_hit_is_bitwise_identical_and_counted(mx):
+    x, w, dy = S.linear_problem(M=1024, N=1024, K=512, seed=5, device="cuda")
+    y0 = mx.linear_fwd(x, w)                       # no cache
+    dx0, dw0 = mx.linear_bwd(dy, x, w)
+    cache = mx.WeightCache()
+    ys = [mx.linear_fwd(x, w, cache) for _ in range(3)]   # 1 miss + 2 hits (recompute)
+    dx1, dw1 = mx.linear_bwd(dy, x, w, cache)             # hit
+    st = cache.stats()
+    assert st == {"hits": 3, "misses": 1, "entries": 1}
+    for y in ys:
+        assert torch.equal(y, y0)
+    assert torch.equal(dx1, dx0) and torch.equal(dw1, dw0)
+    cache.clear()
+    assert cache.stats()["entries"] == 0
+    cache.close()
+
+
+def test_cache_in_place_update_and_isolation(mx):
+    x, w, _ = S.linear_problem(M=256, N=512, K=256, seed=6, device="cuda")
+    w2 = S.normal_bf16((512, 256), 0.02, seed=7, device="cuda")
+    cache = mx.WeightCache()
+    y_a = mx.linear_fwd(x, w, cache)
+    y_b = mx.linear_fwd(x, w2, cache)              # different tensor: its own entry
+    assert cache.stats()["entries"] == 2
+    assert torch.equal(y_a, mx.linear_fwd(x, w)) and torch.equal(y_b, mx.linear_fwd(x, w2))
+    v0 = w._version
+    with torch.no_grad():
+        w.mul_(2.0)                                # in-place update bumps the version
+    assert w._version != v0
+    y_c = mx.linear_fwd(x, w, cache)
+    assert torch.equal(y_c, mx.linear_fwd(x, w))   # re-quantized, not the stale entry
+    assert not torch.equal(y_c, y_a)
+    st = cache.stats()
+    assert st["misses"] == 3 and st["hits"] == 0 and st["entries"] == 2
+    cache.close()
+
+
+def test_stride0_grad_is_materialised(mx):
+    """out.sum().backward() hands an expanded (stride-0) grad: the wrapper materialises it."""
+    x, w, _ = S.linear_problem(M=256, N=256, K=256, seed=8, device="cuda")
+    g = torch.full((1, 1), 0.5, dtype=torch.bfloat16, device="cuda").expand(256, 256)
+    assert g.stride() == (0, 0)
+    dx, dw = mx.linear_bwd(g, x, w)
+    dx2, dw2 = mx.linear_bwd(g.contiguous(), x, w)
+    assert torch.equal(dx, dx2) and torch.equal(dw, dw2)
+    with pytest.raises(ValueError):
+        mx.mx_cast_2d(g, *mx.cast_2d(g.contiguous()))  # the raw entry refuses strided views
