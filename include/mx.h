@@ -212,6 +212,34 @@ MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
                                mx_wcache* cache, uint64_t w_version, void* dx, void* dw,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- linear forward, no allocation --
+ * No counterpart on the source pages: an addition for callers that cannot
+ * allocate device memory and so cannot pass a workspace -- a plain C host
+ * program linking this library without a device allocator of its own, or a
+ * plugin running inside a runtime that reserves all device memory up front
+ * and forbids further cudaMalloc calls (which can also synchronise the
+ * device).
+ *
+ * Computes exactly what mx_linear_fwd computes without a cache
+ * (y [M, N] = x [M, K] w [N, K]^T, x cast 1x32, w cast 32x32), but keeps
+ * its scratch -- the quantized x and w and their scales,
+ * ceil256(M*K) + ceil256(mx_scale_bytes(M, K/32)) + ceil256(N*K)
+ * + ceil256(mx_scale_bytes(N, K/32)) bytes -- in a fixed device array of
+ * MX_LINEAR_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads
+ * the library holds that array until the process exits. Sizes that need
+ * more are rejected with MX_ERR_UNSUPPORTED and a message naming both
+ * sizes. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress); make that first call before any stream
+ * capture. Every call shares the one array and leaves its contents behind
+ * (each call rewrites every byte it reads, so nothing is cleared): calls
+ * whose work overlaps on the GPU (other streams, other host threads) race
+ * on it, so order them. Same size rules as mx_linear_fwd. */
+#define MX_LINEAR_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+MX_API mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t M, int64_t N, int64_t K,
+                                       void* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

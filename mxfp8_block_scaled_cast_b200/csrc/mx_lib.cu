@@ -491,3 +491,74 @@ mx_status mx_linear_bwd(const void* dy, const void* x, const void* w, int64_t M,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Linear forward without a caller workspace and without any allocation.
+//
+// Some callers cannot hand this library a workspace: a plain C host program
+// that links libmx without a device allocator of its own, or a plugin that
+// runs inside a runtime which reserves all device memory up front and does
+// not allow further cudaMalloc calls (cudaMalloc can also synchronise the
+// device, which such hosts avoid). mx_linear_fwd_noalloc serves them: its
+// scratch (the quantized activations and weight) lives in the fixed array
+// below, which every GPU that loads this library holds until the process
+// exits.
+// ---------------------------------------------------------------------------
+namespace mx {
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MX_LINEAR_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is obtained
+// once per device (with that device current) and reused.
+mx_status noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  MX_REQUIRE(dev >= 0 && dev < kMaxDevices, MX_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    MX_REQUIRE(e == cudaSuccess && p != nullptr, MX_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MX_OK;
+}
+
+}  // namespace
+}  // namespace mx
+
+extern "C" mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t M, int64_t N, int64_t K, void* y,
+                                           void* stream) {
+  MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
+  MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
+  MX_REQUIRE(N % kBN == 0 && K % kBN == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 256");
+  const int64_t xq_b = ceil_to(M * K, 256), xs_b = ceil_to(scale_bytes(M, K / kBlock), 256);
+  const int64_t wq_b = ceil_to(N * K, 256), ws_b = ceil_to(scale_bytes(N, K / kBlock), 256);
+  const int64_t need = xq_b + xs_b + wq_b + ws_b;
+  MX_REQUIRE(need <= int64_t(MX_LINEAR_NOALLOC_SCRATCH_BYTES), MX_ERR_UNSUPPORTED,
+             "mx_linear_fwd_noalloc needs %lld bytes of scratch for M=%lld N=%lld K=%lld; its static scratch "
+             "holds %lld bytes (use mx_linear_fwd with a workspace)",
+             (long long)need, (long long)M, (long long)N, (long long)K, (long long)MX_LINEAR_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  MX_TRY(noalloc_scratch(&scratch));
+  uint8_t* xq = static_cast<uint8_t*>(scratch);
+  uint8_t* xs = xq + xq_b;
+  uint8_t* wq = xs + xs_b;
+  uint8_t* wsf = wq + wq_b;
+  // Every scratch byte the GEMM reads is written by the two casts of this
+  // call (codes and every scale byte, pads included), so nothing needs
+  // clearing between calls.
+  MX_TRY(mx_cast_w32x32(w, 1, N, K, wq, wsf, nullptr, nullptr, stream));
+  if (M == 0) return MX_OK;
+  MX_TRY(mx_cast_dim0(x, M, K, xq, xs, stream));
+  return mx_grouped_mm(xq, xs, wq, wsf, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
+}
+

@@ -41,7 +41,11 @@ _SIGNATURES = {
     "mx_linear_fwd": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _sz, _vp]),
     "mx_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _vp, _sz,
                                      _vp]),
+    "mx_linear_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
 }
+
+# size of the library's fixed scratch array used by mx_linear_fwd_noalloc
+MX_LINEAR_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 MX_GROUPS_M = 0
 MX_GROUPS_K = 1
@@ -168,6 +172,13 @@ def mx_linear_bwd(dy, x, w, cache, w_version, dx, dw, ws, stream=None):
     N = w.shape[0]
     _call("mx_linear_bwd", _p(dy), _p(x), _p(w), M, N, K, cache.handle if cache is not None else None,
           int(w_version), _p(dx), _p(dw), _p(ws), ws.numel(), _stream(stream))
+
+
+def mx_linear_fwd_noalloc(x, w, y, stream=None):
+    """Linear forward whose scratch is the library's fixed device array (no allocation)."""
+    M, K = x.shape
+    N = w.shape[0]
+    _call("mx_linear_fwd_noalloc", _p(x), _p(w), M, N, K, _p(y), _stream(stream))
 
 
 class WeightCache:
