@@ -168,7 +168,7 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  *       L = m_cap (padded token columns from mx_cast_dim1_grouped) or M when
  *       offs == NULL (dense, G = 1, M a multiple of 32)
  *   out bf16 [G, N, K]; an empty group gives exact zeros.
- *   N a multiple of 128, K a multiple of 256.
+ *   N and K multiples of 256.
  * offs: device int32 [G] cumulative ends (see the pad path above) or NULL.
  * Invalid offsets set the device flag and leave the output unwritten. */
 #define MX_GROUPS_M 0

@@ -1,4 +1,4 @@
-// MXFP8 scaled grouped GEMM on sm_100a tensor cores (tcgen05, TMEM, TMA).
+// MXFP8 scaled grouped GEMM on sm_100a tensor cores (tcgen05 CTA pairs, TMEM, TMA).
 //
 // Computes, in fp32 with a bf16 result, the grouped products of the MXFP8
 // grouped GEMM over an offsets array (ao "[moe training] Add
@@ -14,44 +14,53 @@
 // starts on a 128-row boundary of the padded layout (the pad path), so every
 // 128-row scale tile and every 128-wide K tile belongs to one group.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialised):
-//   warp 4      TMA producer: per 128-deep K step, two tiled TMA loads
-//               (A 128x128 B, B 256x128 B, 128-byte swizzle) and three
-//               512-byte bulk copies of blocked scale tiles into a 4-stage
-//               shared-memory ring, completing on a per-stage mbarrier.
-//   warp 5      MMA issuer: copies the stage's scale tiles into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues four
-//               tcgen05.mma.kind::mxf8f6f4.block_scale (M=128, N=256, K=32)
-//               into a 128x256 fp32 TMEM accumulator; tcgen05.commit frees
-//               the stage and, after the last K step, signals the epilogue.
-//   warps 0-3   epilogue: tcgen05.ld of the accumulator (one row per thread),
-//               fp32 -> bf16 (round to nearest even), row stores with the
-//               padded->unpadded row map of the group (the unpad step is
-//               fused here).
-// The tile scheduler is static round robin over (group, m tile, n tile);
-// group boundaries come from a per-CTA scan of the device offsets, so no
-// host synchronisation is needed. An empty group in K-groups mode writes
-// exact zeros (no MMA). There is no split-K and no atomic: results are
-// deterministic.
+// Design: clusters of two CTAs (one per SM) compute 256x256 output tiles
+// with the pair form of the block-scaled MMA. Per 128-deep K step each CTA
+// loads, by TMA into its own shared memory, its 128 rows of A, its 128-row
+// half of B, the 512-byte scale tile of its A rows and both scale tiles of
+// the pair's 256 B rows; all loads count on the leader CTA's stage barrier.
+// Per MMA this moves half the shared-memory and L2 bytes of a one-CTA 128x256
+// tile; under the 1 kW power cap that buys clock (measured: 1989 against
+// 1830 TFLOP/s sustained on 8192^3).
+//   warp 4 (both CTAs)   TMA producer over a 6-stage ring.
+//   warp 5 (leader only) MMA issuer: tcgen05.cp.cta_group::2 of the scale
+//                        tiles into each CTA's TMEM, four
+//                        tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale
+//                        (M=256, N=256, K=32) into a 128x256 fp32 accumulator
+//                        per CTA, and tcgen05.commit multicast to both CTAs
+//                        to free the stage / signal the epilogue.
+//   warps 0-3 (both)     epilogue: tcgen05.ld of the CTA's 128 accumulator
+//                        rows into registers (bf16, round to nearest even),
+//                        TMEM released to the leader, then row stores with the
+//                        padded->unpadded row map (the unpad step is fused
+//                        here) while the next tile's MMAs already run.
+// 256-row tiles are enumerated per group; a group's last tile may extend past
+// the group, and those rows are computed but never stored. Static round robin
+// over tiles; group boundaries come from a per-CTA scan of the device offsets,
+// so there is no host synchronisation. An empty group in K-groups mode
+// writes exact zeros. No split-K and no atomics: results are deterministic.
+// No TMA multicast is used.
 #pragma once
 
 #include "mx_sm100.cuh"
 
 namespace mx {
 
-constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStages = 4;
+constexpr int kPairM = 256, kCtaM = 128, kBN = 256, kBK = 128;
+constexpr int kBM = kCtaM;
+constexpr int kStages = 6;
 constexpr int kGemmThreads = 192;
-constexpr uint32_t kABytes = kBM * kBK;                   // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK;                   // 32 KB
+constexpr uint32_t kABytes = kCtaM * kBK;                 // 16 KB per CTA
+constexpr uint32_t kBBytes = (kBN / 2) * kBK;             // 16 KB per CTA (half of B)
 constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
-constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr uint32_t kTxBytes = 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes);   // both CTAs
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;
 constexpr uint32_t kSfaCol = 256;
 constexpr uint32_t kSfbCol = kSfaCol + 4 * kStages;
+static_assert(kSfbCol + 8 * kStages <= kTmemCols, "TMEM budget");
 
-// shared-memory map (offsets from a 1024-byte aligned base)
+// shared-memory map (offsets from a 1024-byte aligned base; identical in both CTAs)
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
@@ -61,86 +70,88 @@ constexpr uint32_t kNumBars = 2 * kStages + 3;            // full, empty, acc_fu
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem slot, abort, info words
 constexpr uint32_t kOffEnds = kOffMisc + 64;
 constexpr uint32_t kOffPstart = kOffEnds + 4 * kMaxGroups;
-constexpr uint32_t kGemmSmem = kOffPstart + 4 * (kMaxGroups + 1) + 1024;   // + alignment slack
+constexpr uint32_t kOffTstart = kOffPstart + 4 * (kMaxGroups + 1);
+constexpr uint32_t kGemmSmem = kOffTstart + 4 * (kMaxGroups + 1) + 1024;   // + alignment slack
+static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 
 // Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 A and B
 // (format 0), both K-major, N>>3 in bits [17,23), E8M0 scales (bit 23),
-// M>>4 in bits [24,29); the scale-factor byte ids (bits [4,6) for B and
-// [29,31) for A) select which of the four K blocks packed in each TMEM
-// scale column this MMA uses.
-constexpr uint32_t kIdescBase = (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24);
+// M>>4 in bits [24,29) (M = 256 for the pair); the scale-factor byte ids
+// (bits [4,6) for B and [29,31) for A) select which of the four K blocks
+// packed in each TMEM scale column this MMA uses.
+constexpr uint32_t kIdescBase = (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kPairM >> 4) << 24);
 
 enum GemmMode : int { kGroupsM = 0, kGroupsK = 1 };
 
 struct GemmArgs {
-  const uint8_t* a_s;          // A blocked scales
-  const uint8_t* b_s;          // B blocked scales (M-groups: G concatenated per-expert buffers)
   const int32_t* offs;         // cumulative group ends, or null for one dense group
   __nv_bfloat16* out;
   int G;
   int64_t M, N, K;             // see the mode description above
   int64_t m_cap;               // padded capacity (rows of A in M mode, token columns in K mode)
-  int64_t a_sc_tiles;          // 4-column scale tiles per 128-row band of A's blocked scales
+  int64_t a_sc_tiles;          // 4-column scale tiles (512-byte chunks) per 128-row band of A
   int64_t b_sc_tiles;          // same for B
-  int64_t b_sc_group_stride;   // bytes between experts' B scale buffers (M mode)
+  int64_t b_sc_group_chunks;   // chunks between experts' B scale buffers (M mode)
 };
 
 struct TileInfo {
   int g;
   int nk;              // number of 128-deep K steps (0: empty K group)
   int kt0;             // first K step (in units of 128)
-  int64_t a_row0;      // first row of A
-  int64_t b_row0;      // first row of B (global row of the TMA map)
-  int64_t b_loc0;      // first row of B inside its scale buffer
+  int64_t m0;          // first row of A for the pair (M mode: padded row)
+  int64_t b_row0;      // first row of B for the pair (global row of the TMA map)
+  int64_t b_chunk0;    // scale chunk of B's first 128 rows at K step 0
   int64_t n0;          // first output column
-  int64_t m_row0;      // M mode: first padded row; K mode: first output row
 };
 
 template <int kMode>
 __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a, const int32_t* ends,
-                                                const int32_t* pstart) {
+                                                const int32_t* pstart, const int32_t* tstart) {
   TileInfo t;
   if (kMode == kGroupsM) {
     const int64_t nt = a.N / kBN;
     const int64_t mt = tile / nt;
     t.n0 = (tile % nt) * kBN;
-    t.m_row0 = mt * kBM;
-    int lo = 0, hi = a.G;   // largest g with pstart[g] <= row
+    int lo = 0, hi = a.G;   // largest g with tstart[g] <= mt
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (pstart[mid] <= t.m_row0) lo = mid; else hi = mid;
+      if (tstart[mid] <= mt) lo = mid; else hi = mid;
     }
     t.g = lo;
+    t.m0 = pstart[t.g] + (mt - tstart[t.g]) * kPairM;
     t.nk = int(a.K / kBK);
     t.kt0 = 0;
-    t.a_row0 = t.m_row0;
-    t.b_loc0 = t.n0;
     t.b_row0 = int64_t(t.g) * a.N + t.n0;
+    t.b_chunk0 = int64_t(t.g) * a.b_sc_group_chunks + (t.n0 / kCtaM) * a.b_sc_tiles;
   } else {
-    const int64_t nt = a.K / kBN, mt = a.N / kBM;
+    const int64_t nt = a.K / kBN, mt = a.N / kPairM;
     const int64_t per_g = nt * mt;
     t.g = int(tile / per_g);
     const int64_t rem = tile % per_g;
-    t.m_row0 = (rem / nt) * kBM;
+    t.m0 = (rem / nt) * kPairM;
     t.n0 = (rem % nt) * kBN;
     const int64_t start = t.g ? ends[t.g - 1] : 0;
     const int64_t size = ends[t.g] - start;
     t.kt0 = int(pstart[t.g] / kBK);
     t.nk = int((size + kBK - 1) / kBK);
-    t.a_row0 = t.m_row0;
-    t.b_loc0 = t.n0;
     t.b_row0 = t.n0;
+    t.b_chunk0 = (t.n0 / kCtaM) * a.b_sc_tiles;
   }
   return t;
 }
 
 // Waits, bounded by time only (used to drain copies and MMAs before exit).
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      flag_error(kErrTimeout);
-      return;
+  uint64_t t0 = 0;
+  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 1023u) == 0) {
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        flag_error(kErrTimeout);
+        return;
+      }
     }
   }
 }
@@ -148,10 +159,13 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+               const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();      // 0 = leader of the pair
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + kOffBar;
@@ -165,75 +179,90 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   int64_t* info = reinterpret_cast<int64_t*>(smem + kOffMisc + 8);        // [0] total tiles
   int32_t* ends = reinterpret_cast<int32_t*>(smem + kOffEnds);
   int32_t* pstart = reinterpret_cast<int32_t*>(smem + kOffPstart);
+  int32_t* tstart = reinterpret_cast<int32_t*>(smem + kOffTstart);
 
   // ---------------------------------------------------------------- setup --
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&map_a);
     tma_prefetch_desc(&map_b);
+    tma_prefetch_desc(&map_sfa);
+    tma_prefetch_desc(&map_sfb);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 8);      // four epilogue warps in each CTA of the pair
     mbar_init(done_bar, 1);
     fence_barrier_init();
     *abort_flag = 0;
   }
   if (warp == 5) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 0) {
-    // group table: ends[g] and padded starts pstart[0..G]
+    // group table: ends[g], padded starts pstart[0..G], 256-row tile starts tstart[0..G]
     bool bad = false;
+    const int G = args.offs ? args.G : 1;
     if (args.offs == nullptr) {
       if (lane == 0) {
-        const int64_t len = args.M;
-        ends[0] = int32_t(len);
+        ends[0] = int32_t(args.M);
         pstart[0] = 0;
-        pstart[1] = int32_t(ceil_to(len, kBM));
+        pstart[1] = int32_t(ceil_to(args.M, kCtaM));
+        tstart[0] = 0;
+        tstart[1] = int32_t(ceil_div(args.M, kPairM));
       }
     } else {
       const unsigned full = 0xFFFFFFFFu;
-      int64_t carry = 0, prev_end = 0;
-      if (lane == 0) pstart[0] = 0;
-      for (int base = 0; base < args.G; base += 32) {
+      int64_t carry = 0, tcarry = 0, prev_end = 0;
+      if (lane == 0) {
+        pstart[0] = 0;
+        tstart[0] = 0;
+      }
+      for (int base = 0; base < G; base += 32) {
         const int g = base + lane;
-        const bool in = g < args.G;
+        const bool in = g < G;
         const int64_t e = in ? int64_t(__ldg(args.offs + g)) : 0;
         int64_t s = __shfl_up_sync(full, e, 1);
         if (lane == 0) s = prev_end;
         const int64_t size = in ? e - s : 0;
         if (in && size < 0) bad = true;
-        const int64_t pad = size > 0 ? ceil_to(size, kBM) : 0;
-        int64_t incl = pad;
+        const int64_t pad = size > 0 ? ceil_to(size, kCtaM) : 0;
+        const int64_t ntl = ceil_div(pad, kPairM);
+        int64_t incl = pad, tincl = ntl;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int64_t t = __shfl_up_sync(full, incl, o);
-          if (lane >= o) incl += t;
+          const int64_t u = __shfl_up_sync(full, tincl, o);
+          if (lane >= o) {
+            incl += t;
+            tincl += u;
+          }
         }
         if (in) {
           ends[g] = int32_t(e);
           pstart[g + 1] = int32_t(carry + incl);
+          tstart[g + 1] = int32_t(tcarry + tincl);
         }
         carry = __shfl_sync(full, carry + incl, 31);
-        prev_end = __shfl_sync(full, e, min(31, args.G - 1 - base));
+        tcarry = __shfl_sync(full, tcarry + tincl, 31);
+        prev_end = __shfl_sync(full, e, min(31, G - 1 - base));
       }
       bad = __any_sync(full, bad);
       if (prev_end != args.M || carry > args.m_cap) bad = true;
     }
     if (lane == 0) {
-      const int G = args.offs ? args.G : 1;
       int64_t total;
-      if (kMode == kGroupsM) total = bad ? 0 : int64_t(pstart[G] / kBM) * (args.N / kBN);
-      else total = bad ? 0 : int64_t(G) * (args.N / kBM) * (args.K / kBN);
-      if (bad) flag_error(kErrOffsets);
+      if (kMode == kGroupsM) total = bad ? 0 : int64_t(tstart[G]) * (args.N / kBN);
+      else total = bad ? 0 : int64_t(G) * (args.N / kPairM) * (args.K / kBN);
+      if (bad && rank == 0) flag_error(kErrOffsets);
       info[0] = total;
     }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();          // the pair's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t total_tiles = info[0];
@@ -242,80 +271,102 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
 
   // ----------------------------------------------------------- producer ---
   if (warp == 4) {
-    if (lane == 0) {
+    {
+      // The whole warp runs the loop (warp-uniform state); one elected lane
+      // issues the copies.
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0;   // bit s: stage s has a load in flight or landed
-      uint32_t last_par = 0; // bit s: parity of the last phase issued on stage s
-      for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart);
-        const uint8_t* sfa = a.a_s + (t.a_row0 / kBM) * a.a_sc_tiles * 512;
-        const uint8_t* sfb = a.b_s + int64_t(kMode == kGroupsM ? t.g : 0) * a.b_sc_group_stride +
-                             (t.b_loc0 / kBM) * a.b_sc_tiles * 512;
+      uint32_t issued = 0, last_par = 0;
+      for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
+        const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
+        const int32_t a_row = int32_t(t.m0 + kCtaM * rank);
+        const int32_t b_row = int32_t(t.b_row0 + (kBN / 2) * rank);
+        const int64_t sfa_chunk0 = ((t.m0 + kCtaM * rank) / kCtaM) * a.a_sc_tiles;
         bool ok = true;
         for (int kt = 0; kt < t.nk; ++kt) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const int kk = t.kt0 + kt;
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, kTxBytes);
-          tma_load_2d(sbase + kOffA + stage * kABytes, &map_a, kk * kBK, int32_t(t.a_row0), fb);
-          tma_load_2d(sbase + kOffB + stage * kBBytes, &map_b, kk * kBK, int32_t(t.b_row0), fb);
-          bulk_load(sbase + kOffSfa + stage * kSfaBytes, sfa + int64_t(kk) * 512, 512, fb);
-          bulk_load(sbase + kOffSfb + stage * kSfbBytes, sfb + int64_t(kk) * 512, 512, fb);
-          bulk_load(sbase + kOffSfb + stage * kSfbBytes + 512, sfb + (a.b_sc_tiles + kk) * 512, 512, fb);
+          if (elect_one()) {
+            if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
+            const uint32_t lb = mapa_shared(fb, 0);
+            tma_load_2d_pair(sbase + kOffA + stage * kABytes, &map_a, kk * kBK, a_row, lb);
+            tma_load_2d_pair(sbase + kOffB + stage * kBBytes, &map_b, kk * kBK, b_row, lb);
+            tma_load_2d_pair(sbase + kOffSfa + stage * kSfaBytes, &map_sfa, 0, int32_t(sfa_chunk0 + kk), lb);
+            tma_load_2d_pair(sbase + kOffSfb + stage * kSfbBytes, &map_sfb, 0, int32_t(t.b_chunk0 + kk), lb);
+            tma_load_2d_pair(sbase + kOffSfb + stage * kSfbBytes + 512, &map_sfb, 0,
+                             int32_t(t.b_chunk0 + a.b_sc_tiles + kk), lb);
+          }
+          __syncwarp();
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
       }
-      // every issued copy must land before this CTA's shared memory is released
-      for (int s = 0; s < kStages; ++s)
-        if (issued & (1u << s)) mbar_drain(full_bar(s), (last_par >> s) & 1u);
+      // the leader's stages count both CTAs' copies: wait for them to land
+      if (rank == 0 && lane == 0)
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s)) mbar_drain(full_bar(s), (last_par >> s) & 1u);
     }
     __syncwarp();
   }
-  // ---------------------------------------------------------------- MMA ---
+  // ------------------------------------------------------ MMA (leader) ---
   else if (warp == 5) {
-    if (lane == 0) {
+    if (rank == 0) {
+      // The whole warp runs the loop so that descriptors and TMEM addresses
+      // stay warp-uniform; one elected lane issues each tcgen05 group.
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t d_tmem = tmem + kAccCol;
-      for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart);
+      // Descriptors of stage 0 / K block 0, built once. A descriptor's start
+      // address field holds (address >> 4) in its low bits, so moving to
+      // another stage or K block is one 64-bit add; the issue loop below is
+      // then a handful of instructions per MMA and keeps the tensor pipe fed.
+      const uint64_t a_desc0 = smem_desc(sbase + kOffA, 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(sbase + kOffB, 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(sbase + kOffSfa, 0, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(sbase + kOffSfb, 0, 128, 0);
+      for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
+        const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
         if (t.nk == 0) continue;
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp(acc_empty, acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < t.nk; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+          // The TMA bytes of this stage are visible to the tensor core once
+          // the stage barrier's phase completes (both are async-proxy
+          // accesses ordered by the mbarrier), so no fence is needed here.
+          if (!mbar_wait_warp(full_bar(stage), phase, abort_flag)) { ok = false; break; }
           const uint32_t sfa_t = tmem + kSfaCol + 4u * stage;
           const uint32_t sfb_t = tmem + kSfbCol + 8u * stage;
-          const uint32_t sfa_s = sbase + kOffSfa + stage * kSfaBytes;
-          const uint32_t sfb_s = sbase + kOffSfb + stage * kSfbBytes;
-          tmem_cp_32x128b_x4(sfa_t, smem_desc(sfa_s, 0, 128, 0));
-          tmem_cp_32x128b_x4(sfb_t, smem_desc(sfb_s, 0, 128, 0));
-          tmem_cp_32x128b_x4(sfb_t + 4, smem_desc(sfb_s + 512, 0, 128, 0));
-          const uint32_t a_s = sbase + kOffA + stage * kABytes;
-          const uint32_t b_s = sbase + kOffB + stage * kBBytes;
-#pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) {
-            const uint64_t ad = smem_desc(a_s + 32u * k, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_s + 32u * k, 16, 1024, 2);
-            const uint32_t idesc = kIdescBase | (uint32_t(k) << 4) | (uint32_t(k) << 29);
-            mma_mxf8(d_tmem, ad, bd, idesc, sfa_t, sfb_t, (kt | k) != 0 ? 1u : 0u);
+          const uint64_t ad = a_desc0 + uint64_t((stage * kABytes) >> 4);
+          const uint64_t bd = b_desc0 + uint64_t((stage * kBBytes) >> 4);
+          const uint32_t acc0 = kt != 0 ? 1u : 0u;
+          if (elect_one()) {
+            tmem_cp_32x128b_x4_pair(sfa_t, sfa_desc0 + uint64_t((stage * kSfaBytes) >> 4));
+            tmem_cp_32x128b_x4_pair(sfb_t, sfb_desc0 + uint64_t((stage * kSfbBytes) >> 4));
+            tmem_cp_32x128b_x4_pair(sfb_t + 4, sfb_desc0 + uint64_t((stage * kSfbBytes + 512) >> 4));
+            // K block k of the 128-deep stage: +32 bytes (2 in the >>4 field)
+            mma_mxf8_pair(d_tmem, ad, bd, kIdescBase, sfa_t, sfb_t, acc0);
+            mma_mxf8_pair(d_tmem, ad + 2, bd + 2, kIdescBase | (1u << 4) | (1u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 4, bd + 4, kIdescBase | (2u << 4) | (2u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 6, bd + 6, kIdescBase | (3u << 4) | (3u << 29), sfa_t, sfb_t, 1u);
+            tc_commit_pair(empty_bar(stage));
           }
-          tc_commit(empty_bar(stage));
+          __syncwarp();
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        if (elect_one()) tc_commit_pair(acc_full);
+        __syncwarp();
         acc_phase ^= 1u;
       }
-      // all MMAs of this thread complete before TMEM is released
-      tc_commit(done_bar);
-      mbar_drain(done_bar, 0);
+      // all MMAs of the pair complete before either CTA releases TMEM
+      if (elect_one()) {
+        tc_commit_pair(done_bar);
+        mbar_drain(done_bar, 0);
+      }
     }
     __syncwarp();
   }
@@ -324,15 +375,17 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     uint32_t acc_phase = 0;
     const int r = warp * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(warp * 32) << 16) + kAccCol;
-    for (int64_t tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart);
+    const uint32_t leader_acc_empty = mapa_shared(acc_empty, 0);
+    for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
+      const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
+      const int64_t row = t.m0 + kCtaM * rank + r;
       __nv_bfloat16* dst = nullptr;
       if (kMode == kGroupsM) {
         const int64_t start = t.g ? ends[t.g - 1] : 0;
-        const int64_t local = t.m_row0 + r - pstart[t.g];
+        const int64_t local = row - pstart[t.g];
         if (local < ends[t.g] - start) dst = a.out + (start + local) * a.N + t.n0;
       } else {
-        dst = a.out + (int64_t(t.g) * a.N + t.m_row0 + r) * a.K + t.n0;
+        dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
       }
       if (t.nk == 0) {
         if (dst) {
@@ -343,37 +396,39 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       }
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
       tc_fence_after();
-#pragma unroll 1
+      // The whole accumulator row is converted into registers (256 bf16 in
+      // 128 words) so that TMEM is released before the global stores: the
+      // stores then overlap the next tile's main loop.
+      uint32_t rowv[kBN / 2];
+#pragma unroll
       for (int chunk = 0; chunk < kBN / 32; ++chunk) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_lane + uint32_t(chunk * 32), v);
         tmem_ld_wait();
-        if (dst) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + chunk * 32);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-            o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-            o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-            o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-            d4[j] = o;
-          }
-        }
+        for (int j = 0; j < 16; ++j)
+          rowv[chunk * 16 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
       acc_phase ^= 1u;
+      if (dst) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int j = 0; j < kBN / 8; ++j)
+          d4[j] = make_uint4(rowv[4 * j], rowv[4 * j + 1], rowv[4 * j + 2], rowv[4 * j + 3]);
+      }
     }
   }
 
   // ------------------------------------------------------------ teardown ---
   tc_fence_before();
   __syncthreads();
+  cluster_sync();          // no CTA leaves while the pair's MMAs or copies may touch it
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 

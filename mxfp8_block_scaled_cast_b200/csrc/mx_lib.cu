@@ -137,12 +137,57 @@ mx_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
   return MX_OK;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
+// 2D map over a blocked scale buffer viewed as [chunks, 128] 32-bit words:
+// one box = one 512-byte 128x4 scale tile; rows past the buffer read as zero.
+mx_status make_scale_map(CUtensorMap* m, const void* base, uint64_t chunks) {
+  auto fn = encode_fn();
+  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {128u, chunks};
+  cuuint64_t strides[1] = {512u};
+  cuuint32_t box[2] = {128u, 1u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
+  return MX_OK;
 }
+
+template <int kMode>
+mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa, const CUtensorMap& msb,
+                      const GemmArgs& ga, int64_t pair_tiles_ub, cudaStream_t st) {
+  static int max_pairs[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  MX_REQUIRE(e == cudaSuccess && dev < 64, MX_ERR_CUDA, "cudaGetDevice failed");
+  e = cudaFuncSetAttribute(mx_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs[dev] == 0) {
+    cfg.gridDim = dim3(2, 1, 1);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<kMode>, &cfg);
+    MX_REQUIRE(e == cudaSuccess && n > 0, MX_ERR_CUDA, "no CTA pair fits on this device (%s)", cudaGetErrorString(e));
+    max_pairs[dev] = n;
+  }
+  const int64_t pairs = pair_tiles_ub < max_pairs[dev] ? pair_tiles_ub : max_pairs[dev];
+  cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, mx_gemm_kernel<kMode>, ma, mb, msa, msb, ga);
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  return cuda_check("gemm launch");
+}
+
 
 }  // namespace
 }  // namespace mx
@@ -302,16 +347,13 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   GemmArgs ga;
   memset(&ga, 0, sizeof(ga));
-  ga.a_s = static_cast<const uint8_t*>(a_s);
-  ga.b_s = static_cast<const uint8_t*>(b_s);
   ga.offs = offs;
   ga.out = static_cast<__nv_bfloat16*>(out);
   ga.G = G;
   ga.M = M;
   ga.N = N;
   ga.K = K;
-  CUtensorMap map_a, map_b;
-  int64_t tiles_ub = 0;
+  CUtensorMap map_a, map_b, map_sa, map_sb;
   if (mode == MX_GROUPS_M) {
     MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
     MX_REQUIRE(K % kBK == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 128", (long long)K);
@@ -321,43 +363,35 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
     MX_REQUIRE(a_q && a_s && b_q && b_s && out, MX_ERR_ARG, "null operand");
     ga.a_sc_tiles = K / kBK;
     ga.b_sc_tiles = K / kBK;
-    ga.b_sc_group_stride = scale_bytes(N, K / kBlock);
-    MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kBM));
-    MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN));
-    tiles_ub = ceil_div(rows_a, kBM) * (N / kBN);
-  } else {
-    MX_REQUIRE(N % kBM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 128", (long long)N);
-    MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
-    MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
-    const int64_t len = offs ? m_cap : M;
-    MX_REQUIRE(offs || M % kBlock == 0, MX_ERR_UNSUPPORTED, "dense K-groups needs M %% 32 == 0");
-    ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
-    if (len == 0) {
-      cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
-      MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
-      return MX_OK;
-    }
-    MX_REQUIRE(a_q && a_s && b_q && b_s, MX_ERR_ARG, "null operand");
-    ga.a_sc_tiles = ceil_div(ceil_div(len, kBlock), 4);
-    ga.b_sc_tiles = ga.a_sc_tiles;
-    ga.b_sc_group_stride = 0;
-    MX_TRY(make_map(&map_a, a_q, uint64_t(len), uint64_t(N), kBM));
-    MX_TRY(make_map(&map_b, b_q, uint64_t(len), uint64_t(K), kBN));
-    tiles_ub = int64_t(G) * (N / kBM) * (K / kBN);
+    ga.b_sc_group_chunks = scale_bytes(N, K / kBlock) / 512;
+    MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kCtaM));
+    MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN / 2));
+    MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(rows_a, K / kBlock) / 512)));
+    MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(G) * uint64_t(ga.b_sc_group_chunks)));
+    const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * (N / kBN);
+    return launch_gemm<kGroupsM>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
   }
-  const int sms = sm_count();
-  MX_REQUIRE(sms > 0, MX_ERR_CUDA, "no CUDA device");
-  const unsigned grid = unsigned(tiles_ub < sms ? tiles_ub : sms);
-  cudaError_t e;
-  if (mode == MX_GROUPS_M) {
-    e = cudaFuncSetAttribute(mx_gemm_kernel<kGroupsM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
-    if (e == cudaSuccess) mx_gemm_kernel<kGroupsM><<<grid, kGemmThreads, kGemmSmem, st>>>(map_a, map_b, ga);
-  } else {
-    e = cudaFuncSetAttribute(mx_gemm_kernel<kGroupsK>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
-    if (e == cudaSuccess) mx_gemm_kernel<kGroupsK><<<grid, kGemmThreads, kGemmSmem, st>>>(map_a, map_b, ga);
+  MX_REQUIRE(N % kPairM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
+  MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
+  MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
+  const int64_t len = offs ? m_cap : M;
+  MX_REQUIRE(offs || M % kBlock == 0, MX_ERR_UNSUPPORTED, "dense K-groups needs M %% 32 == 0");
+  ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
+  if (len == 0) {
+    cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MX_OK;
   }
-  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
-  return cuda_check("gemm launch");
+  MX_REQUIRE(a_q && a_s && b_q && b_s, MX_ERR_ARG, "null operand");
+  ga.a_sc_tiles = ceil_div(ceil_div(len, kBlock), 4);
+  ga.b_sc_tiles = ga.a_sc_tiles;
+  ga.b_sc_group_chunks = 0;
+  MX_TRY(make_map(&map_a, a_q, uint64_t(len), uint64_t(N), kCtaM));
+  MX_TRY(make_map(&map_b, b_q, uint64_t(len), uint64_t(K), kBN / 2));
+  MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(N, ceil_div(len, kBlock)) / 512)));
+  MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(scale_bytes(K, ceil_div(len, kBlock)) / 512)));
+  const int64_t pair_tiles_ub = int64_t(G) * (N / kPairM) * (K / kBN);
+  return launch_gemm<kGroupsK>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
 }
 
 mx_wcache* mx_wcache_create(void) { return new (std::nothrow) mx_wcache(); }

@@ -102,7 +102,7 @@ def test_grouped_dgrad(mx):
 def test_grouped_wgrad_k_groups(mx, sizes):
     """dW_g = dY_g^T X_g over each group's tokens; empty groups are exact zeros."""
     M, G = sum(sizes), len(sizes)
-    dyb = S.normal_bf16((M, 384), 1e-2, seed=9)
+    dyb = S.normal_bf16((M, 512), 1e-2, seed=9)
     xb = S.normal_bf16((M, 512), 1.0, seed=10)
     offs_t = S.offsets_from_sizes(sizes)
     cap = mx.mx_padded_rows_capacity(M, G)
