@@ -31,9 +31,14 @@
 //                        to free the stage / signal the epilogue.
 //   warps 0-3 (both)     epilogue: tcgen05.ld of the CTA's 128 accumulator
 //                        rows into registers (bf16, round to nearest even),
-//                        TMEM released to the leader, then row stores with the
+//                        TMEM released to the leader, then stores with the
 //                        padded->unpadded row map (the unpad step is fused
-//                        here) while the next tile's MMAs already run.
+//                        here), staged through shared memory so each store
+//                        instruction writes whole 64-byte row segments, while
+//                        the next tile's MMAs already run.
+// Two accumulator slots overlap in one 32-column subtile of TMEM; the
+// epilogue drains that subtile first, so the next tile's MMAs start almost
+// as soon as the previous tile ends.
 // 256-row tiles are enumerated per group; a group's last tile may extend past
 // the group, and those rows are computed but never stored. Static round robin
 // over tiles; group boundaries come from a per-CTA scan of the device offsets,
@@ -54,11 +59,15 @@ constexpr uint32_t kABytes = kCtaM * kBK;                 // 16 KB per CTA
 constexpr uint32_t kBBytes = (kBN / 2) * kBK;             // 16 KB per CTA (half of B)
 constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
 constexpr uint32_t kTxBytes = 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes);   // both CTAs
+// TMEM: two accumulator slots that overlap in one 32-column subtile
+// (slot 0 = columns 0..255, slot 1 = columns 224..479) so the next tile's
+// MMAs can start as soon as the epilogue has drained that subtile of the
+// previous tile; scale factors use a two-slot ring at columns 480..503.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;
-constexpr uint32_t kSfaCol = 256;
-constexpr uint32_t kSfbCol = kSfaCol + 4 * kStages;
-static_assert(kSfbCol + 8 * kStages <= kTmemCols, "TMEM budget");
+constexpr uint32_t kAccSlot1 = 224;
+constexpr uint32_t kOverlapCol = 224;                     // shared subtile [224, 256)
+constexpr uint32_t kSfCol = 480;                          // slot k: SFA at +12k (4), SFB at +12k+4 (8)
+static_assert(kSfCol + 24 <= kTmemCols, "TMEM budget");
 
 // shared-memory map (offsets from a 1024-byte aligned base; identical in both CTAs)
 constexpr uint32_t kOffA = 0;
@@ -66,12 +75,14 @@ constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
 constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
 constexpr uint32_t kOffBar = kOffSfb + kStages * kSfbBytes;
-constexpr uint32_t kNumBars = 2 * kStages + 3;            // full, empty, acc_full, acc_empty, done
+constexpr uint32_t kNumBars = 2 * kStages + 6;            // full, empty, acc_full[2], acc_free[2], ovl_free, done
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;     // tmem slot, abort, info words
 constexpr uint32_t kOffEnds = kOffMisc + 64;
 constexpr uint32_t kOffPstart = kOffEnds + 4 * kMaxGroups;
 constexpr uint32_t kOffTstart = kOffPstart + 4 * (kMaxGroups + 1);
-constexpr uint32_t kGemmSmem = kOffTstart + 4 * (kMaxGroups + 1) + 1024;   // + alignment slack
+constexpr uint32_t kOffStage = (kOffTstart + 4 * (kMaxGroups + 1) + 127) & ~127u;   // epilogue staging
+constexpr uint32_t kStageWarpBytes = 32 * 64;            // 32 rows x 32 bf16 per epilogue warp
+constexpr uint32_t kGemmSmem = kOffStage + 4 * kStageWarpBytes + 1024;   // + alignment slack
 static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 
 // Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 A and B
@@ -171,9 +182,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   const uint32_t bar0 = sbase + kOffBar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  const uint32_t acc_full = bar0 + 8u * (2 * kStages);
-  const uint32_t acc_empty = acc_full + 8u;
-  const uint32_t done_bar = acc_full + 16u;
+  const uint32_t acc_full0 = bar0 + 8u * (2 * kStages);   // + 8 * slot
+  const uint32_t acc_free0 = acc_full0 + 16u;              // + 8 * slot
+  const uint32_t ovl_free = acc_full0 + 32u;
+  const uint32_t done_bar = acc_full0 + 40u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int64_t* info = reinterpret_cast<int64_t*>(smem + kOffMisc + 8);        // [0] total tiles
@@ -191,8 +203,11 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);      // four epilogue warps in each CTA of the pair
+    mbar_init(acc_full0, 1);
+    mbar_init(acc_full0 + 8, 1);
+    mbar_init(acc_free0, 8);      // four epilogue warps in each CTA of the pair
+    mbar_init(acc_free0 + 8, 8);
+    mbar_init(ovl_free, 8);
     mbar_init(done_bar, 1);
     fence_barrier_init();
     *abort_flag = 0;
@@ -317,8 +332,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       // The whole warp runs the loop so that descriptors and TMEM addresses
       // stay warp-uniform; one elected lane issues each tcgen05 group.
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      const uint32_t d_tmem = tmem + kAccCol;
+      uint32_t phase = 0;
+      uint32_t tiles_done = 0, ksteps = 0;
       // Descriptors of stage 0 / K block 0, built once. A descriptor's start
       // address field holds (address >> 4) in its low bits, so moving to
       // another stage or K block is one 64-bit add; the issue loop below is
@@ -330,16 +345,23 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
         if (t.nk == 0) continue;
-        if (!mbar_wait_warp(acc_empty, acc_phase ^ 1u, abort_flag)) break;
+        const uint32_t slot = tiles_done & 1u, use = tiles_done >> 1;
+        // this slot's previous tile fully drained, and the previous tile's
+        // shared subtile drained
+        if (!mbar_wait_warp(acc_free0 + 8u * slot, (use & 1u) ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp(ovl_free, (tiles_done & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem + (slot ? kAccSlot1 : 0u);
         bool ok = true;
         for (int kt = 0; kt < t.nk; ++kt) {
           // The TMA bytes of this stage are visible to the tensor core once
           // the stage barrier's phase completes (both are async-proxy
           // accesses ordered by the mbarrier), so no fence is needed here.
           if (!mbar_wait_warp(full_bar(stage), phase, abort_flag)) { ok = false; break; }
-          const uint32_t sfa_t = tmem + kSfaCol + 4u * stage;
-          const uint32_t sfb_t = tmem + kSfbCol + 8u * stage;
+          // scale tiles: two-slot ring; tcgen05.cp and tcgen05.mma issued by
+          // one thread execute in issue order
+          const uint32_t sfa_t = tmem + kSfCol + 12u * (ksteps & 1u);
+          const uint32_t sfb_t = sfa_t + 4u;
           const uint64_t ad = a_desc0 + uint64_t((stage * kABytes) >> 4);
           const uint64_t bd = b_desc0 + uint64_t((stage * kBBytes) >> 4);
           const uint32_t acc0 = kt != 0 ? 1u : 0u;
@@ -355,12 +377,13 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             tc_commit_pair(empty_bar(stage));
           }
           __syncwarp();
+          ++ksteps;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        if (elect_one()) tc_commit_pair(acc_full);
+        if (elect_one()) tc_commit_pair(acc_full0 + 8u * slot);
         __syncwarp();
-        acc_phase ^= 1u;
+        ++tiles_done;
       }
       // all MMAs of the pair complete before either CTA releases TMEM
       if (elect_one()) {
@@ -372,10 +395,12 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   }
   // ----------------------------------------------------------- epilogue ---
   else {
-    uint32_t acc_phase = 0;
+    uint32_t tiles_done = 0;
     const int r = warp * 32 + lane;
-    const uint32_t t_lane = tmem + (uint32_t(warp * 32) << 16) + kAccCol;
-    const uint32_t leader_acc_empty = mapa_shared(acc_empty, 0);
+    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t leader_ovl = mapa_shared(ovl_free, 0);
+    const uint32_t leader_free0 = mapa_shared(acc_free0, 0);
+    uint8_t* stage_buf = smem + kOffStage + warp * kStageWarpBytes;
     for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
       const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
       const int64_t row = t.m0 + kCtaM * rank + r;
@@ -394,30 +419,73 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         }
         continue;
       }
-      if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
+      const uint32_t slot = tiles_done & 1u, use = tiles_done >> 1;
+      if (!mbar_wait(acc_full0 + 8u * slot, use & 1u, abort_flag)) break;
       tc_fence_after();
       // The whole accumulator row is converted into registers (256 bf16 in
       // 128 words) so that TMEM is released before the global stores: the
-      // stores then overlap the next tile's main loop.
+      // stores then overlap the next tile's main loop. The 32-column subtile
+      // shared with the other slot is drained first and released at once.
+      const uint32_t t_acc = lane_base + (slot ? kAccSlot1 : 0u);
       uint32_t rowv[kBN / 2];
-#pragma unroll
-      for (int chunk = 0; chunk < kBN / 32; ++chunk) {
+      auto drain = [&](int chunk) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_lane + uint32_t(chunk * 32), v);
+        tmem_ld_32x32b_x32(t_acc + uint32_t(chunk * 32), v);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          rowv[chunk * 16 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        for (int jj = 0; jj < 16; ++jj)
+          rowv[chunk * 16 + jj] = pack_bf16x2(__uint_as_float(v[2 * jj]), __uint_as_float(v[2 * jj + 1]));
+      };
+      auto release_shared_subtile = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_ovl);
+      };
+      if (slot) {              // shared subtile = chunk 0 of slot 1
+        drain(0);
+        release_shared_subtile();
+#pragma unroll
+        for (int c = 1; c < kBN / 32; ++c) drain(c);
+      } else {                 // shared subtile = chunk 7 of slot 0
+        drain(kBN / 32 - 1);
+        release_shared_subtile();
+#pragma unroll
+        for (int c = 0; c < kBN / 32 - 1; ++c) drain(c);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
-      acc_phase ^= 1u;
-      if (dst) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+      if (lane == 0) mbar_arrive_cluster(leader_free0 + 8u * slot);
+      ++tiles_done;
+      // Coalesced stores: per 32-column chunk the warp's 32 rows go through a
+      // 2 KB shared buffer (16-byte pieces XOR-swizzled by row so both sides
+      // are bank-conflict free), then each instruction writes 8 rows x 64
+      // contiguous bytes -- whole sectors instead of half-filled ones.
+      const bool valid = dst != nullptr;
+      const uint32_t out_lo = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst)) : 0u;
+      const uint32_t out_hi = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst) >> 32) : 0u;
 #pragma unroll
-        for (int j = 0; j < kBN / 8; ++j)
-          d4[j] = make_uint4(rowv[4 * j], rowv[4 * j + 1], rowv[4 * j + 2], rowv[4 * j + 3]);
+      for (int chunk = 0; chunk < kBN / 32; ++chunk) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t phys = uint32_t(k) ^ ((uint32_t(lane) >> 1) & 3u);
+          *reinterpret_cast<uint4*>(stage_buf + lane * 64 + phys * 16) =
+              make_uint4(rowv[chunk * 16 + 4 * k], rowv[chunk * 16 + 4 * k + 1], rowv[chunk * 16 + 4 * k + 2],
+                         rowv[chunk * 16 + 4 * k + 3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = i * 8 + (lane >> 2);       // row within the warp's 32
+          const int k = lane & 3;                   // 16-byte piece within the 64-byte segment
+          const uint32_t lo = __shfl_sync(0xFFFFFFFFu, out_lo, rr);
+          const uint32_t hi = __shfl_sync(0xFFFFFFFFu, out_hi, rr);
+          const uint4 val = *reinterpret_cast<const uint4*>(stage_buf + rr * 64 + ((uint32_t(k) ^ ((uint32_t(rr) >> 1) & 3u)) * 16));
+          if (lo | hi) {
+            __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>((uint64_t(hi) << 32) | lo);
+            *reinterpret_cast<uint4*>(d + chunk * 32 + k * 8) = val;
+          }
+        }
+        __syncwarp();
       }
     }
   }
