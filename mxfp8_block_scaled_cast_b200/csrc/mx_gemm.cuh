@@ -151,22 +151,6 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
   return t;
 }
 
-// Waits, bounded by time only (used to drain copies and MMAs before exit).
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  uint64_t t0 = 0;
-  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
-    if ((it & 1023u) == 0) {
-      const uint64_t now = globaltimer();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
-        flag_error(kErrTimeout);
-        return;
-      }
-    }
-  }
-}
-
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,

@@ -82,6 +82,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Waits, bounded by time only (used to drain copies and MMAs before exit).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 1023u) == 0) {
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        flag_error(kErrTimeout);
+        return;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA ---
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
