@@ -16,6 +16,8 @@ What it computes, and where each step comes from
   block is the smallest power of two 2**e with 448 * 2**e >= amax, stored as
   the E8M0 byte b = e + 127 clamped to [0, 254]. 448 is the largest finite
   E4M3 value. A block whose amax is 0 gets b = 0.
+* FLOOR scale rule (ao backward_override PR, Known follow-ups, "FLOOR is
+  reachable"): scale 2**(floor(log2(amax)) - 8); saturation to 448 is live.
 * Element cast: q = round-to-nearest-even, saturating E4M3 encoding of
   x * 2**(127 - b), with the sign of zero kept.
 * Block geometry: rowwise "dim0" (1x32 along the contiguous axis), columnwise
@@ -149,22 +151,53 @@ def rceil_e8m0(amax) -> np.ndarray:
     return b.astype(np.uint8)
 
 
+def floor_e8m0(amax) -> np.ndarray:
+    """E8M0 byte of the FLOOR scale of blocks with the given amax.
+
+    FLOOR is the other scale rule the ao backward_override page names ("FLOOR
+    is reachable but untested", Known follow-ups). Reading: the OCP MX rule,
+    scale = 2**(floor(log2(amax)) - 8), 8 being the exponent of the largest
+    power of two representable in E4M3 (256 <= 448 < 512); b = that exponent
+    + 127 clamped to [0, 254]; amax == 0 gives b = 0. Scaled elements can then
+    reach up to 511.x and saturate to 448.
+
+    Computed exactly: the largest integer f with 2**f <= amax.
+    """
+    amax = np.asarray(amax, dtype=np.float64)
+    if np.any(~np.isfinite(amax)) or np.any(amax < 0):
+        raise ValueError("floor_e8m0: amax must be finite and non-negative")
+    b = np.zeros(amax.shape, dtype=np.int64)
+    nz = amax > 0
+    if np.any(nz):
+        a = amax[nz]
+        f = np.floor(np.log2(a)).astype(np.int64)
+        for _ in range(4):   # settle with exact comparisons
+            f = np.where(np.ldexp(1.0, f) > a, f - 1, f)
+            f = np.where(np.ldexp(1.0, f + 1) <= a, f + 1, f)
+        assert np.all(np.ldexp(1.0, f) <= a) and np.all(np.ldexp(1.0, f + 1) > a)
+        b[nz] = np.clip(f - 8 + E8M0_BIAS, 0, E8M0_MAX_FINITE)
+    return b.astype(np.uint8)
+
+
+SCALE_RULES = {"rceil": rceil_e8m0, "floor": floor_e8m0}
+
+
 def e8m0_to_f64(b) -> np.ndarray:
     """Value 2**(b - 127) of an E8M0 byte (b = 255, NaN, never produced here)."""
     return np.exp2(np.asarray(b).astype(np.float64) - E8M0_BIAS)
 
 
-def quantize_blocks(xf, axis=-1):
+def quantize_blocks(xf, axis=-1, rule="rceil"):
     """Quantize float64 blocks whose 32 elements lie along ``axis``.
 
     Returns (q, b): q has the shape of xf (uint8 E4M3 codes), b has ``axis``
-    removed (uint8 E8M0 bytes).
+    removed (uint8 E8M0 bytes). ``rule`` is "rceil" (default) or "floor".
     """
     xf = np.asarray(xf, dtype=np.float64)
     if xf.shape[axis] != BLOCK:
         raise ValueError("quantize_blocks: block axis must hold 32 elements")
     amax = np.max(np.abs(xf), axis=axis)
-    b = rceil_e8m0(amax)
+    b = SCALE_RULES[rule](amax)
     inv_scale = np.expand_dims(np.exp2(E8M0_BIAS - b.astype(np.float64)), axis)
     q = e4m3_encode(xf * inv_scale)      # exact: scaling by a power of two
     return q, b
@@ -173,18 +206,18 @@ def quantize_blocks(xf, axis=-1):
 # --------------------------------------------------------------------------
 # The four casts (logical scales; the blocked layout is applied separately)
 # --------------------------------------------------------------------------
-def cast_dim0(x_bits):
+def cast_dim0(x_bits, rule="rceil"):
     """Rowwise 1x32 cast of bf16 X[R, C] -> (Q[R, C], S[R, C/32])."""
     x_bits = np.asarray(x_bits, dtype=np.uint16)
     R, C = x_bits.shape
     if C % BLOCK:
         raise ValueError("cast_dim0: the row length must be a multiple of 32")
     xf = bf16_to_f64(x_bits).reshape(R, C // BLOCK, BLOCK)
-    q, b = quantize_blocks(xf, axis=-1)
+    q, b = quantize_blocks(xf, axis=-1, rule=rule)
     return q.reshape(R, C), b
 
 
-def cast_dim1(x_bits):
+def cast_dim1(x_bits, rule="rceil"):
     """Columnwise 32x1 cast of bf16 X[R, C] -> (Q^T[C, R], S[C, R/32]).
 
     Blocks are X[32i:32i+32, c]; the output is stored transposed so that the
@@ -195,13 +228,13 @@ def cast_dim1(x_bits):
     if R % BLOCK:
         raise ValueError("cast_dim1: the column length must be a multiple of 32")
     xf = bf16_to_f64(x_bits).reshape(R // BLOCK, BLOCK, C)   # [block, row-in-block, col]
-    q, b = quantize_blocks(xf, axis=1)                        # q [R/32, 32, C], b [R/32, C]
+    q, b = quantize_blocks(xf, axis=1, rule=rule)             # q [R/32, 32, C], b [R/32, C]
     return np.ascontiguousarray(q.reshape(R, C).T), np.ascontiguousarray(b.T)
 
 
-def cast_2d(x_bits):
+def cast_2d(x_bits, rule="rceil"):
     """Fused rowwise + columnwise cast: exactly the pair (dim0, dim1)."""
-    return cast_dim0(x_bits), cast_dim1(x_bits)
+    return cast_dim0(x_bits, rule), cast_dim1(x_bits, rule)
 
 
 def cast_32x32(w_bits):

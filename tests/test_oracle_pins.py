@@ -147,6 +147,30 @@ def test_subnormal_block_keeps_nonzero_codes():
     assert np.all(vals != 0) and vals[3] < 0
 
 
+def test_floor_matches_closed_form_on_every_bf16_amax():
+    """FLOOR: b = max(E - 8, 0) from the bf16 exponent field (2^(E-127) <= amax < 2^(E-126))."""
+    bits = _all_finite_bf16()
+    bits = bits[bits < 0x8000]
+    amax = O.bf16_to_f64(bits)
+    E = (bits.astype(np.int64) >> 7) & 0xFF
+    assert np.array_equal(O.floor_e8m0(amax).astype(np.int64), np.maximum(E - 8, 0))
+
+
+def test_floor_vs_rceil_and_saturation():
+    bits = _all_finite_bf16()
+    bits = bits[(bits < 0x8000) & (bits > 0)]
+    amax = O.bf16_to_f64(bits)
+    f, r = O.floor_e8m0(amax).astype(int), O.rceil_e8m0(amax).astype(int)
+    assert np.all((r == f) | (r == f + 1))          # the two rules differ by at most one binade
+    # amax 500 -> floor(log2 500) = 8 -> b = 127, scale 1: 500 saturates to 448, 460 too
+    blk = np.zeros(32)
+    blk[:3] = [500.0, -460.0, 300.0]
+    q, b = O.quantize_blocks(blk, rule="floor")
+    assert b == 127 and q[0] == 0x7E and q[1] == 0xFE and O.e4m3_decode(q[2:3])[0] == 288.0
+    q, b = O.quantize_blocks(blk, rule="rceil")     # RCEIL never saturates: 500 -> scale 2
+    assert b == 128 and O.e4m3_decode(q[:1])[0] == 256.0
+
+
 # ------------------------------------------------------------ geometry -----
 def test_dim1_equals_dim0_of_transpose():
     x = S.bf16_bits(S.tiny_activation(0))
