@@ -121,6 +121,19 @@ MX_API mx_status mx_cast_w32x32(const void* w, int64_t G, int64_t N, int64_t K,
                          void* q, void* s_fwd, void* qt, void* s_dgrad,
                          void* stream);
 
+/* Scale rule selector of mx_cast_ex. RCEIL is the rule of every other entry
+ * point; FLOOR (ao backward_override PR, Known follow-ups: "FLOOR is
+ * reachable") is scale 2^(floor(log2 amax) - 8), with which scaled elements
+ * can exceed 448 and saturate to +-448. */
+#define MX_RCEIL 0
+#define MX_FLOOR 1
+
+/* Rowwise (dims = 1), columnwise (dims = 2) or both (dims = 3) cast under the
+ * given scale rule; buffers and size rules as mx_cast_dim0 / mx_cast_dim1 /
+ * mx_cast_2d (the outputs of an unused direction may be NULL). */
+MX_API mx_status mx_cast_ex(const void* x, int64_t R, int64_t C, int32_t dims, int32_t rule,
+                            void* q, void* s, void* qt, void* st, void* stream);
+
 /* ------------------------------------------------------- group pad path --
  * offs: device int32 [G] cumulative group ends (non-decreasing, offs[G-1] ==
  * M). Group g occupies rows offs[g-1]..offs[g] of x (offs[-1] = 0) and is

@@ -35,7 +35,14 @@ constexpr int kCastPasses = kCastTile * kCastTile / 8 / kCastThreads;   // 8
 constexpr int kXsBytes = kCastTile * kCastTile * 2;                      // bf16 tile
 constexpr int kQsBytes = kCastTile * kCastTile;                          // transposed codes
 
-enum CastMode : int { kModeRow = 1, kModeCol = 2, kModeRowCol = 3, kModeSquare = 4 };
+enum CastMode : int { kModeRow = 1, kModeCol = 2, kModeRowCol = 3, kModeSquare = 4, kModeFloor = 8 };
+
+// Scale byte of a block from its amax bits under the mode's rule (RCEIL by
+// default, FLOOR when the mode carries kModeFloor).
+template <int kMode>
+__device__ __forceinline__ uint32_t scale_b(uint32_t amax_bits) {
+  return (kMode & kModeFloor) ? floor_b(amax_bits) : rceil_b(amax_bits);
+}
 
 struct CastArgs {
   const uint16_t* x;   // bf16 source rows [rows_src, C] (per expert in a stack)
@@ -134,7 +141,7 @@ cast_tile_kernel(const CastArgs a) {
 #pragma unroll
     for (int p = 0; p < kCastPasses; ++p) {
       const int rl = p * 16 + (tid >> 4);
-      const uint32_t b = kSq ? rceil_b(s_amax[(p >> 1) * 4 + (cl >> 5)]) : rceil_b(bamax[p]);
+      const uint32_t b = kSq ? scale_b<kMode>(s_amax[(p >> 1) * 4 + (cl >> 5)]) : scale_b<kMode>(bamax[p]);
       const float inv = inv_scale(b);
       uint2 o;
       o.x = quant4(v[p].x, v[p].y, inv);
@@ -158,10 +165,10 @@ cast_tile_kernel(const CastArgs a) {
       uint32_t acc = 0u;
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc = absmax_bf16x2(acc, w[i]);
-      b_lo = rceil_b(acc & 0xFFFFu);
-      b_hi = rceil_b(acc >> 16);
+      b_lo = scale_b<kMode>(acc & 0xFFFFu);
+      b_hi = scale_b<kMode>(acc >> 16);
     } else {
-      b_lo = b_hi = rceil_b(s_amax[rb * 4 + (cp >> 4)]);
+      b_lo = b_hi = scale_b<kMode>(s_amax[rb * 4 + (cp >> 4)]);
     }
     const float inv_lo = inv_scale(b_lo), inv_hi = inv_scale(b_hi);
     const int c = 2 * cp;
@@ -224,13 +231,13 @@ cast_tile_kernel(const CastArgs a) {
       const int n = tid;
       uint32_t word = 0u;
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) word |= rceil_b(s_amax[(n >> 5) * 4 + kb]) << (8 * kb);
+      for (int kb = 0; kb < 4; ++kb) word |= scale_b<kMode>(s_amax[(n >> 5) * 4 + kb]) << (8 * kb);
       *reinterpret_cast<uint32_t*>(a.s + z * a.s_stride + chunk_row * 512 + (n & 31) * 16 + (n >> 5) * 4) = word;
     } else if (a.st != nullptr) {
       const int k = tid - 128;
       uint32_t word = 0u;
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb) word |= rceil_b(s_amax[nb * 4 + (k >> 5)]) << (8 * nb);
+      for (int nb = 0; nb < 4; ++nb) word |= scale_b<kMode>(s_amax[nb * 4 + (k >> 5)]) << (8 * nb);
       *reinterpret_cast<uint32_t*>(a.st + z * a.st_stride + chunk_col * 512 + (k & 31) * 16 + (k >> 5) * 4) = word;
     }
   }

@@ -47,6 +47,13 @@ __device__ __forceinline__ uint32_t rceil_b(uint32_t amax_bits) {
   return e < 0 ? 0u : uint32_t(e);
 }
 
+// FLOOR E8M0 byte: scale 2^(floor(log2 amax) - 8); floor(log2 amax) = E - 127
+// for a normal bf16 amax, so b = E - 8, clamped at 0 (zero, tiny, subnormal).
+__device__ __forceinline__ uint32_t floor_b(uint32_t amax_bits) {
+  int e = int(amax_bits >> 7) - 8;
+  return e < 0 ? 0u : uint32_t(e);
+}
+
 // 2^(127 - b) as a float (exact; b in [0, 247] keeps the exponent normal).
 __device__ __forceinline__ float inv_scale(uint32_t b) { return __uint_as_float((254u - b) << 23); }
 

@@ -646,3 +646,32 @@ extern "C" mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t
   return mx_grouped_mm(xq, xs, wq, wsf, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
 }
 
+extern "C" mx_status mx_cast_ex(const void* x, int64_t R, int64_t C, int32_t dims, int32_t rule, void* q, void* s,
+                                void* qt, void* st, void* stream) {
+  MX_REQUIRE(dims >= 1 && dims <= 3, MX_ERR_ARG, "dims must be 1 (rowwise), 2 (columnwise) or 3 (both)");
+  MX_REQUIRE(rule == MX_RCEIL || rule == MX_FLOOR, MX_ERR_ARG, "unknown scale rule %d", rule);
+  if (rule == MX_RCEIL) {
+    if (dims == 1) return mx_cast_dim0(x, R, C, q, s, stream);
+    if (dims == 2) return mx_cast_dim1(x, R, C, qt, st, stream);
+    return mx_cast_2d(x, R, C, q, s, qt, st, stream);
+  }
+  MX_TRY(check_cast_geometry(x, R, C, dims != 1));
+  if (dims & 1) {
+    MX_TRY(check_out(q, R > 0, "q"));
+    MX_TRY(check_out(s, R > 0, "s"));
+  }
+  if (dims & 2) {
+    MX_TRY(check_out(qt, R > 0, "qt"));
+    MX_TRY(check_out(st, R > 0, "st"));
+  }
+  CastArgs a = make_args(x, R, C, R);
+  a.q = static_cast<uint8_t*>(q);
+  a.s = static_cast<uint8_t*>(s);
+  a.qt = static_cast<uint8_t*>(qt);
+  a.st = static_cast<uint8_t*>(st);
+  cudaStream_t stm = static_cast<cudaStream_t>(stream);
+  const int64_t ct = ceil_div(C, kCastTile), rt = ceil_div(R, kCastTile);
+  if (dims == 1) return launch_cast<kModeRow | kModeFloor, false>(a, ct, rt, 1, stm);
+  if (dims == 2) return launch_cast<kModeCol | kModeFloor, false>(a, ct, rt, 1, stm);
+  return launch_cast<kModeRowCol | kModeFloor, false>(a, ct, rt, 1, stm);
+}

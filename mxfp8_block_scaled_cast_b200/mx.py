@@ -42,7 +42,11 @@ _SIGNATURES = {
     "mx_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _vp, _sz,
                                      _vp]),
     "mx_linear_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "mx_cast_ex": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
 }
+
+MX_RCEIL = 0
+MX_FLOOR = 1
 
 # size of the library's fixed scratch array used by mx_linear_fwd_noalloc
 MX_LINEAR_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -131,6 +135,11 @@ def mx_cast_2d(x, q, s, qt, st, stream=None):
 def mx_cast_w32x32(w, q, s_fwd, qt=None, s_dgrad=None, stream=None):
     G, N, K = w.shape if w.dim() == 3 else (1, *w.shape)
     _call("mx_cast_w32x32", _p(w), G, N, K, _p(q), _p(s_fwd), _p(qt), _p(s_dgrad), _stream(stream))
+
+
+def mx_cast_ex(x, dims, rule, q=None, s=None, qt=None, st=None, stream=None):
+    R, C = x.shape
+    _call("mx_cast_ex", _p(x), R, C, dims, rule, _p(q), _p(s), _p(qt), _p(st), _stream(stream))
 
 
 def mx_cast_dim0_grouped(x, offs, m_cap, q, s, stream=None):
@@ -332,3 +341,16 @@ def linear_bwd(dy, x, w, cache=None, version=None, ws=None):
     dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
     mx_linear_bwd(dy, x, w, cache, w._version if version is None else version, dx, dw, ws)
     return dx, dw
+
+
+def cast_floor(x, dims=3):
+    """FLOOR-rule cast: returns (q, s, qt, st) with None for the unused direction."""
+    x = _check_bf16(x)
+    R, C = x.shape
+    q = s = qt = st = None
+    if dims & 1:
+        q, s = _u8(R, C, device=x.device), _u8(mx_scale_bytes(R, C // 32), device=x.device)
+    if dims & 2:
+        qt, st = _u8(C, R, device=x.device), _u8(mx_scale_bytes(C, R // 32), device=x.device)
+    mx_cast_ex(x, dims, MX_FLOOR, q, s, qt, st)
+    return q, s, qt, st

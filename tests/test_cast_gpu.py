@@ -277,3 +277,44 @@ def test_expert_stack_full_size_sampled(mx):
         k_idx = 32 * j + np.arange(32)
         assert np.all(sfb[g * per_f + O.blocked_offset(n_idx, j, K // 32)] == st[0, 0])
         assert np.all(sdb[g * per_d + O.blocked_offset(k_idx, i, N // 32)] == st[0, 0])
+
+
+# ------------------------------------------------------------- FLOOR rule --
+@pytest.mark.parametrize("R,C", [(256, 256), (96, 160), (16384 // 16, 576)])
+def test_floor_casts_match_oracle(mx, R, C):
+    xb = S.sweep_tensor((R, C), seed=R + 3 * C)
+    q, s, qt, st = mx.cast_floor(_dev(xb), dims=3)
+    (eq, es), (eqt, est) = O.cast_2d(S.bf16_bits(xb), rule="floor")
+    assert np.array_equal(_np(q), eq) and np.array_equal(_np(s), O.swizzle(es))
+    assert np.array_equal(_np(qt), eqt) and np.array_equal(_np(st), O.swizzle(est))
+    q0, s0, _, _ = mx.cast_floor(_dev(xb), dims=1)
+    _, _, q1, s1 = mx.cast_floor(_dev(xb), dims=2)
+    for u, v in ((q, q0), (s, s0), (qt, q1), (st, s1)):
+        assert torch.equal(u, v)
+
+
+def test_floor_exhaustive_blocks_and_saturation(mx):
+    bits = _exhaustive_blocks()
+    xb = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    q, s, _, _ = mx.cast_floor(_dev(xb), dims=1)
+    eq, es = O.cast_dim0(bits, rule="floor")
+    assert np.array_equal(_np(q), eq) and np.array_equal(_np(s), O.swizzle(es))
+    # the worked saturation block: 500 and -460 at scale 1 saturate to +-448
+    blk = torch.zeros(32, 32, dtype=torch.float32)
+    blk[0, :3] = torch.tensor([500.0, -460.0, 300.0])
+    q, s, _, _ = mx.cast_floor(_dev(blk.to(torch.bfloat16)), dims=1)
+    assert q[0, :3].tolist() == [0x7E, 0xFE, int(O.e4m3_encode(np.array([300.0]))[0])]
+    rq, _ = mx.cast_dim0(_dev(blk.to(torch.bfloat16)))          # RCEIL: no saturation
+    assert rq[0, 0].item() != 0x7E
+
+
+def test_cast_ex_rceil_matches_plain_entries(mx):
+    xb = _dev(S.sweep_tensor((128, 256), seed=4))
+    R, C = xb.shape
+    u8 = lambda *sh: torch.empty(*sh, dtype=torch.uint8, device="cuda")
+    q, s = u8(R, C), u8(mx.mx_scale_bytes(R, C // 32))
+    qt, st = u8(C, R), u8(mx.mx_scale_bytes(C, R // 32))
+    mx.mx_cast_ex(xb, 3, mx.MX_RCEIL, q, s, qt, st)
+    e = mx.cast_2d(xb)
+    for u, v in zip((q, s, qt, st), e):
+        assert torch.equal(u, v)
