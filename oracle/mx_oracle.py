@@ -472,3 +472,130 @@ def linear_wgrad(dy_bits, x_bits):
     qxt, sxt = cast_dim1(x_bits)       # [K, M]
     a, b = dequant(qdt, sdt), dequant(qxt, sxt)
     return mm(a, b), mm(np.abs(a), np.abs(b))
+
+
+# --------------------------------------------------------------------------
+# Backward overrides (ao "[moe training] Add backward_override to the MXFP8
+# grouped GEMM", Design notes): the "high_precision" arm computes dgrad and
+# wgrad as two plain bf16 grouped GEMMs over the saved, unpadded bf16
+# operands; the "dequantized" arm runs the same two GEMMs on the quantized
+# forward operands turned back into bf16, so its gradients are those of the
+# function the quantized forward computes. Reading taken: "dequantize" means
+# the exact value e4m3(q) * 2**(b - 127), rounded to the nearest bf16 (ties
+# to even) -- the operand type of the bf16 grouped GEMM. The rounding only
+# acts on magnitudes below 2**-133, the smallest bf16 subnormal, and on the
+# one value above the bf16 range (256 * 2**120), which becomes infinity.
+# --------------------------------------------------------------------------
+BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127     # largest finite bf16
+BF16_MIN_EXP = -133                            # exponent of the smallest bf16 subnormal
+
+
+def round_to_bf16(x) -> np.ndarray:
+    """Nearest bf16 value of each float64, ties to even, overflow to +-inf.
+
+    bf16 keeps 8 significant bits; below 2**-126 the spacing stays 2**-133.
+    The spacing of |x| is 2**(floor(log2 |x|) - 7), bounded below by 2**-133;
+    np.rint rounds half to even. Zeros keep their sign; inf and NaN pass.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = x.copy()
+    fin = np.isfinite(x) & (x != 0)
+    ax = np.abs(x[fin])
+    _, e = np.frexp(ax)                        # ax = m * 2**e, m in [0.5, 1)
+    q_exp = np.maximum(e - 1 - 7, BF16_MIN_EXP)
+    r = np.ldexp(np.rint(np.ldexp(ax, -q_exp)), q_exp)
+    r = np.where(r > BF16_MAX, np.inf, r)
+    out[fin] = np.copysign(r, x[fin])
+    return out
+
+
+def f64_to_bf16_bits(x) -> np.ndarray:
+    """bf16 bit patterns of float64 values that are already bf16 values."""
+    x = np.asarray(x, dtype=np.float64)
+    r = round_to_bf16(x)
+    if not np.array_equal(r, x, equal_nan=True):
+        raise ValueError("f64_to_bf16_bits: value is not a bf16 value")
+    bits = (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return np.where(np.isnan(r), np.uint16(0x7FC0), bits).astype(np.uint16)
+
+
+def dequant_bf16(q, s):
+    """bf16 value of the MX tensor Q[..., R, C] with logical scales S[..., R, C/32].
+
+    A NaN code (S.1111.111) or the E8M0 NaN byte 255 gives NaN.
+    """
+    v = dequant(q, s)
+    v = np.where(np.repeat(np.asarray(s) == 255, BLOCK, axis=-1), np.nan, v)
+    return round_to_bf16(v)
+
+
+def dequant_dim0_grouped(q, s, offs):
+    """Rows of a padded dim0 cast gathered back to the unpadded order, as bf16.
+
+    q [m_cap, K] and logical scales s [m_cap, K/32] from cast_dim0_grouped;
+    row start_g + i of the result is padded row p_g + i.
+    """
+    starts, ends = group_bounds(offs)
+    p = padded_group_starts(offs)
+    rows = np.concatenate([np.arange(p[g], p[g] + ends[g] - starts[g])
+                           for g in range(len(starts))] + [np.zeros(0, np.int64)])
+    return dequant_bf16(np.asarray(q)[rows], np.asarray(s)[rows])
+
+
+def hp_grouped_mm_m(a, b, offs):
+    """Groups split the rows: Y[start_g:end_g] = A[start_g:end_g] @ B[g].
+
+    a [M, K], b [G, K, N] (float64); offsets are not padded. Rows outside
+    every group (none when offs[-1] == M) stay zero.
+    """
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    starts, ends = group_bounds(offs)
+    y = np.zeros((a.shape[0], b.shape[2]), dtype=np.float64)
+    for g in range(len(starts)):
+        if ends[g] > starts[g]:
+            y[starts[g]:ends[g]] = a[starts[g]:ends[g]] @ b[g]
+    return y
+
+
+def hp_grouped_mm_k(a, b, offs):
+    """Groups split the contraction: D[g] = A[start_g:end_g]^T @ B[start_g:end_g].
+
+    a [M, N], b [M, K] (float64) -> D [G, N, K]; an empty group gives zeros.
+    """
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    starts, ends = group_bounds(offs)
+    d = np.zeros((len(starts), a.shape[1], b.shape[1]), dtype=np.float64)
+    for g in range(len(starts)):
+        if ends[g] > starts[g]:
+            d[g] = a[starts[g]:ends[g]].T @ b[starts[g]:ends[g]]
+    return d
+
+
+def moe_backward_high_precision(x_bits, w_bits, dy_bits, offs):
+    """"high_precision" arm: dX = dY_g W_g per group, dW_g = dY_g^T X_g.
+
+    x [M, K], w [G, N, K], dy [M, N] (bf16 bits). Returns
+    (dX, |dY| |W|, dW, |dY|^T |X|), float64, the magnitudes for gemm_bound.
+    """
+    x, w, dy = bf16_to_f64(x_bits), bf16_to_f64(w_bits), bf16_to_f64(dy_bits)
+    return (hp_grouped_mm_m(dy, w, offs), hp_grouped_mm_m(np.abs(dy), np.abs(w), offs),
+            hp_grouped_mm_k(dy, x, offs), hp_grouped_mm_k(np.abs(dy), np.abs(x), offs))
+
+
+def moe_backward_dequantized(x_bits, w_bits, dy_bits, offs):
+    """"dequantized" arm: the same two GEMMs on the forward's quantized operands.
+
+    The forward casts X rowwise (1x32) and each expert weight in 32x32 tiles;
+    here those codes are dequantized to bf16 (the forward view of the weight
+    scales) and used in place of X and W. Returns what
+    moe_backward_high_precision returns.
+    """
+    qx, sx = cast_dim0(x_bits)
+    qw, st = cast_32x32(w_bits)
+    s_fwd, _ = w32_scale_views(st)
+    xd, wd = dequant_bf16(qx, sx), dequant_bf16(qw, s_fwd)
+    dy = bf16_to_f64(dy_bits)
+    return (hp_grouped_mm_m(dy, wd, offs), hp_grouped_mm_m(np.abs(dy), np.abs(wd), offs),
+            hp_grouped_mm_k(dy, xd, offs), hp_grouped_mm_k(np.abs(dy), np.abs(xd), offs))

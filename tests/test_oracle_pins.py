@@ -392,3 +392,159 @@ def test_planted_swizzle_slip_is_caught(monkeypatch):
     monkeypatch.setattr(O, "blocked_offset", wrong)
     with pytest.raises(AssertionError):
         test_blocked_offsets_golden()
+
+
+# ------------------------------------------- backward overrides (bf16) -----
+def _f32_samples(n=200000, seed=21):
+    """fp32 bit patterns over every exponent (subnormals and near-ties included)."""
+    rng = np.random.default_rng(seed)
+    u = rng.integers(0, 2 ** 32, size=n, dtype=np.uint64).astype(np.uint32)
+    # force a share of exact ties and one-off-ties of the bf16 rounding
+    tie = rng.random(n) < 0.3
+    low = u & np.uint32(0xFFFF)
+    low = np.where(tie, np.uint32(0x8000) + rng.integers(-1, 2, size=n).astype(np.int64).astype(np.uint32),
+                   low)
+    u = (u & np.uint32(0xFFFF0000)) | (low & np.uint32(0xFFFF))
+    f = u.view(np.float32)
+    return f[np.isfinite(f)]
+
+
+def test_round_to_bf16_matches_torch_conversion():
+    """bf16 rounding of fp32 values (exact in float64) against torch's CPU cast."""
+    f = _f32_samples()
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.round_to_bf16(f.astype(np.float64))
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
+    assert np.array_equal(got, ref)
+
+
+def test_round_to_bf16_worked_values():
+    # ties to even at 1 and in the subnormal range, overflow at the top
+    x = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 2.0 ** -134, 3 * 2.0 ** -134,
+                  (2 - 2.0 ** -8) * 2.0 ** 127, (2 - 2.0 ** -7 - 2.0 ** -9) * 2.0 ** 127, -0.0])
+    want = np.array([1.0, 1 + 2.0 ** -6, 0.0, 2.0 ** -132, np.inf, O.BF16_MAX, -0.0])
+    got = O.round_to_bf16(x)
+    assert np.array_equal(got, want) and np.signbit(got[-1])
+
+
+def test_dequant_bf16_matches_torch_float8_decode_every_code_and_scale():
+    """Every E4M3 code at every finite scale byte, against torch's float8 decode."""
+    codes = np.arange(256, dtype=np.uint8)
+    b = np.arange(255, dtype=np.uint8)
+    q = np.repeat(codes[None, :], b.size, axis=0)                   # [255, 256]
+    s = np.repeat(b[:, None], 256 // 32, axis=1)                    # [255, 8]
+    got = O.dequant_bf16(q, s)
+    tq = torch.from_numpy(q.copy()).view(torch.float8_e4m3fn).to(torch.float32)
+    scale = torch.from_numpy(np.ldexp(1.0, b.astype(np.int64) - 127)).to(torch.float32)
+    ref = (tq * scale[:, None]).to(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    # the E8M0 NaN byte
+    assert np.all(np.isnan(O.dequant_bf16(np.ones((1, 32), np.uint8), np.array([[255]], np.uint8))))
+
+
+def _loop_mm_plain(a, b):
+    """C = A B by explicit sums (A [m, k], B [k, n])."""
+    out = np.zeros((a.shape[0], b.shape[1]))
+    for i in range(a.shape[0]):
+        for j in range(b.shape[1]):
+            acc = 0.0
+            for k in range(a.shape[1]):
+                acc += a[i, k] * b[k, j]
+            out[i, j] = acc
+    return out
+
+
+def test_hp_grouped_mm_m_brute_force_unpadded_groups():
+    rng = np.random.default_rng(31)
+    offs = np.array([3, 3, 8, 11])        # sizes 3, 0, 5, 3: no padding
+    a = rng.standard_normal((11, 4))
+    b = rng.standard_normal((4, 4, 6))
+    y = O.hp_grouped_mm_m(a, b, offs)
+    assert np.allclose(y[0:3], _loop_mm_plain(a[0:3], b[0]))
+    assert np.allclose(y[3:8], _loop_mm_plain(a[3:8], b[2]))
+    assert np.allclose(y[8:11], _loop_mm_plain(a[8:11], b[3]))
+
+
+def test_hp_grouped_mm_k_brute_force_and_empty_group():
+    rng = np.random.default_rng(32)
+    offs = np.array([4, 4, 9])
+    a = rng.standard_normal((9, 3))
+    b = rng.standard_normal((9, 5))
+    d = O.hp_grouped_mm_k(a, b, offs)
+    assert d.shape == (3, 3, 5)
+    assert np.allclose(d[0], _loop_mm_plain(a[0:4].T, b[0:4]))
+    assert np.all(d[1] == 0.0)
+    assert np.allclose(d[2], _loop_mm_plain(a[4:9].T, b[4:9]))
+    # the groups together are the dense product
+    assert np.allclose(d.sum(0), a.T @ b)
+
+
+def test_high_precision_arm_is_the_dense_gradient_at_one_group():
+    x, w, dy = S.linear_problem(64, 96, 128, seed=5)
+    xb, wb, db = (S.bf16_bits(t) for t in (x, w, dy))
+    dx, _, dw, _ = O.moe_backward_high_precision(xb, wb[None], db, np.array([64]))
+    xt, wt, dt = (torch.from_numpy(O.bf16_to_f64(t)) for t in (xb, wb, db))
+    assert np.allclose(dx, (dt @ wt).numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dw[0], (dt.T @ xt).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def _mx_exact_bits(shape, rng, tile):
+    """bf16 values that the casts reproduce exactly: per scale block, E4M3
+    values times 2**e with one element at +-448 * 2**e, so RCEIL picks e."""
+    vals = O._POS_VALUES[rng.integers(0, 0x7F, size=shape)]
+    vals = vals * np.where(rng.random(shape) < 0.5, -1.0, 1.0)
+    R, C = shape
+    th, tw = tile
+    e = rng.integers(-20, 20, size=(R // th, C // tw))
+    vals = vals.reshape(R // th, th, C // tw, tw)
+    vals[:, 0, :, 0] = 448.0
+    vals = vals * np.exp2(e)[:, None, :, None]
+    return O.f64_to_bf16_bits(vals.reshape(R, C))
+
+
+def test_dequantized_arm_equals_high_precision_arm_on_mx_exact_operands():
+    """If X and W are MX-representable the quantized forward loses nothing, so
+    the two override arms must give the same gradients."""
+    rng = np.random.default_rng(33)
+    xb = _mx_exact_bits((96, 64), rng, (1, 32))
+    wb = np.stack([_mx_exact_bits((64, 64), rng, (32, 32)) for _ in range(2)])
+    db = S.bf16_bits(S.normal_bf16((96, 64), seed=7))
+    offs = np.array([40, 96])
+    hp = O.moe_backward_high_precision(xb, wb, db, offs)
+    dq = O.moe_backward_dequantized(xb, wb, db, offs)
+    for u, v in zip(hp, dq):
+        assert np.array_equal(u, v)
+    # and a generic X differs (the arm does dequantize the forward's codes)
+    xg = S.bf16_bits(S.normal_bf16((96, 64), seed=8))
+    assert not np.array_equal(O.moe_backward_high_precision(xg, wb, db, offs)[2],
+                              O.moe_backward_dequantized(xg, wb, db, offs)[2])
+
+
+def test_dequant_grouped_gathers_padded_rows():
+    x = S.normal_bf16((300, 64), seed=9)
+    xb = S.bf16_bits(x)
+    offs = np.array([37, 37, 300])
+    cap = O.padded_rows_capacity(300, 3)
+    qp, sp = O.cast_dim0_grouped(xb, offs, cap)
+    got = O.dequant_dim0_grouped(qp, sp, offs)
+    q, s = O.cast_dim0(xb)
+    assert np.array_equal(got, O.dequant_bf16(q, s))
+
+
+def test_planted_padded_starts_in_hp_wgrad_is_caught(monkeypatch):
+    """Taking the group rows at the padded starts (as the MXFP8 GEMMs do)
+    instead of the unpadded ones fails the brute force."""
+    def slip(a, b, offs):
+        starts, ends = O.group_bounds(offs)
+        p = O.padded_group_starts(offs)
+        d = np.zeros((len(starts), a.shape[1], b.shape[1]))
+        for g in range(len(starts)):
+            n = ends[g] - starts[g]
+            d[g] = a[p[g]:p[g] + n].T @ b[p[g]:p[g] + n]
+        return d
+    monkeypatch.setattr(O, "hp_grouped_mm_k", slip)
+    with pytest.raises(AssertionError):
+        test_hp_grouped_mm_k_brute_force_and_empty_group()
