@@ -15,7 +15,9 @@
  *     backward_override PR, Known follow-ups; "pad/unpad" and "M-groups /
  *     K-groups scale rearrange" kernels, ao PR #4705 stack list);
  *   - the MXFP8 scaled grouped GEMM over an offsets array and its dgrad and
- *     wgrad (ao backward_override PR, Summary; ao PR #4705, description);
+ *     wgrad (ao backward_override PR, Summary; ao PR #4705, description),
+ *     and the bf16 grouped GEMMs, dequantization and scale unswizzle of the
+ *     backward-override arms (ao backward_override PR, Design notes);
  *   - the MXFP8 linear forward / dgrad / wgrad (ao PR #4705, "MXFP8Linear
  *     training paths") and a per-weight quantization cache keyed by the
  *     weight's version counter ("Cache quantized weights for full AC",
@@ -189,6 +191,52 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
 MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
                                const int32_t* offs, int32_t G, int32_t mode, void* out,
                                int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
+
+/* ------------------------------------------- backward-override arms -----
+ * ao "[moe training] Add backward_override to the MXFP8 grouped GEMM", Design
+ * notes: the "high_precision" arm computes dgrad and wgrad of the grouped GEMM
+ * with two plain bf16 grouped GEMMs over the saved, unpadded bf16 operands;
+ * the "dequantized" arm runs the same two GEMMs on the forward's quantized
+ * operands turned back into bf16 (it needs logical scales, for which the page
+ * notes that "no unswizzler exists"; mx_scales_unswizzle is one).
+ *
+ * bf16 grouped GEMM, fp32 accumulation on the tensor cores, bf16 output
+ * (round to nearest even); deterministic (no split-K, no atomics). Groups are
+ * the UNPADDED rows offs[g-1]..offs[g] (any sizes, empty groups allowed;
+ * offs as for the pad path, offs[G-1] == M; NULL = one group, G = 1). No
+ * operand is copied or transposed.
+ * mode MX_GROUPS_M (dgrad):  out[rows of g, :] = a[rows of g, :] @ b[g]
+ *   a bf16 [M, K], b bf16 [G, K, N], out bf16 [M, N].
+ *   N a multiple of 256, K a positive multiple of 8.
+ * mode MX_GROUPS_K (wgrad):  out[g] = a[rows of g, :]^T @ b[rows of g, :]
+ *   a bf16 [M, N], b bf16 [M, K], out bf16 [G, N, K]; an empty group gives
+ *   exact zeros. N and K multiples of 256.
+ * M, N, K < 2^31. Invalid offsets set the device flag and leave the output
+ * unwritten. */
+MX_API mx_status mx_grouped_mm_bf16(const void* a, const void* b, const int32_t* offs, int32_t G,
+                                    int32_t mode, void* out, int64_t M, int64_t N, int64_t K,
+                                    void* stream);
+
+/* Dequantization of rowwise-scaled codes to bf16:
+ *   out[i, r, c] = bf16(e4m3(q[i, r, c]) * 2^(S_i[r, c/32] - 127))
+ * rounded to nearest even (exact unless |value| < 2^-133 or the value
+ * overflows bf16); a NaN code or scale byte 255 gives NaN.
+ *   q E4M3 [G, R, C]; s G concatenated blocked(R, C/32) buffers (a dim0 cast
+ *   with G = 1, or the s_fwd output of mx_cast_w32x32); out bf16 [G, R, C].
+ * G >= 1, R >= 0, C a positive multiple of 32. */
+MX_API mx_status mx_dequant_dim0(const void* q, const void* s, int64_t G, int64_t R, int64_t C,
+                                 void* out, void* stream);
+
+/* The same for the padded rows of mx_cast_dim0_grouped, gathered back to the
+ * unpadded order: out[start_g + i, :] = dequant(row p_g + i).
+ *   q [m_cap, K], s blocked(m_cap, K/32) -> out bf16 [M, K].
+ * Size rules and offsets as mx_cast_dim0_grouped. */
+MX_API mx_status mx_dequant_dim0_grouped(const void* q, const void* s, const int32_t* offs, int32_t G,
+                                         int64_t M, int64_t K, int64_t m_cap, void* out, void* stream);
+
+/* Logical scales from the blocked layout: out uint8 [R, C32] row-major,
+ * out[r, c] = S[r, c] of the blocked buffer s = blocked(R, C32). */
+MX_API mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void* out, void* stream);
 
 /* ------------------------------------------------------ MXFP8 linear -----
  * Dense MXFP8 linear (ao PR #4705, "MXFP8Linear training paths"; torchtitan

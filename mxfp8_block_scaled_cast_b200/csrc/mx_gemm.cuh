@@ -151,6 +151,89 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
   return t;
 }
 
+// ------------------------------------------------------------ epilogue ---
+// One warp's part of a 256-column output tile: its 32 accumulator rows in
+// TMEM slot `slot` (lane i of the warp owns row i; `dst` is that row's first
+// output element, or null for a row that is not stored).
+// The whole accumulator row is converted into registers (256 bf16 in 128
+// words, round to nearest even) so that TMEM is released before the global
+// stores, which then overlap the next tile's main loop. The 32-column subtile
+// shared with the other slot is drained first and released at once
+// (`leader_ovl`), then the rest of the slot (`leader_free`), both barriers of
+// the pair's leader CTA.
+// Stores are coalesced: per 32-column chunk the warp's 32 rows go through a
+// 2 KB shared buffer (16-byte pieces XOR-swizzled by row so both sides are
+// bank-conflict free), then each instruction writes 8 rows x 64 contiguous
+// bytes -- whole sectors instead of half-filled ones.
+__device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot, __nv_bfloat16* dst,
+                                              uint32_t leader_ovl, uint32_t leader_free, uint8_t* stage_buf,
+                                              int lane) {
+  const uint32_t t_acc = lane_base + (slot ? kAccSlot1 : 0u);
+  uint32_t rowv[kBN / 2];
+  auto drain = [&](int chunk) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(t_acc + uint32_t(chunk * 32), v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj)
+      rowv[chunk * 16 + jj] = pack_bf16x2(__uint_as_float(v[2 * jj]), __uint_as_float(v[2 * jj + 1]));
+  };
+  auto release_shared_subtile = [&]() {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(leader_ovl);
+  };
+  if (slot) {              // shared subtile = chunk 0 of slot 1
+    drain(0);
+    release_shared_subtile();
+#pragma unroll
+    for (int c = 1; c < kBN / 32; ++c) drain(c);
+  } else {                 // shared subtile = chunk 7 of slot 0
+    drain(kBN / 32 - 1);
+    release_shared_subtile();
+#pragma unroll
+    for (int c = 0; c < kBN / 32 - 1; ++c) drain(c);
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(leader_free);
+  const bool valid = dst != nullptr;
+  const uint32_t out_lo = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst)) : 0u;
+  const uint32_t out_hi = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst) >> 32) : 0u;
+#pragma unroll
+  for (int chunk = 0; chunk < kBN / 32; ++chunk) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t phys = uint32_t(k) ^ ((uint32_t(lane) >> 1) & 3u);
+      *reinterpret_cast<uint4*>(stage_buf + lane * 64 + phys * 16) =
+          make_uint4(rowv[chunk * 16 + 4 * k], rowv[chunk * 16 + 4 * k + 1], rowv[chunk * 16 + 4 * k + 2],
+                     rowv[chunk * 16 + 4 * k + 3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = i * 8 + (lane >> 2);       // row within the warp's 32
+      const int k = lane & 3;                   // 16-byte piece within the 64-byte segment
+      const uint32_t lo = __shfl_sync(0xFFFFFFFFu, out_lo, rr);
+      const uint32_t hi = __shfl_sync(0xFFFFFFFFu, out_hi, rr);
+      const uint4 val = *reinterpret_cast<const uint4*>(stage_buf + rr * 64 + ((uint32_t(k) ^ ((uint32_t(rr) >> 1) & 3u)) * 16));
+      if (lo | hi) {
+        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>((uint64_t(hi) << 32) | lo);
+        *reinterpret_cast<uint4*>(d + chunk * 32 + k * 8) = val;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// Exact zeros for one 256-column output row (an empty K group), if stored.
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
+  if (dst) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = 0; c < kBN; c += 8) *reinterpret_cast<uint4*>(dst + c) = z;
+  }
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
@@ -397,80 +480,14 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
       }
       if (t.nk == 0) {
-        if (dst) {
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          for (int c = 0; c < kBN; c += 8) *reinterpret_cast<uint4*>(dst + c) = z;
-        }
+        store_zero_row(dst);
         continue;
       }
       const uint32_t slot = tiles_done & 1u, use = tiles_done >> 1;
       if (!mbar_wait(acc_full0 + 8u * slot, use & 1u, abort_flag)) break;
       tc_fence_after();
-      // The whole accumulator row is converted into registers (256 bf16 in
-      // 128 words) so that TMEM is released before the global stores: the
-      // stores then overlap the next tile's main loop. The 32-column subtile
-      // shared with the other slot is drained first and released at once.
-      const uint32_t t_acc = lane_base + (slot ? kAccSlot1 : 0u);
-      uint32_t rowv[kBN / 2];
-      auto drain = [&](int chunk) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_acc + uint32_t(chunk * 32), v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj)
-          rowv[chunk * 16 + jj] = pack_bf16x2(__uint_as_float(v[2 * jj]), __uint_as_float(v[2 * jj + 1]));
-      };
-      auto release_shared_subtile = [&]() {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_ovl);
-      };
-      if (slot) {              // shared subtile = chunk 0 of slot 1
-        drain(0);
-        release_shared_subtile();
-#pragma unroll
-        for (int c = 1; c < kBN / 32; ++c) drain(c);
-      } else {                 // shared subtile = chunk 7 of slot 0
-        drain(kBN / 32 - 1);
-        release_shared_subtile();
-#pragma unroll
-        for (int c = 0; c < kBN / 32 - 1; ++c) drain(c);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_free0 + 8u * slot);
+      epilogue_tile(lane_base, slot, dst, leader_ovl, leader_free0 + 8u * slot, stage_buf, lane);
       ++tiles_done;
-      // Coalesced stores: per 32-column chunk the warp's 32 rows go through a
-      // 2 KB shared buffer (16-byte pieces XOR-swizzled by row so both sides
-      // are bank-conflict free), then each instruction writes 8 rows x 64
-      // contiguous bytes -- whole sectors instead of half-filled ones.
-      const bool valid = dst != nullptr;
-      const uint32_t out_lo = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst)) : 0u;
-      const uint32_t out_hi = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst) >> 32) : 0u;
-#pragma unroll
-      for (int chunk = 0; chunk < kBN / 32; ++chunk) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t phys = uint32_t(k) ^ ((uint32_t(lane) >> 1) & 3u);
-          *reinterpret_cast<uint4*>(stage_buf + lane * 64 + phys * 16) =
-              make_uint4(rowv[chunk * 16 + 4 * k], rowv[chunk * 16 + 4 * k + 1], rowv[chunk * 16 + 4 * k + 2],
-                         rowv[chunk * 16 + 4 * k + 3]);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int rr = i * 8 + (lane >> 2);       // row within the warp's 32
-          const int k = lane & 3;                   // 16-byte piece within the 64-byte segment
-          const uint32_t lo = __shfl_sync(0xFFFFFFFFu, out_lo, rr);
-          const uint32_t hi = __shfl_sync(0xFFFFFFFFu, out_hi, rr);
-          const uint4 val = *reinterpret_cast<const uint4*>(stage_buf + rr * 64 + ((uint32_t(k) ^ ((uint32_t(rr) >> 1) & 3u)) * 16));
-          if (lo | hi) {
-            __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>((uint64_t(hi) << 32) | lo);
-            *reinterpret_cast<uint4*>(d + chunk * 32 + k * 8) = val;
-          }
-        }
-        __syncwarp();
-      }
     }
   }
 

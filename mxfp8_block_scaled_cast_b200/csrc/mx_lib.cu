@@ -1,7 +1,7 @@
 // libmx: the C ABI declared in include/mx.h.
 //
 // This single translation unit holds every kernel of the library (casts,
-// the tcgen05 grouped GEMM, the linear and its weight cache) so that they
+// the tcgen05 grouped GEMMs, dequantization, the linear and its weight cache) so that they
 // share the sticky device error flag without relocatable device code.
 // Host functions validate every argument before any launch and report the
 // reason of a failure through mx_last_error().
@@ -15,7 +15,9 @@
 #include "mx_common.cuh"
 #include "mx_cast.cuh"
 #include "mx_gemm.cuh"
+#include "mx_gemm_bf16.cuh"
 #include "mx_cast_pipe.cuh"
+#include "mx_dequant.cuh"
 #include "mx_linear.cuh"
 
 namespace mx {
@@ -238,6 +240,70 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   return cuda_check("gemm launch");
 }
 
+
+// bf16 tensor map over a row-major [outer, inner] matrix (rank 2) or a stack
+// [depth, outer, inner] (rank 3): boxes of 64 elements (128 bytes) x
+// box_outer rows (x 1 matrix), 128-byte swizzle, zero fill outside.
+mx_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t depth,
+                        uint32_t box_outer) {
+  auto fn = encode_fn();
+  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint32_t rank = depth > 0 ? 3u : 2u;
+  cuuint64_t dims[3] = {inner, outer, depth};
+  cuuint64_t strides[2] = {inner * 2, inner * outer * 2};
+  cuuint32_t box[3] = {64u, box_outer, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (bf16) failed (%d)", int(r));
+  return MX_OK;
+}
+
+template <int kMode>
+mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const HGemmArgs& ha, int64_t pair_tiles_ub,
+                           cudaStream_t st) {
+  static int max_pairs[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  MX_REQUIRE(e == cudaSuccess && dev < 64, MX_ERR_CUDA, "cudaGetDevice failed");
+  e = cudaFuncSetAttribute(bf16_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kHGemmSmem));
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm smem attribute: %s", cudaGetErrorString(e));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kHGemmSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs[dev] == 0) {
+    cfg.gridDim = dim3(2, 1, 1);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, bf16_gemm_kernel<kMode>, &cfg);
+    MX_REQUIRE(e == cudaSuccess && n > 0, MX_ERR_CUDA, "no CTA pair fits on this device (%s)", cudaGetErrorString(e));
+    max_pairs[dev] = n;
+  }
+  const int64_t pairs = pair_tiles_ub < max_pairs[dev] ? pair_tiles_ub : max_pairs[dev];
+  cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, bf16_gemm_kernel<kMode>, ma, mb, ha);
+  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm launch: %s", cudaGetErrorString(e));
+  return cuda_check("bf16 gemm launch");
+}
+
+// Grid for the grid-stride memory-bound kernels: enough CTAs to fill every SM
+// several times, never more than the work.
+unsigned streaming_grid(int64_t items, int threads) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t need = ceil_div(items, threads);
+  const int64_t cap = int64_t(sms) * 8;
+  return unsigned(need < cap ? need : cap);
+}
 
 }  // namespace
 }  // namespace mx
@@ -674,4 +740,110 @@ extern "C" mx_status mx_cast_ex(const void* x, int64_t R, int64_t C, int32_t dim
   if (dims == 1) return launch_cast<kModeRow | kModeFloor, false>(a, ct, rt, 1, stm);
   if (dims == 2) return launch_cast<kModeCol | kModeFloor, false>(a, ct, rt, 1, stm);
   return launch_cast<kModeRowCol | kModeFloor, false>(a, ct, rt, 1, stm);
+}
+
+// ------------------------------------------------ backward-override arms ---
+extern "C" mx_status mx_grouped_mm_bf16(const void* a, const void* b, const int32_t* offs, int32_t G, int32_t mode,
+                                        void* out, int64_t M, int64_t N, int64_t K, void* stream) {
+  MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K, MX_ERR_ARG, "unknown mode %d", mode);
+  MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
+  MX_REQUIRE(M < (1ll << 31) && N < (1ll << 31) && K < (1ll << 31), MX_ERR_ARG, "a size is 2^31 or more");
+  if (offs != nullptr) {
+    MX_REQUIRE(G >= 1 && G <= kMaxGroups, MX_ERR_ARG, "G = %d outside [1, %d]", G, kMaxGroups);
+    MX_REQUIRE((reinterpret_cast<uintptr_t>(offs) & 3u) == 0, MX_ERR_ALIGN, "offsets not 4-byte aligned");
+  } else {
+    MX_REQUIRE(G == 1, MX_ERR_ARG, "without offsets G must be 1 (dense)");
+  }
+  const void* ptrs[3] = {a, b, out};
+  for (const void* p : ptrs) MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "operand not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  HGemmArgs ha;
+  memset(&ha, 0, sizeof(ha));
+  ha.offs = offs;
+  ha.out = static_cast<__nv_bfloat16*>(out);
+  ha.G = G;
+  ha.M = M;
+  ha.N = N;
+  ha.K = K;
+  CUtensorMap map_a, map_b;
+  if (mode == MX_GROUPS_M) {
+    MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
+    MX_REQUIRE(K % 8 == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 8 (16-byte rows)", (long long)K);
+    if (M == 0) return MX_OK;
+    MX_REQUIRE(a && b && out, MX_ERR_ARG, "null operand");
+    MX_TRY(make_map_bf16(&map_a, a, uint64_t(K), uint64_t(M), 0, kCtaM));
+    MX_TRY(make_map_bf16(&map_b, b, uint64_t(N), uint64_t(K), uint64_t(G), 64));
+    const int64_t pair_tiles_ub = (ceil_div(M, kPairM) + (offs ? G : 0)) * (N / kBN);
+    return launch_bf16_gemm<kGroupsM>(map_a, map_b, ha, pair_tiles_ub, st);
+  }
+  MX_REQUIRE(N % kPairM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
+  MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
+  MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
+  if (M == 0) {
+    cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MX_OK;
+  }
+  MX_REQUIRE(a && b, MX_ERR_ARG, "null operand");
+  MX_TRY(make_map_bf16(&map_a, a, uint64_t(N), uint64_t(M), 0, 64));
+  MX_TRY(make_map_bf16(&map_b, b, uint64_t(K), uint64_t(M), 0, 64));
+  const int64_t pair_tiles_ub = int64_t(G) * (N / kPairM) * (K / kBN);
+  return launch_bf16_gemm<kGroupsK>(map_a, map_b, ha, pair_tiles_ub, st);
+}
+
+extern "C" mx_status mx_dequant_dim0(const void* q, const void* s, int64_t G, int64_t R, int64_t C, void* out,
+                                     void* stream) {
+  MX_REQUIRE(G >= 1 && R >= 0 && C > 0, MX_ERR_ARG, "sizes must be G >= 1, R >= 0, C > 0");
+  MX_REQUIRE(C % kBlock == 0, MX_ERR_UNSUPPORTED, "C = %lld is not a multiple of 32", (long long)C);
+  const void* ptrs[3] = {q, s, out};
+  for (const void* p : ptrs) MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "operand not 16-byte aligned");
+  if (R == 0) return MX_OK;
+  MX_REQUIRE(q && s && out, MX_ERR_ARG, "null operand");
+  DequantArgs da;
+  memset(&da, 0, sizeof(da));
+  da.q = static_cast<const uint8_t*>(q);
+  da.s = static_cast<const uint8_t*>(s);
+  da.out = static_cast<__nv_bfloat16*>(out);
+  da.rows_out = G * R;
+  da.C = C;
+  da.layout_rows = R;
+  const int64_t items = da.rows_out * (C / kBlock);
+  dequant_dim0_kernel<false><<<streaming_grid(items, kDeqThreads), kDeqThreads, 0,
+                               static_cast<cudaStream_t>(stream)>>>(da);
+  return cuda_check("dequant launch");
+}
+
+extern "C" mx_status mx_dequant_dim0_grouped(const void* q, const void* s, const int32_t* offs, int32_t G, int64_t M,
+                                             int64_t K, int64_t m_cap, void* out, void* stream) {
+  MX_TRY(check_grouped(q, M, K, offs, G, m_cap));
+  MX_REQUIRE(m_cap < (1ll << 31), MX_ERR_ARG, "m_cap must be < 2^31");
+  MX_REQUIRE(aligned16(s) && aligned16(out), MX_ERR_ALIGN, "operand not 16-byte aligned");
+  if (M == 0) return MX_OK;
+  MX_REQUIRE(s && out, MX_ERR_ARG, "null operand");
+  DequantArgs da;
+  memset(&da, 0, sizeof(da));
+  da.q = static_cast<const uint8_t*>(q);
+  da.s = static_cast<const uint8_t*>(s);
+  da.out = static_cast<__nv_bfloat16*>(out);
+  da.rows_out = M;
+  da.C = K;
+  da.layout_rows = m_cap;
+  da.offs = offs;
+  da.G = G;
+  da.m_cap = m_cap;
+  const int64_t items = M * (K / kBlock);
+  dequant_dim0_kernel<true><<<streaming_grid(items, kDeqThreads), kDeqThreads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(da);
+  return cuda_check("grouped dequant launch");
+}
+
+extern "C" mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void* out, void* stream) {
+  MX_REQUIRE(R >= 0 && C32 > 0, MX_ERR_ARG, "sizes must be R >= 0, C32 > 0");
+  MX_REQUIRE(aligned16(s), MX_ERR_ALIGN, "scales not 16-byte aligned");
+  if (R == 0) return MX_OK;
+  MX_REQUIRE(s && out, MX_ERR_ARG, "null operand");
+  scales_unswizzle_kernel<<<streaming_grid(R * C32, kDeqThreads), kDeqThreads, 0,
+                            static_cast<cudaStream_t>(stream)>>>(static_cast<const uint8_t*>(s), R, C32,
+                                                                 static_cast<uint8_t*>(out));
+  return cuda_check("unswizzle launch");
 }

@@ -43,6 +43,10 @@ _SIGNATURES = {
                                      _vp]),
     "mx_linear_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "mx_cast_ex": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "mx_grouped_mm_bf16": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _vp]),
+    "mx_dequant_dim0": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "mx_dequant_dim0_grouped": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i64, _i64, _vp, _vp]),
+    "mx_scales_unswizzle": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
 }
 
 MX_RCEIL = 0
@@ -188,6 +192,23 @@ def mx_linear_fwd_noalloc(x, w, y, stream=None):
     M, K = x.shape
     N = w.shape[0]
     _call("mx_linear_fwd_noalloc", _p(x), _p(w), M, N, K, _p(y), _stream(stream))
+
+
+def mx_grouped_mm_bf16(a, b, offs, G, mode, out, M, N, K, stream=None):
+    _call("mx_grouped_mm_bf16", _p(a), _p(b), _p(offs), G, mode, _p(out), M, N, K, _stream(stream))
+
+
+def mx_dequant_dim0(q, s, G, R, C, out, stream=None):
+    _call("mx_dequant_dim0", _p(q), _p(s), G, R, C, _p(out), _stream(stream))
+
+
+def mx_dequant_dim0_grouped(q, s, offs, M, K, m_cap, out, stream=None):
+    _call("mx_dequant_dim0_grouped", _p(q), _p(s), _p(offs), offs.numel(), M, K, m_cap, _p(out),
+          _stream(stream))
+
+
+def mx_scales_unswizzle(s, R, C32, out, stream=None):
+    _call("mx_scales_unswizzle", _p(s), R, C32, _p(out), _stream(stream))
 
 
 class WeightCache:
@@ -354,3 +375,121 @@ def cast_floor(x, dims=3):
         qt, st = _u8(C, R, device=x.device), _u8(mx_scale_bytes(C, R // 32), device=x.device)
     mx_cast_ex(x, dims, MX_FLOOR, q, s, qt, st)
     return q, s, qt, st
+
+
+# ------------------------------------------------- backward-override arms --
+def grouped_mm_bf16(a, b, offs):
+    """Row groups (dgrad form): out[rows of g] = a[rows of g] @ b[g]; a [M, K], b [G, K, N]."""
+    a, b = _check_bf16(a), _check_bf16(b)
+    M, K = a.shape
+    G, _, N = b.shape
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    mx_grouped_mm_bf16(a, b, offs, G if offs is not None else 1, MX_GROUPS_M, out, M, N, K)
+    return out
+
+
+def grouped_mm_bf16_wgrad(a, b, offs):
+    """Token groups (wgrad form): out[g] = a[rows of g]^T @ b[rows of g]; a [M, N], b [M, K]."""
+    a, b = _check_bf16(a), _check_bf16(b)
+    M, N = a.shape
+    K = b.shape[1]
+    G = offs.numel() if offs is not None else 1
+    out = torch.empty(G, N, K, dtype=torch.bfloat16, device=a.device)
+    mx_grouped_mm_bf16(a, b, offs, G, MX_GROUPS_K, out, M, N, K)
+    return out
+
+
+def dequant_dim0(q, s):
+    """bf16 values of rowwise-scaled codes q [R, C] or a stack [G, R, C] (s blocked per matrix)."""
+    G, R, C = q.shape if q.dim() == 3 else (1, *q.shape)
+    out = torch.empty(*q.shape, dtype=torch.bfloat16, device=q.device)
+    mx_dequant_dim0(q, s, G, R, C, out)
+    return out
+
+
+def dequant_dim0_grouped(q, s, offs, M):
+    """bf16 rows of a padded grouped dim0 cast, back in the unpadded order [M, K]."""
+    m_cap, K = q.shape
+    out = torch.empty(M, K, dtype=torch.bfloat16, device=q.device)
+    mx_dequant_dim0_grouped(q, s, offs, M, K, m_cap, out)
+    return out
+
+
+def scales_unswizzle(s, R, C32):
+    """Logical scales [R, C32] (uint8) from a blocked scale buffer."""
+    out = torch.empty(R, C32, dtype=torch.uint8, device=s.device)
+    mx_scales_unswizzle(s, R, C32, out)
+    return out
+
+
+BACKWARD_OVERRIDES = (None, "quantized", "high_precision", "dequantized")
+
+
+class MXFP8GroupedMM:
+    """MXFP8 grouped GEMM of an MoE layer, y[rows of g] = x[rows of g] @ w[g]^T.
+
+    forward(x [M, K], w [G, N, K], offs) casts x rowwise into the padded group
+    layout and w in 32x32 tiles, and runs the scaled grouped GEMM; backward(dy)
+    returns (dx, dw). ``backward_override`` selects where the gradients come
+    from (ao "[moe training] Add backward_override to the MXFP8 grouped GEMM",
+    Design notes): None or "quantized" (alias) is the MXFP8 backward;
+    "high_precision" uses bf16 grouped GEMMs on the saved bf16 x and w;
+    "dequantized" uses the same bf16 GEMMs on the forward's codes turned back
+    into bf16 (the gradient of the function the quantized forward computes).
+    Only bf16 operands are accepted; a strided dy is made contiguous first.
+    """
+
+    def __init__(self, backward_override=None):
+        if backward_override not in BACKWARD_OVERRIDES:
+            raise ValueError(f"backward_override must be one of {BACKWARD_OVERRIDES}, "
+                             f"got {backward_override!r}")
+        self.backward_override = None if backward_override == "quantized" else backward_override
+        self._saved = None
+
+    def forward(self, x, w, offs):
+        for name, t in (("x", x), ("w", w)):
+            if t.dtype != torch.bfloat16:
+                raise TypeError(f"MXFP8GroupedMM takes bf16 operands ({name} is {t.dtype})")
+        x, w = x.contiguous(), w.contiguous()
+        M, K = x.shape
+        G, N, _ = w.shape
+        if offs.numel() != G:
+            raise ValueError("offs must hold one end offset per expert")
+        m_cap = mx_padded_rows_capacity(M, G)
+        xq, xs = cast_dim0_grouped(x, offs, m_cap)
+        wq, wsf, wqt, wsd = cast_w32x32(w, transposed=self.backward_override is None)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        mx_grouped_mm(xq, xs, wq, wsf, offs, G, MX_GROUPS_M, y, M, N, K, m_cap)
+        if self.backward_override == "high_precision":
+            self._saved = (x, w, offs)
+        elif self.backward_override == "dequantized":
+            self._saved = (xq, xs, wq, wsf, offs, M, m_cap)
+        else:
+            self._saved = (x, wqt, wsd, offs, m_cap)
+        return y
+
+    def backward(self, dy):
+        if self._saved is None:
+            raise RuntimeError("backward before forward")
+        if dy.dtype != torch.bfloat16:
+            raise TypeError("MXFP8GroupedMM takes a bf16 gradient")
+        dy = dy.contiguous()
+        saved, self._saved = self._saved, None
+        if self.backward_override == "high_precision":
+            x, w, offs = saved
+            return grouped_mm_bf16(dy, w, offs), grouped_mm_bf16_wgrad(dy, x, offs)
+        if self.backward_override == "dequantized":
+            xq, xs, wq, wsf, offs, M, m_cap = saved
+            xd = dequant_dim0_grouped(xq, xs, offs, M)
+            wd = dequant_dim0(wq, wsf)
+            return grouped_mm_bf16(dy, wd, offs), grouped_mm_bf16_wgrad(dy, xd, offs)
+        x, wqt, wsd, offs, m_cap = saved
+        M, K = x.shape
+        G, _, N = wqt.shape
+        dq, ds, dqt, dst = cast_2d_grouped(dy, offs, m_cap)
+        xqt, xst = cast_dim1_grouped(x, offs, m_cap)
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
+        mx_grouped_mm(dq, ds, wqt, wsd, offs, G, MX_GROUPS_M, dx, M, K, N, m_cap)
+        dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=x.device)
+        mx_grouped_mm(dqt, dst, xqt, xst, offs, G, MX_GROUPS_K, dw, M, N, K, m_cap)
+        return dx, dw
