@@ -254,6 +254,61 @@ def cast_sweep(mx, device, flush):
     return out
 
 
+def override_arms(mx, step, flush, peaks):
+    """Backward of the same MoE layer under the two backward overrides.
+
+    high_precision: dX = dY_g W_g and dW_g = dY_g^T X_g as bf16 grouped GEMMs
+    on the bf16 operands; dequantized: the same GEMMs on the forward's codes
+    dequantized to bf16 (X from the padded dim0 codes, W from the 32x32 codes).
+    Times are medians of 10 L2-flushed repetitions of each launch.
+    """
+    import torch
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2] * 1e-3
+
+    dev = step.x.device
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=dev)
+    xd = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    wd = torch.empty(G, N, K, dtype=torch.bfloat16, device=dev)
+    step.run()     # the forward codes of this step are what the dequantized arm reads
+    t_dgrad = timed(lambda: mx.mx_grouped_mm_bf16(step.dy, step.w, step.offs, G, mx.MX_GROUPS_M, dx, M, K, N))
+    t_wgrad = timed(lambda: mx.mx_grouped_mm_bf16(step.dy, step.x, step.offs, G, mx.MX_GROUPS_K, dw, M, N, K))
+    t_dqx = timed(lambda: mx.mx_dequant_dim0_grouped(step.xq, step.xs, step.offs, M, K, step.cap, xd))
+    t_dqw = timed(lambda: mx.mx_dequant_dim0(step.wq, step.wsf, G, N, K, wd))
+    mx.mx_device_error()
+    bf16_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    deq_gbs = lambda elems, sec: round(elems * (3 + 1 / 32) / sec / 1e9, 1)
+    return {
+        "high_precision": {
+            "backward_ms": round((t_dgrad + t_wgrad) * 1e3, 4),
+            "dgrad_bf16_tflops": round(GEMM_FLOPS / t_dgrad / 1e12, 1),
+            "wgrad_bf16_tflops": round(GEMM_FLOPS / t_wgrad / 1e12, 1),
+            "frac_of_measured_bf16_sustained": round(2 * GEMM_FLOPS / (t_dgrad + t_wgrad) / 1e12 / bf16_peak, 3),
+        },
+        "dequantized": {
+            "backward_ms": round((t_dgrad + t_wgrad + t_dqx + t_dqw) * 1e3, 4),
+            "dequant_x_gbs": deq_gbs(M * K, t_dqx),
+            "dequant_w_gbs": deq_gbs(G * N * K, t_dqw),
+            "dequant_frac_of_measured_hbm": round(deq_gbs(G * N * K, t_dqw) / hbm, 3),
+        },
+    }
+
+
 # ------------------------------------------------------ CPU (the oracle) --
 def oracle_sample(tokens=512, seed=0):
     """One bounded sample of the step on the host: one expert, `tokens` tokens.
@@ -336,6 +391,7 @@ def main(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-sweep", action="store_true", help="skip the cast bandwidth sweep")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--ref-tokens", type=int, default=512)
     args = p.parse_args(argv)
@@ -423,6 +479,10 @@ def main(argv=None):
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         casts = {k: {"gbs": v, "frac_of_measured_hbm": round(v / hbm, 3), "frac_of_8tbs_spec": round(v / 8000, 3)}
                  for k, v in casts.items()}
+    arms = None
+    if not args.no_arms:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        arms = override_arms(mx, step, flush, peaks)
 
     if rank != 0:
         if world > 1:
@@ -445,6 +505,7 @@ def main(argv=None):
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
         "casts": casts,
+        "backward_overrides": arms,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

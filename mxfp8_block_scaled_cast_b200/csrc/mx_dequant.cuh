@@ -13,9 +13,10 @@
 // cvt.rn.bf16x2.f32 rounds once. A NaN code or the E8M0 NaN byte 255 gives
 // NaN.
 //
-// Memory bound: one thread per 32-element block reads 32 code bytes and one
-// scale byte and writes 64 bytes; consecutive threads take consecutive blocks
-// of a row, so each warp reads 1 KB and writes 2 KB contiguously.
+// Memory bound (1 byte read, 2 bytes written per element): a warp takes 1024
+// consecutive elements of a row in four passes in which lane i converts 8
+// codes, so each load instruction of the warp reads 256 contiguous bytes and
+// each store writes 512.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -109,13 +110,19 @@ dequant_dim0_kernel(const DequantArgs a) {
     __syncthreads();
     if (s_bad) return;
   }
+  // Work item = one row and a chunk of 32 consecutive blocks (1024 elements)
+  // of it, taken by one warp. The row's source and scale base are found once
+  // per item.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t cb = a.C / kBlock;                      // blocks per row
-  const int64_t total = a.rows_out * cb;
+  const int64_t chunks = ceil_div(cb, 32);
+  const int64_t items = a.rows_out * chunks;
   const int64_t sc_tiles = ceil_div(cb, 4);             // 4-column scale tiles per band
   const int64_t layout_bytes = ceil_to(a.layout_rows, 128) * ceil_to(cb, 4);
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = i / cb, c = i % cb;
+  const int64_t wstride = int64_t(gridDim.x) * (kDeqThreads / 32);
+  for (int64_t it = int64_t(blockIdx.x) * (kDeqThreads / 32) + warp; it < items; it += wstride) {
+    const int64_t r = it / chunks;
+    const int64_t c0 = (it - r * chunks) * 32;            // first block of the chunk
     int64_t src_row, srow;
     const uint8_t* sbase = a.s;
     if (kGrouped) {
@@ -128,20 +135,35 @@ dequant_dim0_kernel(const DequantArgs a) {
       src_row = s_pstart[lo] + (r - start);
       srow = src_row;
     } else {
+      const int64_t layout = r / a.layout_rows;
       src_row = r;
-      sbase += (r / a.layout_rows) * layout_bytes;
-      srow = r % a.layout_rows;
+      sbase += layout * layout_bytes;
+      srow = r - layout * a.layout_rows;
     }
-    const uint32_t b = sbase[(srow >> 7) * sc_tiles * 512 + (c >> 2) * 512 + in_tile(uint32_t(srow & 127), uint32_t(c))];
-    const float scale = e8m0_value(b);
-    const uint4* qp = reinterpret_cast<const uint4*>(a.q + src_row * a.C + c * kBlock);
-    const uint4 q0 = ld_stream16(qp), q1 = ld_stream16(qp + 1);
-    uint4* op = reinterpret_cast<uint4*>(a.out + r * a.C + c * kBlock);
-    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const uint8_t* qrow = a.q + src_row * a.C;
+    __nv_bfloat16* orow = a.out + r * a.C;
+    const int64_t e0 = c0 * kBlock;                     // first element of the chunk
+    // four passes of 256 elements: lane i takes 8 codes (8 bytes in, 16 bytes
+    // out), so every load and store instruction of the warp is contiguous
+    uint2 qv[4];
+    uint32_t bv[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint2 lo = dequant4(w[2 * j], scale), hi = dequant4(w[2 * j + 1], scale);
-      op[j] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    for (int k = 0; k < 4; ++k) {
+      const int64_t e = e0 + k * 256 + lane * 8;
+      if (e < a.C) {
+        qv[k] = *reinterpret_cast<const uint2*>(qrow + e);
+        const int64_t c = e >> 5;
+        bv[k] = sbase[(srow >> 7) * sc_tiles * 512 + (c >> 2) * 512 + in_tile(uint32_t(srow & 127), uint32_t(c))];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t e = e0 + k * 256 + lane * 8;
+      if (e < a.C) {
+        const float scale = e8m0_value(bv[k]);
+        const uint2 lo = dequant4(qv[k].x, scale), hi = dequant4(qv[k].y, scale);
+        *reinterpret_cast<uint4*>(orow + e) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      }
     }
   }
 }

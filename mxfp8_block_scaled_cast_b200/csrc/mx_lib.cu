@@ -295,13 +295,17 @@ mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const H
   return cuda_check("bf16 gemm launch");
 }
 
-// Grid for the grid-stride memory-bound kernels: enough CTAs to fill every SM
-// several times, never more than the work.
-unsigned streaming_grid(int64_t items, int threads) {
-  int dev = 0, sms = 148;
+// Grid for a grid-stride memory-bound kernel: every CTA resident at once
+// (SMs x resident CTAs per SM, from the occupancy calculator), never more
+// CTAs than the work needs.
+template <typename Kernel>
+unsigned streaming_grid(Kernel kernel, int64_t items, int threads) {
+  int dev = 0, sms = 148, per_sm = 1;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
   const int64_t need = ceil_div(items, threads);
-  const int64_t cap = int64_t(sms) * 8;
+  const int64_t cap = int64_t(sms) * per_sm;
   return unsigned(need < cap ? need : cap);
 }
 
@@ -807,8 +811,8 @@ extern "C" mx_status mx_dequant_dim0(const void* q, const void* s, int64_t G, in
   da.rows_out = G * R;
   da.C = C;
   da.layout_rows = R;
-  const int64_t items = da.rows_out * (C / kBlock);
-  dequant_dim0_kernel<false><<<streaming_grid(items, kDeqThreads), kDeqThreads, 0,
+  const int64_t items = da.rows_out * ceil_div(C / kBlock, 32) * 32;
+  dequant_dim0_kernel<false><<<streaming_grid(dequant_dim0_kernel<false>, items, kDeqThreads), kDeqThreads, 0,
                                static_cast<cudaStream_t>(stream)>>>(da);
   return cuda_check("dequant launch");
 }
@@ -831,8 +835,8 @@ extern "C" mx_status mx_dequant_dim0_grouped(const void* q, const void* s, const
   da.offs = offs;
   da.G = G;
   da.m_cap = m_cap;
-  const int64_t items = M * (K / kBlock);
-  dequant_dim0_kernel<true><<<streaming_grid(items, kDeqThreads), kDeqThreads, 0,
+  const int64_t items = M * ceil_div(K / kBlock, 32) * 32;
+  dequant_dim0_kernel<true><<<streaming_grid(dequant_dim0_kernel<true>, items, kDeqThreads), kDeqThreads, 0,
                               static_cast<cudaStream_t>(stream)>>>(da);
   return cuda_check("grouped dequant launch");
 }
@@ -842,7 +846,7 @@ extern "C" mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, 
   MX_REQUIRE(aligned16(s), MX_ERR_ALIGN, "scales not 16-byte aligned");
   if (R == 0) return MX_OK;
   MX_REQUIRE(s && out, MX_ERR_ARG, "null operand");
-  scales_unswizzle_kernel<<<streaming_grid(R * C32, kDeqThreads), kDeqThreads, 0,
+  scales_unswizzle_kernel<<<streaming_grid(scales_unswizzle_kernel, R * C32, kDeqThreads), kDeqThreads, 0,
                             static_cast<cudaStream_t>(stream)>>>(static_cast<const uint8_t*>(s), R, C32,
                                                                  static_cast<uint8_t*>(out));
   return cuda_check("unswizzle launch");
