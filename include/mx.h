@@ -9,8 +9,8 @@
  *     the MXFP8 grouped GEMM", Summary and Design notes), the fused
  *     rowwise+columnwise cast and 32x32 weight blocks (torchtitan PR #5334,
  *     description); scales are written straight into the blocked layout the
- *     block-scaled MMA reads ("no need for scale rearrangements since swizzled
- *     layouts are directly output", same page);
+ *     block-scaled MMA reads, so no separate scale rearrangement pass is
+ *     needed (same page);
  *   - the group pad path ("pad_token_groups_for_grouped_mm", ao
  *     backward_override PR, Known follow-ups; "pad/unpad" and "M-groups /
  *     K-groups scale rearrange" kernels, ao PR #4705 stack list);
@@ -124,8 +124,8 @@ MX_API mx_status mx_cast_w32x32(const void* w, int64_t G, int64_t N, int64_t K,
                          void* stream);
 
 /* Scale rule selector of mx_cast_ex. RCEIL is the rule of every other entry
- * point; FLOOR (ao backward_override PR, Known follow-ups: "FLOOR is
- * reachable") is scale 2^(floor(log2 amax) - 8), with which scaled elements
+ * point; FLOOR (ao backward_override PR, Known follow-ups: the other scale
+ * rule, reachable there but untested) is scale 2^(floor(log2 amax) - 8), with which scaled elements
  * can exceed 448 and saturate to +-448. */
 #define MX_RCEIL 0
 #define MX_FLOOR 1
@@ -197,8 +197,9 @@ MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q
  * notes: the "high_precision" arm computes dgrad and wgrad of the grouped GEMM
  * with two plain bf16 grouped GEMMs over the saved, unpadded bf16 operands;
  * the "dequantized" arm runs the same two GEMMs on the forward's quantized
- * operands turned back into bf16 (it needs logical scales, for which the page
- * notes that "no unswizzler exists"; mx_scales_unswizzle is one).
+ * operands turned back into bf16 (it needs logical scales, and the page notes
+ * that no kernel turned blocked scales back into logical ones;
+ * mx_scales_unswizzle does).
  *
  * bf16 grouped GEMM, fp32 accumulation on the tensor cores, bf16 output
  * (round to nearest even); deterministic (no split-K, no atomics). Groups are
@@ -240,7 +241,7 @@ MX_API mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void
 
 /* ------------------------------------------------------ MXFP8 linear -----
  * Dense MXFP8 linear (ao PR #4705, "MXFP8Linear training paths"; torchtitan
- * PR #5334, "a single API for dense and grouped mxfp8 linears"):
+ * PR #5334, description: one entry point for dense and grouped MXFP8 linears):
  *   forward  y  [M, N] = x [M, K] w [N, K]^T   x cast 1x32 (dim0), w 32x32
  *   backward dx [M, K] = dy [M, N] w           dy cast 1x32 along N
  *            dw [N, K] = dy^T x                dy and x cast 32x1 along M

@@ -2,8 +2,8 @@
 // the "dequantized" backward arm (ao "[moe training] Add backward_override to
 // the MXFP8 grouped GEMM", Design notes: that arm differentiates the
 // quantized-forward function, so it needs the forward's operands back in
-// bf16, and it needs logical (pre-blocking) scales, for which "no unswizzler
-// exists").
+// bf16, and it needs logical (pre-blocking) scales, which the page notes no
+// existing kernel recovered from the blocked layout).
 //
 // Element value: e4m3(q) * 2^(b - 127) rounded to bf16 (nearest, ties to
 // even). The E4M3 pair is widened exactly by cvt.rn.f16x2.e4m3x2 (every E4M3

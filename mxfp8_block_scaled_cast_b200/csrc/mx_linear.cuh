@@ -1,8 +1,8 @@
 // MXFP8 linear forward / dgrad / wgrad and the per-weight quantization cache.
 //
 // The linear composes the casts and the grouped GEMM at one dense group
-// (ao PR #4705, "MXFP8Linear training paths"; torchtitan PR #5334, "a single
-// API for dense and grouped mxfp8 linears"):
+// (ao PR #4705, "MXFP8Linear training paths"; torchtitan PR #5334,
+// description: one entry point serves dense and grouped MXFP8 linears):
 //   forward  Y  = X W^T   X cast 1x32 along K, W cast with 32x32 blocks
 //   dgrad    dX = dY W    dY cast 1x32 along N, W^T codes of the same 32x32 cast
 //   wgrad    dW = dY^T X  dY and X cast 32x1 along the token axis

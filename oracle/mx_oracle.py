@@ -16,8 +16,8 @@ What it computes, and where each step comes from
   block is the smallest power of two 2**e with 448 * 2**e >= amax, stored as
   the E8M0 byte b = e + 127 clamped to [0, 254]. 448 is the largest finite
   E4M3 value. A block whose amax is 0 gets b = 0.
-* FLOOR scale rule (ao backward_override PR, Known follow-ups, "FLOOR is
-  reachable"): scale 2**(floor(log2(amax)) - 8); saturation to 448 is live.
+* FLOOR scale rule (ao backward_override PR, Known follow-ups: the other
+  scale rule, reachable but untested there): scale 2**(floor(log2(amax)) - 8); saturation to 448 is live.
 * Element cast: q = round-to-nearest-even, saturating E4M3 encoding of
   x * 2**(127 - b), with the sign of zero kept.
 * Block geometry: rowwise "dim0" (1x32 along the contiguous axis), columnwise
@@ -154,8 +154,8 @@ def rceil_e8m0(amax) -> np.ndarray:
 def floor_e8m0(amax) -> np.ndarray:
     """E8M0 byte of the FLOOR scale of blocks with the given amax.
 
-    FLOOR is the other scale rule the ao backward_override page names ("FLOOR
-    is reachable but untested", Known follow-ups). Reading: the OCP MX rule,
+    FLOOR is the other scale rule the ao backward_override page names (Known
+    follow-ups: it can be selected there but has no parity test). Reading: the OCP MX rule,
     scale = 2**(floor(log2(amax)) - 8), 8 being the exponent of the largest
     power of two representable in E4M3 (256 <= 448 < 512); b = that exponent
     + 127 clamped to [0, 254]; amax == 0 gives b = 0. Scaled elements can then
