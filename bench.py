@@ -7,11 +7,11 @@ default", roofline benchmark at K=N=4096, G=8, M=16384), run through every
 cast and GEMM of the path:
 
   1. X   [16384, 4096]      dim0 cast into padded groups (pad path)
-  2. W   [8, 4096, 4096]    32x32 cast (forward codes + transposed codes)
+  2. W   [8, 4096, 4096]    32x32 cast (codes + forward and dgrad scale views)
   3. fwd grouped GEMM       Y  = X_g W_g^T          (M groups)
   4. dY  [16384, 4096]      fused dim0 + dim1 cast into padded groups
   5. X                      dim1 cast into padded groups
-  6. dgrad grouped GEMM     dX = dY_g W_g           (M groups)
+  6. dgrad grouped GEMM     dX = dY_g W_g           (M groups, W codes read MN-major)
   7. wgrad grouped GEMM     dW_g = dY_g^T X_g       (K groups)
 
 value = 3 * 2*M*N*K FLOPs per step / step time (TFLOP/s, whole job). Inputs
@@ -174,7 +174,7 @@ class MoEStep:
         self.xq, self.xs = u8(cap, K), u8(mx.mx_scale_bytes(cap, K // 32))
         self.xqt, self.xst = u8(K, cap), u8(mx.mx_scale_bytes(K, cap // 32))
         self.wq, self.wsf = u8(G, N, K), u8(G * mx.mx_scale_bytes(N, K // 32))
-        self.wqt, self.wsd = u8(G, K, N), u8(G * mx.mx_scale_bytes(K, N // 32))
+        self.wsd = u8(G * mx.mx_scale_bytes(K, N // 32))
         self.dq, self.ds = u8(cap, N), u8(mx.mx_scale_bytes(cap, N // 32))
         self.dqt, self.dst = u8(N, cap), u8(mx.mx_scale_bytes(N, cap // 32))
         self.y, self.dx, self.dw = bf(M, N), bf(M, K), bf(G, N, K)
@@ -184,13 +184,13 @@ class MoEStep:
     def run(self, timed_gemms=False):
         mx, t = self.mx, self.torch
         mx.mx_cast_dim0_grouped(self.x, self.offs, self.cap, self.xq, self.xs)
-        mx.mx_cast_w32x32(self.w, self.wq, self.wsf, self.wqt, self.wsd)
+        mx.mx_cast_w32x32(self.w, self.wq, self.wsf, None, self.wsd)
         gemms = (
             lambda: mx.mx_grouped_mm(self.xq, self.xs, self.wq, self.wsf, self.offs, G, mx.MX_GROUPS_M, self.y,
                                      M, N, K, self.cap),
             None,
-            lambda: mx.mx_grouped_mm(self.dq, self.ds, self.wqt, self.wsd, self.offs, G, mx.MX_GROUPS_M, self.dx,
-                                     M, K, N, self.cap),
+            lambda: mx.mx_grouped_mm(self.dq, self.ds, self.wq, self.wsd, self.offs, G, mx.MX_GROUPS_M_KN,
+                                     self.dx, M, K, N, self.cap),
             lambda: mx.mx_grouped_mm(self.dqt, self.dst, self.xqt, self.xst, self.offs, G, mx.MX_GROUPS_K,
                                      self.dw, M, N, K, self.cap),
         )

@@ -177,6 +177,13 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  *   out bf16 [M, N]; rows of the padded layout that are padding are not read
  *       into the output (the unpad is fused into the store).
  *   N a multiple of 256, K a multiple of 128.
+ * mode MX_GROUPS_M_KN (dgrad straight from the forward's weight codes): as
+ *   MX_GROUPS_M with B codes stored [G, K, N] (N contiguous; read by the MMA
+ *   as an MN-major operand, so no transposed copy is needed) and b_s G
+ *   concatenated blocked(N, K/32) buffers, i.e.
+ *   out[start_g + i, n] = sum_k A[p_g + i, k] B[g, k, n].
+ *   For dX = dY W of a weight W [G, Nw, Kw] cast 32x32: B = its codes q,
+ *   b_s = its s_dgrad view, N = Kw, K = Nw.
  * mode MX_GROUPS_K (wgrad; groups split the contraction, "K groups"):
  *   out[g, n, k] = sum over the tokens t of group g of A[n, t] B[k, t]
  *   a_q [N, L], a_s blocked(N, L/32); b_q [K, L], b_s blocked(K, L/32) with
@@ -188,6 +195,7 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  * Invalid offsets set the device flag and leave the output unwritten. */
 #define MX_GROUPS_M 0
 #define MX_GROUPS_K 1
+#define MX_GROUPS_M_KN 2
 MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
                                const int32_t* offs, int32_t G, int32_t mode, void* out,
                                int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);

@@ -6,11 +6,14 @@
 // wgrad of _MXFP8GroupedMM; ao PR #4705, "MXFP8 MoE grouped-mm"):
 //
 //   M-groups (forward, dgrad): out[rows of g, :] = A[padded rows of g, :] * B[g]^T
-//     A codes [rows_a, K] (padded token rows), B codes [G, N, K], out [M, N].
+//     A codes [rows_a, K] (padded token rows), B codes [G, N, K], out [M, N];
+//     or B codes [G, K, N] read MN-major (the dgrad from the forward's weight
+//     codes, no transposed copy).
 //   K-groups (wgrad):          out[g] = A[:, tokens of g] * B[:, tokens of g]^T
 //     A codes [N, m_cap], B codes [K, m_cap] (padded token columns), out [G, N, K].
 //
-// Both operands are K-major E4M3 with blocked E8M0 scales; each token group
+// Operands are E4M3 with blocked E8M0 scales along K (K-major, except B in
+// the MN-major M-groups form); each token group
 // starts on a 128-row boundary of the padded layout (the pad path), so every
 // 128-row scale tile and every 128-wide K tile belongs to one group.
 //
@@ -92,7 +95,9 @@ static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 // packed in each TMEM scale column this MMA uses.
 constexpr uint32_t kIdescBase = (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kPairM >> 4) << 24);
 
-enum GemmMode : int { kGroupsM = 0, kGroupsK = 1 };
+// kGroupsMKn: M groups with B stored [G, K, N] (N contiguous), read as an
+// MN-major operand -- the dgrad straight from the forward's weight codes.
+enum GemmMode : int { kGroupsM = 0, kGroupsK = 1, kGroupsMKn = 2 };
 
 struct GemmArgs {
   const int32_t* offs;         // cumulative group ends, or null for one dense group
@@ -119,7 +124,7 @@ template <int kMode>
 __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a, const int32_t* ends,
                                                 const int32_t* pstart, const int32_t* tstart) {
   TileInfo t;
-  if (kMode == kGroupsM) {
+  if (kMode != kGroupsK) {
     const int64_t nt = a.N / kBN;
     const int64_t mt = tile / nt;
     t.n0 = (tile % nt) * kBN;
@@ -132,7 +137,7 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
     t.m0 = pstart[t.g] + (mt - tstart[t.g]) * kPairM;
     t.nk = int(a.K / kBK);
     t.kt0 = 0;
-    t.b_row0 = int64_t(t.g) * a.N + t.n0;
+    t.b_row0 = kMode == kGroupsMKn ? int64_t(t.g) * a.K : int64_t(t.g) * a.N + t.n0;
     t.b_chunk0 = int64_t(t.g) * a.b_sc_group_chunks + (t.n0 / kCtaM) * a.b_sc_tiles;
   } else {
     const int64_t nt = a.K / kBN, mt = a.N / kPairM;
@@ -336,7 +341,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     }
     if (lane == 0) {
       int64_t total;
-      if (kMode == kGroupsM) total = bad ? 0 : int64_t(tstart[G]) * (args.N / kBN);
+      if (kMode != kGroupsK) total = bad ? 0 : int64_t(tstart[G]) * (args.N / kBN);
       else total = bad ? 0 : int64_t(G) * (args.N / kPairM) * (args.K / kBN);
       if (bad && rank == 0) flag_error(kErrOffsets);
       info[0] = total;
@@ -373,7 +378,11 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
             const uint32_t lb = mapa_shared(fb, 0);
             tma_load_2d_pair(sbase + kOffA + stage * kABytes, &map_a, kk * kBK, a_row, lb);
-            tma_load_2d_pair(sbase + kOffB + stage * kBBytes, &map_b, kk * kBK, b_row, lb);
+            if (kMode == kGroupsMKn)     // 128 K rows x this CTA's 128 N columns
+              tma_load_2d_pair(sbase + kOffB + stage * kBBytes, &map_b, int32_t(t.n0 + (kBN / 2) * rank),
+                               int32_t(t.b_row0 + int64_t(kk) * kBK), lb);
+            else
+              tma_load_2d_pair(sbase + kOffB + stage * kBBytes, &map_b, kk * kBK, b_row, lb);
             tma_load_2d_pair(sbase + kOffSfa + stage * kSfaBytes, &map_sfa, 0, int32_t(sfa_chunk0 + kk), lb);
             tma_load_2d_pair(sbase + kOffSfb + stage * kSfbBytes, &map_sfb, 0, int32_t(t.b_chunk0 + kk), lb);
             tma_load_2d_pair(sbase + kOffSfb + stage * kSfbBytes + 512, &map_sfb, 0,
@@ -406,7 +415,13 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       // another stage or K block is one 64-bit add; the issue loop below is
       // then a handful of instructions per MMA and keeps the tensor pipe fed.
       const uint64_t a_desc0 = smem_desc(sbase + kOffA, 16, 1024, 2);
-      const uint64_t b_desc0 = smem_desc(sbase + kOffB, 16, 1024, 2);
+      // B MN-major (kGroupsMKn): one 128-byte swizzle atom of N per CTA, K rows
+      // 128 bytes apart in 8-row groups 1024 bytes apart, so a 32-deep K block
+      // is four groups (+4096 bytes); K-major: +32 bytes per K block.
+      const uint64_t b_desc0 = kMode == kGroupsMKn ? smem_desc(sbase + kOffB, kBBytes, 1024, 2)
+                                                   : smem_desc(sbase + kOffB, 16, 1024, 2);
+      constexpr uint64_t kBStep = kMode == kGroupsMKn ? (4096 >> 4) : (32 >> 4);
+      constexpr uint32_t kIdesc = kIdescBase | (kMode == kGroupsMKn ? (1u << 16) : 0u);
       const uint64_t sfa_desc0 = smem_desc(sbase + kOffSfa, 0, 128, 0);
       const uint64_t sfb_desc0 = smem_desc(sbase + kOffSfb, 0, 128, 0);
       for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
@@ -437,10 +452,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             tmem_cp_32x128b_x4_pair(sfb_t, sfb_desc0 + uint64_t((stage * kSfbBytes) >> 4));
             tmem_cp_32x128b_x4_pair(sfb_t + 4, sfb_desc0 + uint64_t((stage * kSfbBytes + 512) >> 4));
             // K block k of the 128-deep stage: +32 bytes (2 in the >>4 field)
-            mma_mxf8_pair(d_tmem, ad, bd, kIdescBase, sfa_t, sfb_t, acc0);
-            mma_mxf8_pair(d_tmem, ad + 2, bd + 2, kIdescBase | (1u << 4) | (1u << 29), sfa_t, sfb_t, 1u);
-            mma_mxf8_pair(d_tmem, ad + 4, bd + 4, kIdescBase | (2u << 4) | (2u << 29), sfa_t, sfb_t, 1u);
-            mma_mxf8_pair(d_tmem, ad + 6, bd + 6, kIdescBase | (3u << 4) | (3u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad, bd, kIdesc, sfa_t, sfb_t, acc0);
+            mma_mxf8_pair(d_tmem, ad + 2, bd + kBStep, kIdesc | (1u << 4) | (1u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 4, bd + 2 * kBStep, kIdesc | (2u << 4) | (2u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 6, bd + 3 * kBStep, kIdesc | (3u << 4) | (3u << 29), sfa_t, sfb_t, 1u);
             tc_commit_pair(empty_bar(stage));
           }
           __syncwarp();
@@ -472,7 +487,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
       const int64_t row = t.m0 + kCtaM * rank + r;
       __nv_bfloat16* dst = nullptr;
-      if (kMode == kGroupsM) {
+      if (kMode != kGroupsK) {
         const int64_t start = t.g ? ends[t.g - 1] : 0;
         const int64_t local = row - pstart[t.g];
         if (local < ends[t.g] - start) dst = a.out + (start + local) * a.N + t.n0;

@@ -451,7 +451,8 @@ mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K, const int32_t*
 mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
                         const int32_t* offs, int32_t G, int32_t mode, void* out, int64_t M, int64_t N,
                         int64_t K, int64_t m_cap, void* stream) {
-  MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K, MX_ERR_ARG, "unknown mode %d", mode);
+  MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K || mode == MX_GROUPS_M_KN, MX_ERR_ARG, "unknown mode %d",
+             mode);
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   if (offs != nullptr) {
     MX_REQUIRE(G >= 1 && G <= kMaxGroups, MX_ERR_ARG, "G = %d outside [1, %d]", G, kMaxGroups);
@@ -474,7 +475,7 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
   ga.N = N;
   ga.K = K;
   CUtensorMap map_a, map_b, map_sa, map_sb;
-  if (mode == MX_GROUPS_M) {
+  if (mode != MX_GROUPS_K) {
     MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
     MX_REQUIRE(K % kBK == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 128", (long long)K);
     const int64_t rows_a = offs ? m_cap : M;
@@ -485,10 +486,14 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
     ga.b_sc_tiles = K / kBK;
     ga.b_sc_group_chunks = scale_bytes(N, K / kBlock) / 512;
     MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kCtaM));
-    MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN / 2));
+    if (mode == MX_GROUPS_M_KN)
+      MX_TRY(make_map(&map_b, b_q, uint64_t(N), uint64_t(G) * uint64_t(K), kBK));
+    else
+      MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN / 2));
     MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(rows_a, K / kBlock) / 512)));
     MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(G) * uint64_t(ga.b_sc_group_chunks)));
     const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * (N / kBN);
+    if (mode == MX_GROUPS_M_KN) return launch_gemm<kGroupsMKn>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
     return launch_gemm<kGroupsM>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
   }
   MX_REQUIRE(N % kPairM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
@@ -567,7 +572,7 @@ mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, ui
                        WeightView* out, cudaStream_t st) {
   if (cache == nullptr) {
     *out = carve_weight(ws_tail, N, K);
-    return mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, out->qt, out->s_dgrad, st);
+    return mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, nullptr, out->s_dgrad, st);
   }
   std::lock_guard<std::mutex> lk(cache->mu);
   mx_wcache::Entry* e = nullptr;
@@ -592,7 +597,7 @@ mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, ui
   }
   *out = carve_weight(e->q, N, K);
   e->valid = false;
-  MX_TRY(mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, out->qt, out->s_dgrad, st));
+  MX_TRY(mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, nullptr, out->s_dgrad, st));
   e->version = version;
   e->valid = true;
   return MX_OK;
@@ -640,7 +645,7 @@ mx_status mx_linear_bwd(const void* dy, const void* x, const void* w, int64_t M,
   }
   MX_TRY(mx_cast_2d(dy, M, N, dyq, dys, dyqt, dyst, stream));
   MX_TRY(mx_cast_dim1(x, M, K, xqt, xst, stream));
-  MX_TRY(mx_grouped_mm(dyq, dys, wv.qt, wv.s_dgrad, nullptr, 1, MX_GROUPS_M, dx, M, K, N, 0, stream));
+  MX_TRY(mx_grouped_mm(dyq, dys, wv.q, wv.s_dgrad, nullptr, 1, MX_GROUPS_M_KN, dx, M, K, N, 0, stream));
   return mx_grouped_mm(dyqt, dyst, xqt, xst, nullptr, 1, MX_GROUPS_K, dw, M, N, K, 0, stream);
 }
 

@@ -4,7 +4,8 @@
 // (ao PR #4705, "MXFP8Linear training paths"; torchtitan PR #5334,
 // description: one entry point serves dense and grouped MXFP8 linears):
 //   forward  Y  = X W^T   X cast 1x32 along K, W cast with 32x32 blocks
-//   dgrad    dX = dY W    dY cast 1x32 along N, W^T codes of the same 32x32 cast
+//   dgrad    dX = dY W    dY cast 1x32 along N, the same 32x32 codes read
+//                         MN-major with the dgrad scale view
 //   wgrad    dW = dY^T X  dY and X cast 32x1 along the token axis
 // dY is cast once with the fused rowwise+columnwise kernel.
 //
@@ -31,7 +32,6 @@ struct mx_wcache {
     bool valid = false;
     uint8_t* q = nullptr;        // [N, K]
     uint8_t* s_fwd = nullptr;    // blocked(N, K/32)
-    uint8_t* qt = nullptr;       // [K, N]
     uint8_t* s_dgrad = nullptr;  // blocked(K, N/32)
   };
   std::vector<Entry> entries;
@@ -41,21 +41,21 @@ struct mx_wcache {
 
 namespace mx {
 
-// Device bytes of one 32x32-quantized weight (codes, both scale views and the
-// transposed codes), each piece rounded up to 256 bytes.
+// Device bytes of one 32x32-quantized weight (codes and both scale views),
+// each piece rounded up to 256 bytes. The dgrad reads the same codes as an
+// MN-major operand, so no transposed copy is kept.
 inline int64_t wq_bytes(int64_t N, int64_t K) {
-  return ceil_to(N * K, 256) * 2 + ceil_to(scale_bytes(N, K / kBlock), 256) + ceil_to(scale_bytes(K, N / kBlock), 256);
+  return ceil_to(N * K, 256) + ceil_to(scale_bytes(N, K / kBlock), 256) + ceil_to(scale_bytes(K, N / kBlock), 256);
 }
 
 struct WeightView {
-  uint8_t *q, *s_fwd, *qt, *s_dgrad;
+  uint8_t *q, *s_fwd, *s_dgrad;
 };
 
 inline WeightView carve_weight(uint8_t* base, int64_t N, int64_t K) {
   WeightView v;
   v.q = base;
-  v.qt = v.q + ceil_to(N * K, 256);
-  v.s_fwd = v.qt + ceil_to(N * K, 256);
+  v.s_fwd = v.q + ceil_to(N * K, 256);
   v.s_dgrad = v.s_fwd + ceil_to(scale_bytes(N, K / kBlock), 256);
   return v;
 }

@@ -57,6 +57,7 @@ MX_LINEAR_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 MX_GROUPS_M = 0
 MX_GROUPS_K = 1
+MX_GROUPS_M_KN = 2
 
 _lib = None
 
@@ -275,14 +276,19 @@ def cast_2d(x):
     return q, s, qt, st
 
 
-def cast_w32x32(w, transposed=True):
+def cast_w32x32(w, transposed=True, dgrad_scales=None):
+    """32x32 cast: (q, s_fwd, qt or None, s_dgrad or None).
+
+    The dgrad scale view is written when ``dgrad_scales`` is true (default: with
+    the transposed codes); the MN-major dgrad needs it without ``qt``."""
     w = _check_bf16(w)
+    dgrad_scales = transposed if dgrad_scales is None else dgrad_scales
     G, N, K = w.shape if w.dim() == 3 else (1, *w.shape)
     dev = w.device
     q = _u8(*w.shape, device=dev)
     s_fwd = _u8(G * mx_scale_bytes(N, K // 32), device=dev)
     qt = _u8(*((G, K, N) if w.dim() == 3 else (K, N)), device=dev) if transposed else None
-    s_dgrad = _u8(G * mx_scale_bytes(K, N // 32), device=dev) if transposed else None
+    s_dgrad = _u8(G * mx_scale_bytes(K, N // 32), device=dev) if dgrad_scales else None
     mx_cast_w32x32(w, q, s_fwd, qt, s_dgrad)
     return q, s_fwd, qt, s_dgrad
 
@@ -457,7 +463,7 @@ class MXFP8GroupedMM:
             raise ValueError("offs must hold one end offset per expert")
         m_cap = mx_padded_rows_capacity(M, G)
         xq, xs = cast_dim0_grouped(x, offs, m_cap)
-        wq, wsf, wqt, wsd = cast_w32x32(w, transposed=self.backward_override is None)
+        wq, wsf, _, wsd = cast_w32x32(w, transposed=False, dgrad_scales=self.backward_override is None)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
         mx_grouped_mm(xq, xs, wq, wsf, offs, G, MX_GROUPS_M, y, M, N, K, m_cap)
         if self.backward_override == "high_precision":
@@ -465,7 +471,7 @@ class MXFP8GroupedMM:
         elif self.backward_override == "dequantized":
             self._saved = (xq, xs, wq, wsf, offs, M, m_cap)
         else:
-            self._saved = (x, wqt, wsd, offs, m_cap)
+            self._saved = (x, wq, wsd, offs, m_cap)
         return y
 
     def backward(self, dy):
@@ -483,13 +489,13 @@ class MXFP8GroupedMM:
             xd = dequant_dim0_grouped(xq, xs, offs, M)
             wd = dequant_dim0(wq, wsf)
             return grouped_mm_bf16(dy, wd, offs), grouped_mm_bf16_wgrad(dy, xd, offs)
-        x, wqt, wsd, offs, m_cap = saved
+        x, wq, wsd, offs, m_cap = saved
         M, K = x.shape
-        G, _, N = wqt.shape
+        G, N, _ = wq.shape
         dq, ds, dqt, dst = cast_2d_grouped(dy, offs, m_cap)
         xqt, xst = cast_dim1_grouped(x, offs, m_cap)
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
-        mx_grouped_mm(dq, ds, wqt, wsd, offs, G, MX_GROUPS_M, dx, M, K, N, m_cap)
+        mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
         dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=x.device)
         mx_grouped_mm(dqt, dst, xqt, xst, offs, G, MX_GROUPS_K, dw, M, N, K, m_cap)
         return dx, dw

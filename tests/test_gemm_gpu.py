@@ -98,6 +98,31 @@ def test_grouped_dgrad(mx):
                   O.grouped_mm_m(np.abs(a), np.abs(b), offs_t.numpy()), "dgrad")
 
 
+@pytest.mark.parametrize("sizes,N,K", [([130, 0, 384, 7], 512, 768), ([300], 256, 1024), ([1, 600], 1024, 256)])
+def test_grouped_dgrad_from_forward_codes(mx, sizes, N, K):
+    """The MN-major dgrad (B = the forward's 32x32 codes [G, N, K], no transposed
+    copy) against the oracle, and bitwise against the K-major dgrad on W^T codes."""
+    G = len(sizes)
+    dyb = S.normal_bf16((sum(sizes), N), 1e-2, seed=N + K)
+    wb = S.normal_bf16((G, N, K), 0.02, seed=G + 3)           # [G, N, K]
+    offs_t = S.offsets_from_sizes(sizes)
+    M, cap = dyb.shape[0], mx.mx_padded_rows_capacity(sum(sizes), G)
+    q, s = mx.cast_dim0_grouped(dyb.cuda(), offs_t.cuda(), cap)
+    wq, _, wqt, wsd = mx.cast_w32x32(wb.cuda())
+    out = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    mx.mx_grouped_mm(q, s, wq, wsd, offs_t.cuda(), G, mx.MX_GROUPS_M_KN, out, M, K, N, cap)
+    ref_km = mx.grouped_mm(q, s, wqt, wsd, offs_t.cuda(), M)
+    mx.mx_device_error()
+    assert torch.equal(out, ref_km)
+    qd, sd = O.cast_dim0_grouped(S.bf16_bits(dyb), offs_t.numpy(), cap)
+    qw, st = O.cast_32x32(S.bf16_bits(wb))
+    _, s_dg = O.w32_scale_views(st)
+    a = O.dequant(qd, sd)
+    b = O.dequant(np.ascontiguousarray(np.swapaxes(qw, 1, 2)), s_dg)
+    _assert_close(_f64(out), O.grouped_mm_m(a, b, offs_t.numpy()),
+                  O.grouped_mm_m(np.abs(a), np.abs(b), offs_t.numpy()), "dgrad (MN-major B)")
+
+
 @pytest.mark.parametrize("sizes", [[256, 128], [100, 0, 250, 1, 37], [0, 0, 300]])
 def test_grouped_wgrad_k_groups(mx, sizes):
     """dW_g = dY_g^T X_g over each group's tokens; empty groups are exact zeros."""
