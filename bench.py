@@ -6,13 +6,13 @@ shape of ao PR #4705 ("Wire MoE and MXFP8Linear training paths to CuTeDSL by
 default", roofline benchmark at K=N=4096, G=8, M=16384), run through every
 cast and GEMM of the path:
 
-  1. X   [16384, 4096]      dim0 cast into padded groups (pad path)
+  1. X   [16384, 4096]      fused dim0 + dim1 cast into padded groups (pad path;
+                            the dim1 codes are kept for the wgrad)
   2. W   [8, 4096, 4096]    32x32 cast (codes + forward and dgrad scale views)
   3. fwd grouped GEMM       Y  = X_g W_g^T          (M groups)
   4. dY  [16384, 4096]      fused dim0 + dim1 cast into padded groups
-  5. X                      dim1 cast into padded groups
-  6. dgrad grouped GEMM     dX = dY_g W_g           (M groups, W codes read MN-major)
-  7. wgrad grouped GEMM     dW_g = dY_g^T X_g       (K groups)
+  5. dgrad grouped GEMM     dX = dY_g W_g           (M groups, W codes read MN-major)
+  6. wgrad grouped GEMM     dW_g = dY_g^T X_g       (K groups)
 
 value = 3 * 2*M*N*K FLOPs per step / step time (TFLOP/s, whole job). Inputs
 are seeded synthetic bf16 tensors on the device (512 MB > the 126 MB L2, so
@@ -160,7 +160,7 @@ def profile_traffic(name, source_files):
 
 # ------------------------------------------------------------ our step ----
 class MoEStep:
-    """Preallocated buffers and the seven launches of one MoE fwd+bwd step."""
+    """Preallocated buffers and the six launches of one MoE fwd+bwd step."""
 
     def __init__(self, mx, device, seed=0):
         import torch
@@ -178,12 +178,12 @@ class MoEStep:
         self.dq, self.ds = u8(cap, N), u8(mx.mx_scale_bytes(cap, N // 32))
         self.dqt, self.dst = u8(N, cap), u8(mx.mx_scale_bytes(N, cap // 32))
         self.y, self.dx, self.dw = bf(M, N), bf(M, K), bf(G, N, K)
-        self.launches_per_step = 7
+        self.launches_per_step = 6
         self.gemm_events = []
 
     def run(self, timed_gemms=False):
         mx, t = self.mx, self.torch
-        mx.mx_cast_dim0_grouped(self.x, self.offs, self.cap, self.xq, self.xs)
+        mx.mx_cast_2d_grouped(self.x, self.offs, self.cap, self.xq, self.xs, self.xqt, self.xst)
         mx.mx_cast_w32x32(self.w, self.wq, self.wsf, None, self.wsd)
         gemms = (
             lambda: mx.mx_grouped_mm(self.xq, self.xs, self.wq, self.wsf, self.offs, G, mx.MX_GROUPS_M, self.y,
@@ -197,7 +197,6 @@ class MoEStep:
         for i, g in enumerate(gemms):
             if g is None:
                 mx.mx_cast_2d_grouped(self.dy, self.offs, self.cap, self.dq, self.ds, self.dqt, self.dst)
-                mx.mx_cast_dim1_grouped(self.x, self.offs, self.cap, self.xqt, self.xst)
                 continue
             if timed_gemms:
                 a, b = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)

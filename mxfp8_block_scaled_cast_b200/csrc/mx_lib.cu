@@ -17,6 +17,7 @@
 #include "mx_gemm.cuh"
 #include "mx_gemm_bf16.cuh"
 #include "mx_cast_pipe.cuh"
+#include "mx_cast_warp.cuh"
 #include "mx_dequant.cuh"
 #include "mx_linear.cuh"
 
@@ -56,11 +57,18 @@ mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, i
   if (col_tiles == 0 || row_tiles == 0 || depth == 0) return MX_OK;
   // dim1 and the 32x32 cast with transposed codes go through the TMA-pipelined
   // kernel (it needs a source row to map). The fused rowwise+columnwise cast
-  // stays on the tile kernel: it converts every element twice and is bound by
-  // instruction issue, where the tile kernel's higher occupancy wins (measured
-  // 4493 against 3873 GB/s at 16384^2).
+  // goes through the warp-sliced kernel (no CTA barriers, every output
+  // written as whole sectors from registers); dim0 and the plain 32x32 cast
+  // stay on the tile kernel.
   if (kMode == kModeCol || ((kMode & kModeSquare) && a.qt != nullptr))
     if (a.rows_src > 0) return launch_cast_pipe<kMode, kGrouped>(a, col_tiles, row_tiles, depth, stream);
+  if constexpr ((kMode & kModeRowCol) == kModeRowCol && !(kMode & kModeSquare)) {
+    MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth == 1, MX_ERR_UNSUPPORTED,
+               "cast grid too large (%lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles);
+    cast_warp_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), 1u), kWarpCastThreads,
+                                        kWarpCastSmem, stream>>>(a);
+    return cuda_check("fused cast launch");
+  }
   MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth <= 65535, MX_ERR_UNSUPPORTED,
              "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles,
              (long long)row_tiles, (long long)depth);

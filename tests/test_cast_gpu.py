@@ -124,6 +124,23 @@ def test_fused_2d_equals_oracle_and_split(mx, R, C):
         assert torch.equal(u, v)
 
 
+def test_fused_2d_outputs_only_16_byte_aligned(mx):
+    """Code buffers at a 16-byte (not 32-byte) offset take the 128-bit store path."""
+    R, C = 160, 288
+    xb = S.sweep_tensor((R, C), seed=12)
+    raw_q = torch.zeros(R * C + 16, dtype=torch.uint8, device="cuda")
+    raw_qt = torch.zeros(R * C + 16, dtype=torch.uint8, device="cuda")
+    q, qt = raw_q[16:].view(R, C), raw_qt[16:].view(C, R)
+    assert q.data_ptr() % 32 == 16 and qt.data_ptr() % 32 == 16
+    s = torch.empty(mx.mx_scale_bytes(R, C // 32), dtype=torch.uint8, device="cuda")
+    st = torch.empty(mx.mx_scale_bytes(C, R // 32), dtype=torch.uint8, device="cuda")
+    mx.mx_cast_2d(_dev(xb), q, s, qt, st)
+    (eq, es), (eqt, est) = O.cast_2d(S.bf16_bits(xb))
+    assert np.array_equal(_np(q), eq) and np.array_equal(_np(s), O.swizzle(es))
+    assert np.array_equal(_np(qt), eqt) and np.array_equal(_np(st), O.swizzle(est))
+    assert not raw_q[:16].any() and not raw_qt[:16].any()
+
+
 def test_unaligned_576_grad_full(mx):
     """The 576-wide gradient (18 scale columns padded to 20) at its full size."""
     xb = S.normal_bf16((16384, 576), 1.0, seed=0)
