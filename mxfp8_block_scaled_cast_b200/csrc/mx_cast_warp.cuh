@@ -5,18 +5,19 @@
 // A CTA of four warps owns a 128x128 bf16 tile -- exactly one 512-byte tile
 // of each blocked scale output -- and each warp owns 32 rows of it. A 32-row
 // slice holds whole blocks in both directions: four 1x32 blocks per row and
-// one 32x1 block per column. So every warp works alone (no CTA barrier):
+// one 32x1 block per column. So every warp works alone (one CTA barrier, at
+// the end, before the two 512-byte scale tiles are stored):
 //   load     the slice (32 rows x 256 bytes) into the warp's 8 KB of shared
 //            memory with 16-byte cp.async copies (zero fill past the tensor
 //            or the group); 16-byte chunk ch of row i is stored at chunk
 //            ch ^ (i % 8) of that row, so that both passes below read
 //            without bank conflicts;
 //   rows     lane i converts row i: four blocks, each 32 codes written as one
-//            32-byte sector, and the row's four scale bytes written as one
-//            word of the blocked tile;
+//            32-byte sector, and the row's four scale bytes staged as one
+//            word of the shared scale tile;
 //   columns  lane l converts column pairs l and l + 32: 32 rows each, the two
 //            columns' 32 codes written as two 32-byte sectors of the
-//            transposed output, and their scale bytes into the blocked tile.
+//            transposed output, and their scale bytes staged likewise.
 // Every code is written from registers as whole 32-byte sectors (one 256-bit
 // store per sector); the only shared-memory traffic is the staged input.
 #pragma once
@@ -64,6 +65,8 @@ cast_warp_kernel(const CastArgs a) {
   static_assert((kMode & kModeRowCol) == kModeRowCol && !(kMode & kModeSquare), "fused rowwise + columnwise only");
   extern __shared__ __align__(128) uint8_t wsmem[];
   __shared__ GroupSlot slots[kWarpCastWarps];
+  __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise scale tile
+  __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise scale tile
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t c0 = int64_t(blockIdx.x) * kCastTile;
   const int64_t r0 = int64_t(blockIdx.y) * kCastTile;
@@ -132,7 +135,7 @@ cast_warp_kernel(const CastArgs a) {
         st_sector(a.q + row * a.C + c0 + kb * 32, q_al, q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y);
     }
     // S[row, c0/32 + kb] for kb = 0..3: four consecutive bytes of the tile
-    *reinterpret_cast<uint32_t*>(a.s + chunk_row * 512 + i * 16 + warp * 4) = bytes;
+    *reinterpret_cast<uint32_t*>(s_row + i * 16 + warp * 4) = bytes;
   }
 
   // ---- columns: lane l converts column pairs l and l + 32 ----
@@ -164,9 +167,18 @@ cast_warp_kernel(const CastArgs a) {
       st_sector(a.qt + (c + 1) * a.rows_out + r0 + rw, qt_al, hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
     }
     // S_col[c, r/32]: row c of blocked(C, rows_out/32), column block r0/32 + warp
-    a.st[chunk_col * 512 + in_tile(uint32_t(2 * cp), uint32_t(warp))] = uint8_t(b_lo);
-    a.st[chunk_col * 512 + in_tile(uint32_t(2 * cp + 1), uint32_t(warp))] = uint8_t(b_hi);
+    s_col[in_tile(uint32_t(2 * cp), uint32_t(warp))] = uint8_t(b_lo);
+    s_col[in_tile(uint32_t(2 * cp + 1), uint32_t(warp))] = uint8_t(b_hi);
   }
+
+  // ---- both scale tiles leave as whole 512-byte stores ----
+  __syncthreads();
+  if (threadIdx.x < 32)
+    *reinterpret_cast<uint4*>(a.s + chunk_row * 512 + threadIdx.x * 16) =
+        *reinterpret_cast<const uint4*>(s_row + threadIdx.x * 16);
+  else if (threadIdx.x < 64)
+    *reinterpret_cast<uint4*>(a.st + chunk_col * 512 + (threadIdx.x - 32) * 16) =
+        *reinterpret_cast<const uint4*>(s_col + (threadIdx.x - 32) * 16);
 }
 
 }  // namespace mx

@@ -14,9 +14,9 @@
 // NaN.
 //
 // Memory bound (1 byte read, 2 bytes written per element): a warp takes 1024
-// consecutive elements of a row in four passes in which lane i converts 8
-// codes, so each load instruction of the warp reads 256 contiguous bytes and
-// each store writes 512.
+// consecutive elements of a row in two passes in which lane i converts 16
+// codes, so each load instruction of the warp reads 512 contiguous bytes and
+// each (256-bit per lane) store writes 1 KB.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -120,6 +120,9 @@ dequant_dim0_kernel(const DequantArgs a) {
   const int64_t sc_tiles = ceil_div(cb, 4);             // 4-column scale tiles per band
   const int64_t layout_bytes = ceil_to(a.layout_rows, 128) * ceil_to(cb, 4);
   const int64_t wstride = int64_t(gridDim.x) * (kDeqThreads / 32);
+  // element offsets are multiples of 16 (32 bytes of bf16): 256-bit stores
+  // need only a 32-byte aligned output (the ABI promises 16)
+  const bool out_al = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
   for (int64_t it = int64_t(blockIdx.x) * (kDeqThreads / 32) + warp; it < items; it += wstride) {
     const int64_t r = it / chunks;
     const int64_t c0 = (it - r * chunks) * 32;            // first block of the chunk
@@ -143,26 +146,36 @@ dequant_dim0_kernel(const DequantArgs a) {
     const uint8_t* qrow = a.q + src_row * a.C;
     __nv_bfloat16* orow = a.out + r * a.C;
     const int64_t e0 = c0 * kBlock;                     // first element of the chunk
-    // four passes of 256 elements: lane i takes 8 codes (8 bytes in, 16 bytes
-    // out), so every load and store instruction of the warp is contiguous
-    uint2 qv[4];
-    uint32_t bv[4];
+    // two passes of 512 elements: lane i takes 16 codes (16 bytes in, 32 bytes
+    // out), so every load instruction of the warp reads 512 contiguous bytes
+    // and every store writes 1 KB
+    uint4 qv[2];
+    uint32_t bv[2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t e = e0 + k * 256 + lane * 8;
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = e0 + k * 512 + lane * 16;
       if (e < a.C) {
-        qv[k] = *reinterpret_cast<const uint2*>(qrow + e);
+        qv[k] = ld_stream16(qrow + e);
         const int64_t c = e >> 5;
         bv[k] = sbase[(srow >> 7) * sc_tiles * 512 + (c >> 2) * 512 + in_tile(uint32_t(srow & 127), uint32_t(c))];
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t e = e0 + k * 256 + lane * 8;
+    for (int k = 0; k < 2; ++k) {
+      const int64_t e = e0 + k * 512 + lane * 16;
       if (e < a.C) {
         const float scale = e8m0_value(bv[k]);
-        const uint2 lo = dequant4(qv[k].x, scale), hi = dequant4(qv[k].y, scale);
-        *reinterpret_cast<uint4*>(orow + e) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        const uint2 p0 = dequant4(qv[k].x, scale), p1 = dequant4(qv[k].y, scale);
+        const uint2 p2 = dequant4(qv[k].z, scale), p3 = dequant4(qv[k].w, scale);
+        __nv_bfloat16* dst = orow + e;
+        if (out_al) {
+          asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(p0.x), "r"(p0.y),
+                       "r"(p1.x), "r"(p1.y), "r"(p2.x), "r"(p2.y), "r"(p3.x), "r"(p3.y)
+                       : "memory");
+        } else {
+          reinterpret_cast<uint4*>(dst)[0] = make_uint4(p0.x, p0.y, p1.x, p1.y);
+          reinterpret_cast<uint4*>(dst)[1] = make_uint4(p2.x, p2.y, p3.x, p3.y);
+        }
       }
     }
   }

@@ -61,6 +61,20 @@ def test_dequant_every_code_random_scales(mx, G, R, C):
     _assert_bf16_equal(out.reshape(G, R, C), O.dequant_bf16(q, s), "dequant")
 
 
+def test_dequant_output_only_16_byte_aligned(mx):
+    """An output at a 16-byte (not 32-byte) offset takes the 128-bit store path."""
+    rng = np.random.default_rng(5)
+    R, C = 130, 96
+    q = rng.integers(0, 0x7F, size=(R, C), dtype=np.uint8)
+    s = rng.integers(100, 140, size=(R, C // 32), dtype=np.uint8)
+    raw = torch.zeros(R * C + 8, dtype=torch.bfloat16, device="cuda")
+    out = raw[8:].view(R, C)
+    assert out.data_ptr() % 32 == 16
+    mx.mx_dequant_dim0(torch.from_numpy(q).cuda(), torch.from_numpy(O.swizzle(s)).cuda(), 1, R, C, out)
+    _assert_bf16_equal(out, O.dequant_bf16(q, s), "dequant, 16-byte aligned output")
+    assert not raw[:8].any()
+
+
 @pytest.mark.parametrize("sizes", [[37, 0, 263], [128, 128], [1, 2, 3, 500]])
 def test_dequant_grouped_round_trip(mx, sizes):
     M = int(sum(sizes))
