@@ -274,3 +274,36 @@ def test_high_precision_full_size_sampled(mx):
             n, k = int(rng.integers(4096)), int(rng.integers(4096))
             ref, absref = A[:, n] @ B[:, k], np.abs(A[:, n]) @ np.abs(B[:, k])
             assert abs(dwc[g, n, k] - ref) <= 2 ** -7 * abs(ref) + 1e-3 * absref, (g, n, k)
+
+
+def test_high_precision_skewed_full_size_sampled(mx):
+    """G=32, K=7168, N=2048, M=32768, Zipf groups with 3 empty: both bf16 gradients of
+    the high-precision arm, sampled, and exact zeros for the empty groups' dW."""
+    xb, wb, dyb, offs_t = S.unaligned_grouped_problem(device="cuda")    # x [M, K], w [G, N, K], dy [M, N]
+    offs_d = offs_t.cuda()
+    dx = mx.grouped_mm_bf16(dyb, wb, offs_d)                           # [M, K]
+    dw = mx.grouped_mm_bf16_wgrad(dyb, xb, offs_d)                     # [G, N, K]
+    mx.mx_device_error()
+    G, N, K = wb.shape
+    ends = offs_t.numpy().astype(np.int64)
+    starts = np.concatenate([[0], ends[:-1]])
+    rng = np.random.default_rng(6)
+    dxc = dx.float().cpu().numpy()
+    for r in rng.choice(dyb.shape[0], 24, replace=False):
+        g = int(np.searchsorted(ends, r, side="right"))
+        a = O.bf16_to_f64(_bits(dyb[r]))
+        cols = rng.choice(K, 16, replace=False)
+        bm = O.bf16_to_f64(_bits(wb[g][:, cols]))
+        ref, absref = a @ bm, np.abs(a) @ np.abs(bm)
+        assert np.all(np.abs(dxc[r, cols] - ref) <= 2 ** -7 * np.abs(ref) + 1e-3 * absref), r
+    for g in range(G):
+        if ends[g] == starts[g]:
+            assert not dw[g].any(), g
+    for g in rng.choice([g for g in range(G) if ends[g] > starts[g]], 5, replace=False):
+        A = O.bf16_to_f64(_bits(dyb[starts[g]:ends[g]]))
+        B = O.bf16_to_f64(_bits(xb[starts[g]:ends[g]]))
+        for _ in range(6):
+            n, k = int(rng.integers(N)), int(rng.integers(K))
+            ref, absref = A[:, n] @ B[:, k], np.abs(A[:, n]) @ np.abs(B[:, k])
+            got = float(dw[g, n, k])
+            assert abs(got - ref) <= 2 ** -7 * abs(ref) + 1e-3 * absref, (g, n, k)

@@ -233,3 +233,30 @@ def test_skewed_full_size_sampled(mx):
         a, b = O.dequant(qa, sa), O.dequant(qb, sb)
         ref, absref = O.mm(a, b), O.mm(np.abs(a), np.abs(b))
         _assert_close(_f64(dw[g, n:n + 32, k:k + 32]), ref, absref, f"wgrad g={g}")
+
+
+def test_skewed_dgrad_from_forward_codes_full_size_sampled(mx):
+    """G=32, K=7168, N=2048, M=32768 (Zipf groups, 3 empty): the MXFP8 dgrad with the
+    weight's forward codes read MN-major, sampled 32-column slices of sampled rows."""
+    xb, wb, dyb, offs_t = S.unaligned_grouped_problem(device="cuda")    # w [G, N=2048, K=7168]
+    offs_d = offs_t.cuda()
+    G, N, K = wb.shape
+    M = dyb.shape[0]
+    cap = mx.mx_padded_rows_capacity(M, G)
+    dq, ds = mx.cast_dim0_grouped(dyb, offs_d, cap)
+    wq, _, _, wsd = mx.cast_w32x32(wb, transposed=False, dgrad_scales=True)
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    mx.mx_grouped_mm(dq, ds, wq, wsd, offs_d, G, mx.MX_GROUPS_M_KN, dx, M, K, N, cap)
+    mx.mx_device_error()
+    ends = offs_t.numpy().astype(np.int64)
+    rng = np.random.default_rng(4)
+    dxc = _f64(dx)
+    for r in rng.choice(M, 24, replace=False):
+        g = int(np.searchsorted(ends, r, side="right"))
+        qd, sd = O.cast_dim0(S.bf16_bits(dyb[r:r + 1]))
+        a = O.dequant(qd, sd)                                            # [1, N]
+        k0 = int(rng.integers(K // 32)) * 32
+        qw, st = O.cast_32x32(S.bf16_bits(wb[g][:, k0:k0 + 32]))         # [N, 32]
+        _, s_dg = O.w32_scale_views(st)
+        bt = O.dequant(np.ascontiguousarray(qw.T), s_dg)                 # W^T [32, N]
+        _assert_close(dxc[r:r + 1, k0:k0 + 32], O.mm(a, bt), O.mm(np.abs(a), np.abs(bt)), f"dgrad row {r}")
