@@ -1,12 +1,13 @@
-// Warp-sliced fused rowwise + columnwise cast (torchtitan PR #5334,
-// description: one read of the input gives both the rowwise 1x32 and the
-// columnwise 32x1 casts), plain and over the group pad path.
+// Warp-sliced block-32 casts: rowwise 1x32 ("dim0"), columnwise 32x1
+// ("dim1"), both from one read (torchtitan PR #5334, description: the fused
+// rowwise/columnwise cast), and 32x32 weight blocks (same page, "32x32 RCEIL
+// weight-scale policy"), plain and over the group pad path.
 //
 // A CTA of four warps owns a 128x128 bf16 tile -- exactly one 512-byte tile
 // of each blocked scale output -- and each warp owns 32 rows of it. A 32-row
-// slice holds whole blocks in both directions: four 1x32 blocks per row and
-// one 32x1 block per column. So every warp works alone (one CTA barrier, at
-// the end, before the two 512-byte scale tiles are stored):
+// slice holds whole blocks of every geometry: four 1x32 blocks per row, one
+// 32x1 block per column, four 32x32 blocks. So every warp works alone (one
+// CTA barrier, at the end, before the 512-byte scale tiles are stored):
 //   load     the slice (32 rows x 256 bytes) into the warp's 8 KB of shared
 //            memory with 16-byte cp.async copies (zero fill past the tensor
 //            or the group); 16-byte chunk ch of row i is stored at chunk
@@ -17,7 +18,11 @@
 //            word of the shared scale tile;
 //   columns  lane l converts column pairs l and l + 32: 32 rows each, the two
 //            columns' 32 codes written as two 32-byte sectors of the
-//            transposed output, and their scale bytes staged likewise.
+//            transposed output, and their scale bytes staged likewise;
+//   32x32    the four block maxima are reduced over the warp's lanes first;
+//            rows then use the block scale (codes and the forward scale
+//            view), columns the same scale (optional transposed codes and
+//            the dgrad scale view).
 // Every code is written from registers as whole 32-byte sectors (one 256-bit
 // store per sector); the only shared-memory traffic is the staged input.
 #pragma once
@@ -59,18 +64,33 @@ __device__ __forceinline__ uint2 quant8(uint4 w, float inv) {
   return r;
 }
 
+// Largest of each 16-bit half over the 32 lanes of a warp.
+__device__ __forceinline__ uint32_t warp_max_u16x2(uint32_t v) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) v = __vmaxu2(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
 template <int kMode, bool kGrouped>
 __global__ void __launch_bounds__(kWarpCastThreads)
 cast_warp_kernel(const CastArgs a) {
-  static_assert((kMode & kModeRowCol) == kModeRowCol && !(kMode & kModeSquare), "fused rowwise + columnwise only");
+  constexpr bool kRow = (kMode & kModeRow) != 0;
+  constexpr bool kCol = (kMode & kModeCol) != 0;
+  constexpr bool kSq = (kMode & kModeSquare) != 0;
+  static_assert(!(kSq && (kRow || kCol || kGrouped)), "the 32x32 cast is its own mode");
   extern __shared__ __align__(128) uint8_t wsmem[];
   __shared__ GroupSlot slots[kWarpCastWarps];
-  __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise scale tile
-  __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise scale tile
+  __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
+  __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t c0 = int64_t(blockIdx.x) * kCastTile;
   const int64_t r0 = int64_t(blockIdx.y) * kCastTile;
-  const uint16_t* __restrict__ x = a.x;
+  const int64_t z = blockIdx.z;                       // expert of a 32x32 stack
+  const uint16_t* __restrict__ x = a.x + z * a.x_stride;
+  uint8_t* const q = a.q ? a.q + z * a.q_stride : nullptr;
+  uint8_t* const s = a.s ? a.s + z * a.s_stride : nullptr;
+  uint8_t* const qt = a.qt ? a.qt + z * a.qt_stride : nullptr;
+  uint8_t* const st = a.st ? a.st + z * a.st_stride : nullptr;
 
   // rows of this tile that hold data, and their first source row
   long long src0 = r0, live = a.rows_src - r0;
@@ -104,81 +124,130 @@ cast_warp_kernel(const CastArgs a) {
   const bool rows_out_ok = r0 + rw < a.rows_out;       // the warp's 32 output rows exist
   // row and column code offsets are multiples of 32 bytes, so 256-bit stores
   // only need 32-byte aligned base pointers (the ABI promises 16)
-  const bool q_al = (reinterpret_cast<uintptr_t>(a.q) & 31u) == 0;
-  const bool qt_al = (reinterpret_cast<uintptr_t>(a.qt) & 31u) == 0;
+  const bool q_al = (reinterpret_cast<uintptr_t>(q) & 31u) == 0;
+  const bool qt_al = (reinterpret_cast<uintptr_t>(qt) & 31u) == 0;
+  const uint8_t* rowp = slice + lane * 256;            // lane i works on row rw + i
+  auto chunk_of_row = [&](int c) {                     // 16-byte chunk c of row `lane`
+    return *reinterpret_cast<const uint4*>(rowp + ((c ^ (lane & 7)) << 4));
+  };
 
-  // ---- rows: lane i converts row rw + i ----
-  {
-    const int i = lane;
-    const uint8_t* rowp = slice + i * 256;
-    const int64_t row = r0 + rw + i;
+  // ---- square: one scale per 32x32 block, the max over the warp's rows ----
+  uint32_t bsq[4] = {0u, 0u, 0u, 0u};
+  if constexpr (kSq) {
+    uint32_t m01 = 0u, m23 = 0u;                       // blocks 0,1 and 2,3 in the 16-bit halves
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      uint32_t m = 0u;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint4 v = chunk_of_row(kb * 4 + cc);
+        m = absmax_bf16x2(m, v.x);
+        m = absmax_bf16x2(m, v.y);
+        m = absmax_bf16x2(m, v.z);
+        m = absmax_bf16x2(m, v.w);
+      }
+      m = max(m & 0xFFFFu, m >> 16);
+      if (kb == 0) m01 |= m; else if (kb == 1) m01 |= m << 16; else if (kb == 2) m23 |= m; else m23 |= m << 16;
+    }
+    m01 = warp_max_u16x2(m01);
+    m23 = warp_max_u16x2(m23);
+    bsq[0] = scale_b<kMode>(m01 & 0xFFFFu);
+    bsq[1] = scale_b<kMode>(m01 >> 16);
+    bsq[2] = scale_b<kMode>(m23 & 0xFFFFu);
+    bsq[3] = scale_b<kMode>(m23 >> 16);
+  }
+
+  // ---- rows: lane i converts row rw + i (rowwise blocks, or square blocks) ----
+  if constexpr (kRow || kSq) {
+    const int64_t row = r0 + rw + lane;
     uint32_t bytes = 0u;
 #pragma unroll
     for (int kb = 0; kb < 4; ++kb) {
       uint4 v[4];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) v[cc] = *reinterpret_cast<const uint4*>(rowp + (((kb * 4 + cc) ^ (i & 7)) << 4));
-      uint32_t m = 0u;
+      for (int cc = 0; cc < 4; ++cc) v[cc] = chunk_of_row(kb * 4 + cc);
+      uint32_t b;
+      if constexpr (kSq) {
+        b = bsq[kb];
+      } else {
+        uint32_t m = 0u;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        m = absmax_bf16x2(m, v[cc].x);
-        m = absmax_bf16x2(m, v[cc].y);
-        m = absmax_bf16x2(m, v[cc].z);
-        m = absmax_bf16x2(m, v[cc].w);
+        for (int cc = 0; cc < 4; ++cc) {
+          m = absmax_bf16x2(m, v[cc].x);
+          m = absmax_bf16x2(m, v[cc].y);
+          m = absmax_bf16x2(m, v[cc].z);
+          m = absmax_bf16x2(m, v[cc].w);
+        }
+        b = scale_b<kMode>(max(m & 0xFFFFu, m >> 16));
       }
-      m = max(m & 0xFFFFu, m >> 16);
-      const uint32_t b = scale_b<kMode>(m);
       bytes |= b << (8 * kb);
       const float inv = inv_scale(b);
       const uint2 q0 = quant8(v[0], inv), q1 = quant8(v[1], inv), q2 = quant8(v[2], inv), q3 = quant8(v[3], inv);
       if (row < a.rows_out && c0 + kb * 32 < a.C)
-        st_sector(a.q + row * a.C + c0 + kb * 32, q_al, q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y);
+        st_sector(q + row * a.C + c0 + kb * 32, q_al, q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y);
     }
     // S[row, c0/32 + kb] for kb = 0..3: four consecutive bytes of the tile
-    *reinterpret_cast<uint32_t*>(s_row + i * 16 + warp * 4) = bytes;
+    *reinterpret_cast<uint32_t*>(s_row + lane * 16 + warp * 4) = bytes;
   }
 
   // ---- columns: lane l converts column pairs l and l + 32 ----
+  const bool col_codes = kCol || (kSq && qt != nullptr);
+  if (kCol || (kSq && (qt != nullptr || st != nullptr))) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int cp = h * 32 + lane;                      // columns 2cp, 2cp + 1 of the tile
-    const int chunk = cp >> 2, word = cp & 3;
-    uint32_t w[32];
+    for (int h = 0; h < 2; ++h) {
+      const int cp = h * 32 + lane;                    // columns 2cp, 2cp + 1 of the tile
+      const int chunk = cp >> 2, word = cp & 3;
+      const int blk = cp >> 4;                         // 32-column block of these columns
+      uint32_t b_lo = 0u;
+      if constexpr (kSq) b_lo = blk == 0 ? bsq[0] : blk == 1 ? bsq[1] : blk == 2 ? bsq[2] : bsq[3];
+      uint32_t b_hi = b_lo;
+      if (col_codes) {
+        uint32_t w[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      w[i] = *reinterpret_cast<const uint32_t*>(slice + i * 256 + ((chunk ^ (i & 7)) << 4) + word * 4);
-    uint32_t acc = 0u;
+        for (int i = 0; i < 32; ++i)
+          w[i] = *reinterpret_cast<const uint32_t*>(slice + i * 256 + ((chunk ^ (i & 7)) << 4) + word * 4);
+        if constexpr (kCol) {
+          uint32_t acc = 0u;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc = absmax_bf16x2(acc, w[i]);
-    const uint32_t b_lo = scale_b<kMode>(acc & 0xFFFFu), b_hi = scale_b<kMode>(acc >> 16);
-    const float inv_lo = inv_scale(b_lo), inv_hi = inv_scale(b_hi);
-    uint32_t lo[8], hi[8];
+          for (int i = 0; i < 32; ++i) acc = absmax_bf16x2(acc, w[i]);
+          b_lo = scale_b<kMode>(acc & 0xFFFFu);
+          b_hi = scale_b<kMode>(acc >> 16);
+        }
+        const float inv_lo = inv_scale(b_lo), inv_hi = inv_scale(b_hi);
+        uint32_t lo[8], hi[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = 4 * j;
-      lo[j] = cvt_e4m3x2(bf16_lo(w[i]) * inv_lo, bf16_lo(w[i + 1]) * inv_lo) |
-              (cvt_e4m3x2(bf16_lo(w[i + 2]) * inv_lo, bf16_lo(w[i + 3]) * inv_lo) << 16);
-      hi[j] = cvt_e4m3x2(bf16_hi(w[i]) * inv_hi, bf16_hi(w[i + 1]) * inv_hi) |
-              (cvt_e4m3x2(bf16_hi(w[i + 2]) * inv_hi, bf16_hi(w[i + 3]) * inv_hi) << 16);
+        for (int j = 0; j < 8; ++j) {
+          const int i = 4 * j;
+          lo[j] = cvt_e4m3x2(bf16_lo(w[i]) * inv_lo, bf16_lo(w[i + 1]) * inv_lo) |
+                  (cvt_e4m3x2(bf16_lo(w[i + 2]) * inv_lo, bf16_lo(w[i + 3]) * inv_lo) << 16);
+          hi[j] = cvt_e4m3x2(bf16_hi(w[i]) * inv_hi, bf16_hi(w[i + 1]) * inv_hi) |
+                  (cvt_e4m3x2(bf16_hi(w[i + 2]) * inv_hi, bf16_hi(w[i + 3]) * inv_hi) << 16);
+        }
+        const int64_t c = c0 + 2 * cp;
+        if (rows_out_ok && c < a.C) {
+          st_sector(qt + c * a.rows_out + r0 + rw, qt_al, lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
+          st_sector(qt + (c + 1) * a.rows_out + r0 + rw, qt_al, hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6],
+                    hi[7]);
+        }
+      }
+      // S_col[c, r/32] (square: S_dgrad[k, n/32]): row c of blocked(C, rows_out/32),
+      // column block r0/32 + warp
+      s_col[in_tile(uint32_t(2 * cp), uint32_t(warp))] = uint8_t(b_lo);
+      s_col[in_tile(uint32_t(2 * cp + 1), uint32_t(warp))] = uint8_t(b_hi);
     }
-    const int64_t c = c0 + 2 * cp;
-    if (rows_out_ok && c < a.C) {
-      st_sector(a.qt + c * a.rows_out + r0 + rw, qt_al, lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
-      st_sector(a.qt + (c + 1) * a.rows_out + r0 + rw, qt_al, hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
-    }
-    // S_col[c, r/32]: row c of blocked(C, rows_out/32), column block r0/32 + warp
-    s_col[in_tile(uint32_t(2 * cp), uint32_t(warp))] = uint8_t(b_lo);
-    s_col[in_tile(uint32_t(2 * cp + 1), uint32_t(warp))] = uint8_t(b_hi);
   }
 
-  // ---- both scale tiles leave as whole 512-byte stores ----
+  // ---- the scale tiles leave as whole 512-byte stores ----
   __syncthreads();
-  if (threadIdx.x < 32)
-    *reinterpret_cast<uint4*>(a.s + chunk_row * 512 + threadIdx.x * 16) =
-        *reinterpret_cast<const uint4*>(s_row + threadIdx.x * 16);
-  else if (threadIdx.x < 64)
-    *reinterpret_cast<uint4*>(a.st + chunk_col * 512 + (threadIdx.x - 32) * 16) =
-        *reinterpret_cast<const uint4*>(s_col + (threadIdx.x - 32) * 16);
+  if (threadIdx.x < 32) {
+    if ((kRow || kSq) && s != nullptr)
+      *reinterpret_cast<uint4*>(s + chunk_row * 512 + threadIdx.x * 16) =
+          *reinterpret_cast<const uint4*>(s_row + threadIdx.x * 16);
+  } else if (threadIdx.x < 64) {
+    if ((kCol || kSq) && st != nullptr)
+      *reinterpret_cast<uint4*>(st + chunk_col * 512 + (threadIdx.x - 32) * 16) =
+          *reinterpret_cast<const uint4*>(s_col + (threadIdx.x - 32) * 16);
+  }
 }
 
 }  // namespace mx

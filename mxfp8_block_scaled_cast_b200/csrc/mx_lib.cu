@@ -16,7 +16,6 @@
 #include "mx_cast.cuh"
 #include "mx_gemm.cuh"
 #include "mx_gemm_bf16.cuh"
-#include "mx_cast_pipe.cuh"
 #include "mx_cast_warp.cuh"
 #include "mx_dequant.cuh"
 #include "mx_linear.cuh"
@@ -48,39 +47,16 @@ mx_status cuda_check(const char* what) {
   } while (0)
 
 template <int kMode, bool kGrouped>
-mx_status launch_cast_pipe(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
-                           cudaStream_t stream);
-
-template <int kMode, bool kGrouped>
 mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
                       cudaStream_t stream) {
   if (col_tiles == 0 || row_tiles == 0 || depth == 0) return MX_OK;
-  // dim1 and the 32x32 cast with transposed codes go through the TMA-pipelined
-  // kernel (it needs a source row to map). The fused rowwise+columnwise cast
-  // goes through the warp-sliced kernel (no CTA barriers, every output
-  // written as whole sectors from registers); dim0 and the plain 32x32 cast
-  // stay on the tile kernel.
-  if (kMode == kModeCol || ((kMode & kModeSquare) && a.qt != nullptr))
-    if (a.rows_src > 0) return launch_cast_pipe<kMode, kGrouped>(a, col_tiles, row_tiles, depth, stream);
-  if constexpr ((kMode & kModeRowCol) == kModeRowCol && !(kMode & kModeSquare)) {
-    MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth == 1, MX_ERR_UNSUPPORTED,
-               "cast grid too large (%lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles);
-    cast_warp_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), 1u), kWarpCastThreads,
-                                        kWarpCastSmem, stream>>>(a);
-    return cuda_check("fused cast launch");
-  }
+  // Every cast goes through the warp-sliced kernel (no CTA barrier before the
+  // scale tiles, every code written as whole 32-byte sectors from registers).
   MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth <= 65535, MX_ERR_UNSUPPORTED,
-             "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles,
-             (long long)row_tiles, (long long)depth);
-  const bool colpass = (kMode & kModeCol) || ((kMode & kModeSquare) && a.qt != nullptr);
-  const size_t smem = colpass ? size_t(kXsBytes + kQsBytes) : 0;
-  if (smem > 0) {
-    cudaError_t e = cudaFuncSetAttribute(cast_tile_kernel<kMode, kGrouped>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return fail(MX_ERR_CUDA, "cast smem attribute: %s", cudaGetErrorString(e));
-  }
-  cast_tile_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)),
-                                       kCastThreads, smem, stream>>>(a);
+             "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles,
+             (long long)depth);
+  cast_warp_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)),
+                                      kWarpCastThreads, kWarpCastSmem, stream>>>(a);
   return cuda_check("cast launch");
 }
 
@@ -173,44 +149,6 @@ mx_status make_scale_map(CUtensorMap* m, const void* base, uint64_t chunks) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
   return MX_OK;
-}
-
-template <int kMode, bool kGrouped>
-mx_status launch_cast_pipe(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
-                           cudaStream_t stream) {
-  auto fn = encode_fn();
-  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  // bf16 source viewed as [depth * rows_src, C]; 128x128 boxes, zero fill outside
-  CUtensorMap xmap;
-  cuuint64_t dims[2] = {cuuint64_t(a.C), cuuint64_t(depth * a.rows_src)};
-  cuuint64_t strides[1] = {cuuint64_t(a.C) * 2};
-  cuuint32_t box[2] = {uint32_t(kCastTile), uint32_t(kCastTile)};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (cast input) failed (%d)", int(r));
-  static int per_sm[64] = {};
-  static int sms[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  MX_REQUIRE(e == cudaSuccess && dev < 64, MX_ERR_CUDA, "cudaGetDevice failed");
-  e = cudaFuncSetAttribute(cast_pipe_kernel<kMode, kGrouped>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(kPipeSmem));
-  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "cast smem attribute: %s", cudaGetErrorString(e));
-  if (per_sm[dev] == 0) {
-    int n = 0, m = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cast_pipe_kernel<kMode, kGrouped>, kPipeThreads, kPipeSmem);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev);
-    MX_REQUIRE(e == cudaSuccess && n > 0 && m > 0, MX_ERR_CUDA, "cast occupancy query failed");
-    per_sm[dev] = n;
-    sms[dev] = m;
-  }
-  const int64_t total = col_tiles * row_tiles * depth;
-  const int64_t cap = int64_t(per_sm[dev]) * sms[dev];
-  const unsigned grid = unsigned(total < cap ? total : cap);
-  cast_pipe_kernel<kMode, kGrouped><<<grid, kPipeThreads, kPipeSmem, stream>>>(xmap, a, col_tiles, row_tiles, total);
-  return cuda_check("cast launch");
 }
 
 template <int kMode>
