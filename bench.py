@@ -253,6 +253,52 @@ def cast_sweep(mx, device, flush):
     return out
 
 
+def linear_bench(mx, device, flush, peaks, reps=20):
+    """MXFP8 linear forward + backward at M=4096, N=4096, K=2048 (the MXFP8Linear
+    benchmark shape of ao PR #4705): y = x w^T, dx = dy w, dw = dy^T x, each step
+    re-quantizing w (no cache) or reusing its cached quantization (cache hit, as in
+    activation-checkpoint recompute). Median of L2-flushed repetitions."""
+    import torch
+    from mxfp8_block_scaled_cast_b200 import synthetic as S
+    Ml, Nl, Kl = 4096, 4096, 2048
+    x, w, dy = S.linear_problem(Ml, Nl, Kl, seed=0, device=device)
+    ws = mx.linear_workspace(Ml, Nl, Kl, device)
+    y = torch.empty(Ml, Nl, dtype=torch.bfloat16, device=device)
+    dx = torch.empty(Ml, Kl, dtype=torch.bfloat16, device=device)
+    dw = torch.empty(Nl, Kl, dtype=torch.bfloat16, device=device)
+    cache = mx.WeightCache()
+
+    def step(c):
+        mx.mx_linear_fwd(x, w, c, 0, y, ws)
+        mx.mx_linear_bwd(dy, x, w, c, 0, dx, dw, ws)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2] * 1e-3
+
+    t_nc = timed(lambda: step(None))
+    t_hit = timed(lambda: step(cache))
+    mx.mx_device_error()
+    hits = cache.stats()["hits"]
+    cache.close()
+    flops = 3 * 2 * Ml * Nl * Kl
+    return {"shape": {"M": Ml, "N": Nl, "K": Kl}, "flops_per_step": flops,
+            "no_cache": {"ms_per_step": round(t_nc * 1e3, 4), "tflops": round(flops / t_nc / 1e12, 1)},
+            "cache_hit": {"ms_per_step": round(t_hit * 1e3, 4), "tflops": round(flops / t_hit / 1e12, 1),
+                          "hits": hits}}
+
+
 def override_arms(mx, step, flush, peaks):
     """Backward of the same MoE layer under the two backward overrides.
 
@@ -391,6 +437,7 @@ def main(argv=None):
     p.add_argument("--no-sweep", action="store_true", help="skip the cast bandwidth sweep")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
+    p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--ref-tokens", type=int, default=512)
     args = p.parse_args(argv)
@@ -508,6 +555,10 @@ def main(argv=None):
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         casts = {k: {"gbs": v, "frac_of_measured_hbm": round(v / hbm, 3), "frac_of_8tbs_spec": round(v / 8000, 3)}
                  for k, v in casts.items()}
+    linear = None
+    if not args.no_linear:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        linear = linear_bench(mx, dev, flush, peaks)
     arms = None
     if not args.no_arms:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -535,6 +586,7 @@ def main(argv=None):
         "cpu_baseline": cpu,
         "casts": casts,
         "backward_overrides": arms,
+        "linear": linear,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
