@@ -115,7 +115,9 @@ MX_API mx_status mx_cast_2d(const void* x, int64_t R, int64_t C,
  * stack of G weights w bf16 [G, N, K] (G = 1 for a dense weight):
  *   q        E4M3 [G, N, K]
  *   s_fwd    G concatenated blocked(N, K/32) buffers, S_fwd[n, kb] = S[n/32, kb]
- *   qt       E4M3 [G, K, N] (the same codes transposed) or NULL
+ *   qt       E4M3 [G, K, N] (the same codes transposed) or NULL; the dgrad
+ *            does not need it (mx_grouped_mm mode MX_GROUPS_M_KN reads q
+ *            itself with s_dgrad)
  *   s_dgrad  G concatenated blocked(K, N/32) buffers, S_dgrad[k, nb] = S[nb, k/32],
  *            or NULL
  * N and K positive multiples of 32. */
