@@ -158,6 +158,21 @@ def profile_traffic(name, source_files):
         return None
 
 
+class L2Flush:
+    """Empties the 126 MB L2 between timed iterations: writes a 256 MB buffer, then
+    reads a second one, so that the written lines are evicted (and written back)
+    before the timed kernel starts rather than during it."""
+
+    def __init__(self, device, nbytes=256 * 1024 * 1024):
+        import torch
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(nbytes // 4, dtype=torch.int32, device=device)
+
+    def zero_(self):
+        self.w.zero_()
+        self.r.max()
+
+
 # ------------------------------------------------------------ our step ----
 class MoEStep:
     """Preallocated buffers and the six launches of one MoE fwd+bwd step."""
@@ -209,7 +224,8 @@ class MoEStep:
 
 
 def cast_sweep(mx, device, flush):
-    """GB/s of each cast mode on the 16384^2 sweep tensor and the expert stack."""
+    """GB/s of each cast mode on the 1024^2 ... 16384^2 sweep tensors and the expert
+    stack (L2 flushed between iterations; 8192^2, 16384^2 and the stack exceed L2)."""
     import torch
     from mxfp8_block_scaled_cast_b200 import synthetic as S
 
@@ -229,20 +245,20 @@ def cast_sweep(mx, device, flush):
         return ts[len(ts) // 2] * 1e-3
 
     out = {}
-    n = 16384
-    x = S.sweep_tensor((n, n), seed=0, device=device)
-    u8 = lambda *s: torch.empty(*s, dtype=torch.uint8, device=device)
-    q, s, qt, st = u8(n, n), u8(mx.mx_scale_bytes(n, n // 32)), u8(n, n), u8(mx.mx_scale_bytes(n, n // 32))
-    E = n * n
-    modes = {
-        "dim0": (lambda: mx.mx_cast_dim0(x, q, s), 2 + 1 + 1 / 32),
-        "dim1": (lambda: mx.mx_cast_dim1(x, qt, st), 2 + 1 + 1 / 32),
-        "2d": (lambda: mx.mx_cast_2d(x, q, s, qt, st), 2 + 2 + 2 / 32),
-        "32x32": (lambda: mx.mx_cast_w32x32(x, q, s, None, st), 2 + 1 + 2 / 32),
-    }
-    for name, (fn, bpe) in modes.items():
-        sec = timed(fn)
-        out[f"{name}_16384x16384_gbs"] = round(E * bpe / sec / 1e9, 1)
+    for n in (1024, 4096, 8192, 16384):
+        x = S.sweep_tensor((n, n), seed=0, device=device)
+        u8 = lambda *s: torch.empty(*s, dtype=torch.uint8, device=device)
+        q, s, qt, st = u8(n, n), u8(mx.mx_scale_bytes(n, n // 32)), u8(n, n), u8(mx.mx_scale_bytes(n, n // 32))
+        E = n * n
+        modes = {
+            "dim0": (lambda: mx.mx_cast_dim0(x, q, s), 2 + 1 + 1 / 32),
+            "dim1": (lambda: mx.mx_cast_dim1(x, qt, st), 2 + 1 + 1 / 32),
+            "2d": (lambda: mx.mx_cast_2d(x, q, s, qt, st), 2 + 2 + 2 / 32),
+            "32x32": (lambda: mx.mx_cast_w32x32(x, q, s, None, st), 2 + 1 + 2 / 32),
+        }
+        for name, (fn, bpe) in modes.items():
+            sec = timed(fn)
+            out[f"{name}_{n}x{n}_gbs"] = round(E * bpe / sec / 1e9, 1)
     del x, q, s, qt, st
     g3, n3, k3 = 64, 2048, 7168
     w = S.sweep_tensor((g3, n3, k3), seed=0, device=device)
@@ -250,6 +266,57 @@ def cast_sweep(mx, device, flush):
     sf, sd = u8(g3 * mx.mx_scale_bytes(n3, k3 // 32)), u8(g3 * mx.mx_scale_bytes(k3, n3 // 32))
     sec = timed(lambda: mx.mx_cast_w32x32(w, wq, sf, None, sd), reps=5)
     out["32x32_64x2048x7168_gbs"] = round(g3 * n3 * k3 * (2 + 1 + 2 / 32) / sec / 1e9, 1)
+    return out
+
+
+def gemm_only(mx, step, peaks, iters=100, runs=5):
+    """The three grouped GEMMs of the step alone, on the step's prequantized
+    operands: each captured as a CUDA graph of `iters` launches and replayed
+    `runs` times; median time per launch. No flush (operands 201-335 MB per
+    launch, above the 126 MB L2)."""
+    import torch
+    step.run()
+    torch.cuda.synchronize()
+    calls = {
+        "fwd": lambda: mx.mx_grouped_mm(step.xq, step.xs, step.wq, step.wsf, step.offs, G, mx.MX_GROUPS_M,
+                                        step.y, M, N, K, step.cap),
+        "dgrad": lambda: mx.mx_grouped_mm(step.dq, step.ds, step.wq, step.wsd, step.offs, G, mx.MX_GROUPS_M_KN,
+                                          step.dx, M, K, N, step.cap),
+        "wgrad": lambda: mx.mx_grouped_mm(step.dqt, step.dst, step.xqt, step.xst, step.offs, G, mx.MX_GROUPS_K,
+                                          step.dw, M, N, K, step.cap),
+    }
+    out = {}
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_OVER_BF16
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_OVER_BF16
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                for _ in range(iters):
+                    fn()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(runs):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / iters)
+        ts.sort()
+        tf = GEMM_FLOPS / (ts[len(ts) // 2] * 1e-3) / 1e12
+        out[name] = {"us_per_launch": round(ts[len(ts) // 2] * 1e3, 1), "tflops": round(tf, 1),
+                     "frac_of_measured_sustained_fp8": round(tf / sustained, 3),
+                     "frac_of_measured_burst_fp8": round(tf / burst, 3), "frac_of_4500_spec": round(tf / 4500.0, 3)}
+        del g
+    mx.mx_device_error()
+    out["method"] = (f"CUDA graph of {iters} back-to-back launches (power-capped), median of {runs} replays; "
+                     f"fp8 peaks = measured bf16 (sustained, burst) x {FP8_OVER_BF16}")
     return out
 
 
@@ -438,6 +505,7 @@ def main(argv=None):
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
     p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
+    p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--ref-tokens", type=int, default=512)
     args = p.parse_args(argv)
@@ -550,18 +618,19 @@ def main(argv=None):
 
     casts = None
     if not args.no_sweep:
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         casts = cast_sweep(mx, dev, flush)
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         casts = {k: {"gbs": v, "frac_of_measured_hbm": round(v / hbm, 3), "frac_of_8tbs_spec": round(v / 8000, 3)}
                  for k, v in casts.items()}
+    gemm_alone = None if args.no_gemm_only else gemm_only(mx, step, peaks)
     linear = None
     if not args.no_linear:
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         linear = linear_bench(mx, dev, flush, peaks)
     arms = None
     if not args.no_arms:
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         arms = override_arms(mx, step, flush, peaks)
 
     if rank != 0:
@@ -587,6 +656,7 @@ def main(argv=None):
         "casts": casts,
         "backward_overrides": arms,
         "linear": linear,
+        "gemm_only": gemm_alone,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
