@@ -307,3 +307,35 @@ def test_high_precision_skewed_full_size_sampled(mx):
             ref, absref = A[:, n] @ B[:, k], np.abs(A[:, n]) @ np.abs(B[:, k])
             got = float(dw[g, n, k])
             assert abs(got - ref) <= 2 ** -7 * abs(ref) + 1e-3 * absref, (g, n, k)
+
+
+@pytest.mark.parametrize("M,K,sizes", [(50, 40, None), (50, 40, [20, 0, 30]), (7, 8, [7])])
+def test_bf16_row_groups_tiny_shapes(mx, M, K, sizes):
+    """Fewer rows than a tile and a contraction shorter than one 64-deep step:
+    the operand boxes reach past the tensors and read zeros."""
+    N = 256
+    G = len(sizes) if sizes else 1
+    a = S.normal_bf16((M, K), seed=M + K)
+    b = S.normal_bf16((G, K, N), 0.05, seed=G + K)
+    offs_t = S.offsets_from_sizes(sizes) if sizes else None
+    out = mx.grouped_mm_bf16(a.cuda(), b.cuda(), offs_t.cuda() if sizes else None)
+    mx.mx_device_error()
+    af, bf = O.bf16_to_f64(S.bf16_bits(a)), O.bf16_to_f64(S.bf16_bits(b))
+    offs = offs_t.numpy() if sizes else np.array([M])
+    _assert_close(_f64(out), O.hp_grouped_mm_m(af, bf, offs), O.hp_grouped_mm_m(np.abs(af), np.abs(bf), offs),
+                  "tiny row groups")
+
+
+def test_bf16_token_groups_tiny_shapes(mx):
+    """Groups of a few tokens (every one a partial 64-token step)."""
+    sizes = [3, 0, 1, 10]
+    M, N, K = sum(sizes), 256, 256
+    a = S.normal_bf16((M, N), seed=5)
+    b = S.normal_bf16((M, K), seed=6)
+    offs_t = S.offsets_from_sizes(sizes)
+    out = mx.grouped_mm_bf16_wgrad(a.cuda(), b.cuda(), offs_t.cuda())
+    mx.mx_device_error()
+    af, bf = O.bf16_to_f64(S.bf16_bits(a)), O.bf16_to_f64(S.bf16_bits(b))
+    offs = offs_t.numpy()
+    _assert_close(_f64(out), O.hp_grouped_mm_k(af, bf, offs), O.hp_grouped_mm_k(np.abs(af), np.abs(bf), offs),
+                  "tiny token groups")
