@@ -52,3 +52,41 @@ def test_host_helpers_match_oracle():
         assert mx.mx_padded_rows_capacity(m, g) == O.padded_rows_capacity(m, g)
     assert mx.lib().mx_last_error() is not None
     assert np.int64(mx.mx_padded_rows_capacity(-1, 1)) == -1
+
+
+def test_no_silent_fallback_without_the_library_or_a_gpu(monkeypatch, tmp_path):
+    """The product path raises when libmx.so is missing or a tensor is on the
+    host: there is no CPU implementation behind the binding."""
+    import pytest
+    import torch
+    from mxfp8_block_scaled_cast_b200 import mx
+    monkeypatch.setattr(mx, "_lib", None)
+    monkeypatch.setattr(mx, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mx.lib()
+    monkeypatch.undo()
+    x = torch.zeros(32, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="device tensors"):
+        mx.cast_dim0(x)
+    with pytest.raises(ValueError):
+        mx.MXFP8GroupedMM(backward_override="fp32")
+
+
+def test_host_argument_checks_return_before_any_launch():
+    """Argument errors are reported from host checks alone (no device is touched:
+    the pointers below are never dereferenced)."""
+    from mxfp8_block_scaled_cast_b200 import mx
+    L = mx.lib()
+    ok16, odd = ctypes.c_void_p(0x100000), ctypes.c_void_p(0x100008)
+    assert L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None) == 3          # C not a multiple of 32
+    assert L.mx_cast_dim0(odd, 64, 64, ok16, ok16, None) == 2           # misaligned input
+    assert L.mx_cast_dim1(ok16, 48, 64, ok16, ok16, None) == 3          # R not a multiple of 32
+    assert L.mx_cast_ex(ok16, 64, 64, 3, 7, ok16, ok16, ok16, ok16, None) == 1   # unknown rule
+    assert L.mx_grouped_mm(ok16, ok16, ok16, ok16, None, 1, 5, ok16, 128, 256, 128, 0, None) == 1  # mode
+    assert L.mx_grouped_mm(ok16, ok16, ok16, ok16, None, 1, 0, ok16, 128, 200, 128, 0, None) == 3  # N % 256
+    assert L.mx_grouped_mm_bf16(ok16, ok16, None, 1, 0, ok16, 128, 256, 60, None) == 3      # K % 8
+    assert L.mx_grouped_mm_bf16(ok16, ok16, ok16, 0, 0, ok16, 128, 256, 64, None) == 1      # G = 0
+    assert L.mx_dequant_dim0(ok16, ok16, 1, 4, 40, ok16, None) == 3     # C not a multiple of 32
+    assert L.mx_scales_unswizzle(odd, 4, 4, ok16, None) == 2
+    msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
+    assert b"not a multiple of 32" in msg
