@@ -312,6 +312,15 @@ MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
 MX_API mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t M, int64_t N, int64_t K,
                                        void* y, void* stream);
 
+/* ---------------------------------------------------- failure detection --
+ * No counterpart on the source pages: a diagnostic of the library's own
+ * failure detection. It launches one thread that waits, through the same
+ * bounded wait the GEMM pipelines use, on a barrier nothing ever arrives
+ * on; after that wait's 2-second limit the thread gives up, sets the sticky
+ * device flag and returns. mx_device_error(stream) then reports
+ * MX_ERR_TIMEOUT (and clears the flag); the context stays usable. */
+MX_API mx_status mx_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

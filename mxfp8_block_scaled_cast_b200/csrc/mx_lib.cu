@@ -802,3 +802,27 @@ extern "C" mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, 
                                                                  static_cast<uint8_t*>(out));
   return cuda_check("unswizzle launch");
 }
+
+// ---------------------------------------------------- failure detection ---
+// One thread waits, through the bounded wait every GEMM pipeline uses, on a
+// barrier that nothing ever arrives on; after the wait's time limit it gives
+// up, sets the sticky timeout flag and returns.
+namespace mx {
+namespace {
+__global__ void wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    abort_word = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    (void)mbar_wait(smem_u32(&bar), 0u, &abort_word);
+  }
+}
+}  // namespace
+}  // namespace mx
+
+extern "C" mx_status mx_selftest_wait_timeout(void* stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_check("selftest launch");
+}

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "mx_dequant_dim0": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "mx_dequant_dim0_grouped": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i64, _i64, _vp, _vp]),
     "mx_scales_unswizzle": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
+    "mx_selftest_wait_timeout": (ctypes.c_int, [_vp]),
 }
 
 MX_RCEIL = 0
