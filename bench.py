@@ -458,6 +458,17 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def blas_threads():
+    """Threads of the BLAS numpy's float64 matmuls run on (None if unknown)."""
+    try:
+        import numpy  # noqa: F401  (loads the BLAS the oracle uses)
+        from threadpoolctl import threadpool_info
+        counts = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(counts) if counts else None
+    except Exception:
+        return None
+
+
 def cpu_baseline(budget_s=12.0, tokens=512):
     flops, secs, n = 0, 0.0, 0
     while secs < budget_s:
@@ -465,8 +476,10 @@ def cpu_baseline(budget_s=12.0, tokens=512):
         flops += f
         secs += s
         n += 1
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{n} x (one expert, {tokens} tokens, K=N=4096: oracle casts + float64 fwd/dgrad/wgrad)"}
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "blas_threads": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} x (one expert, {tokens} tokens, K=N=4096: oracle casts (single-threaded numpy) + "
+                      f"float64 fwd/dgrad/wgrad (BLAS))"}
 
 
 def run_reference(args, rank):
@@ -486,7 +499,8 @@ def run_reference(args, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "G": G, "M": M, "N": N, "K": K,
                    "sample": f"one expert, {args.ref_tokens} tokens per step"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "blas_threads": blas_threads(),
+                         "kind": "oracle",
                          "sample": f"{args.steps} x (one expert, {args.ref_tokens} tokens)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
