@@ -320,11 +320,14 @@ def gemm_only(mx, step, peaks, iters=100, runs=5):
     return out
 
 
-def linear_bench(mx, device, flush, peaks, reps=20):
+def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
     """MXFP8 linear forward + backward at M=4096, N=4096, K=2048 (the MXFP8Linear
     benchmark shape of ao PR #4705): y = x w^T, dx = dy w, dw = dy^T x, each step
     re-quantizing w (no cache) or reusing its cached quantization (cache hit, as in
-    activation-checkpoint recompute). Median of L2-flushed repetitions."""
+    activation-checkpoint recompute). A step is ~0.15 ms of GPU work in seven
+    launches, so it is timed both as issued from Python (eager, median of
+    L2-flushed repetitions, includes host submission) and as CUDA-graph replays of
+    `graph_steps` steps (median of 5 replays, per step)."""
     import torch
     from mxfp8_block_scaled_cast_b200 import synthetic as S
     Ml, Nl, Kl = 4096, 4096, 2048
@@ -354,16 +357,40 @@ def linear_bench(mx, device, flush, peaks, reps=20):
         ts.sort()
         return ts[len(ts) // 2] * 1e-3
 
-    t_nc = timed(lambda: step(None))
-    t_hit = timed(lambda: step(cache))
+    def graphed(fn):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                for _ in range(graph_steps):
+                    fn()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / graph_steps)
+        ts.sort()
+        del g
+        return ts[2] * 1e-3
+
+    t_nc, g_nc = timed(lambda: step(None)), graphed(lambda: step(None))
+    t_hit, g_hit = timed(lambda: step(cache)), graphed(lambda: step(cache))
     mx.mx_device_error()
     hits = cache.stats()["hits"]
     cache.close()
     flops = 3 * 2 * Ml * Nl * Kl
+    entry = lambda te, tg: {"ms_per_step_graph": round(tg * 1e3, 4), "tflops_graph": round(flops / tg / 1e12, 1),
+                            "ms_per_step_eager": round(te * 1e3, 4), "tflops_eager": round(flops / te / 1e12, 1)}
     return {"shape": {"M": Ml, "N": Nl, "K": Kl}, "flops_per_step": flops,
-            "no_cache": {"ms_per_step": round(t_nc * 1e3, 4), "tflops": round(flops / t_nc / 1e12, 1)},
-            "cache_hit": {"ms_per_step": round(t_hit * 1e3, 4), "tflops": round(flops / t_hit / 1e12, 1),
-                          "hits": hits}}
+            "no_cache": entry(t_nc, g_nc), "cache_hit": dict(entry(t_hit, g_hit), hits=hits)}
 
 
 def override_arms(mx, step, flush, peaks):
