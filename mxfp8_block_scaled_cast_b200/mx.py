@@ -500,3 +500,67 @@ class MXFP8GroupedMM:
         dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=x.device)
         mx_grouped_mm(dqt, dst, xqt, xst, offs, G, MX_GROUPS_K, dw, M, N, K, m_cap)
         return dx, dw
+
+
+# ------------------------------------------------------------- autograd --
+class _GroupedMMFn(torch.autograd.Function):
+    """Autograd wrapper of MXFP8GroupedMM: forward and backward are its calls."""
+
+    @staticmethod
+    def forward(ctx, x, w, offs, backward_override):
+        op = MXFP8GroupedMM(backward_override=backward_override)
+        y = op.forward(x, w, offs)
+        ctx.op = op
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        dx, dw = ctx.op.backward(dy)
+        ctx.op = None
+        return dx, dw, None, None
+
+
+def mxfp8_grouped_mm(x, w, offs, backward_override=None):
+    """y[rows of g] = x[rows of g] @ w[g]^T through the MXFP8 path, differentiable.
+
+    x bf16 [M, K], w bf16 [G, N, K], offs int32 [G] on the device (cumulative
+    group ends). ``backward_override`` as in MXFP8GroupedMM (ao "[moe
+    training] Add backward_override to the MXFP8 grouped GEMM", Design notes).
+    """
+    return _GroupedMMFn.apply(x, w, offs, backward_override)
+
+
+class _LinearFn(torch.autograd.Function):
+    """Autograd wrapper of the MXFP8 linear (mx_linear_fwd / mx_linear_bwd)."""
+
+    @staticmethod
+    def forward(ctx, x, w, cache):
+        x, w = _check_bf16(x), _check_bf16(w)
+        version = w._version
+        M, K = x.shape
+        N = w.shape[0]
+        ws = linear_workspace(M, N, K, x.device)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        mx_linear_fwd(x, w, cache, version, y, ws)
+        ctx.save_for_backward(x, w)
+        ctx.cache, ctx.version, ctx.ws = cache, version, ws
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, w = ctx.saved_tensors
+        dy = _check_bf16(dy)
+        M, K = x.shape
+        N = w.shape[0]
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
+        dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
+        mx_linear_bwd(dy, x, w, ctx.cache, ctx.version, dx, dw, ctx.ws)
+        ctx.ws = None
+        return dx, dw, None
+
+
+def mxfp8_linear(x, w, cache=None):
+    """y = x @ w^T through the MXFP8 linear, differentiable (ao PR #4705,
+    "MXFP8Linear training paths"). With a WeightCache, the 32x32 quantization
+    of w is reused while w's version counter is unchanged."""
+    return _LinearFn.apply(x, w, cache)

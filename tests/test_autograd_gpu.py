@@ -1,0 +1,70 @@
+"""The autograd entry points give exactly the library calls' results."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mx_oracle as O
+from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from mxfp8_block_scaled_cast_b200 import mx as _mx
+    _mx.lib()
+    return _mx
+
+
+@pytest.mark.parametrize("arm", [None, "high_precision", "dequantized"])
+def test_grouped_mm_autograd_equals_module(mx, arm):
+    sizes = [90, 0, 333, 200, 377]
+    M, G, N, K = sum(sizes), len(sizes), 256, 512
+    x = S.normal_bf16((M, K), seed=1).cuda().requires_grad_()
+    w = S.normal_bf16((G, N, K), 0.02, seed=2).cuda().requires_grad_()
+    dy = S.normal_bf16((M, N), 0.1, seed=3).cuda()
+    offs = S.offsets_from_sizes(sizes).cuda()
+    y = mx.mxfp8_grouped_mm(x, w, offs, backward_override=arm)
+    y.backward(dy)
+    op = mx.MXFP8GroupedMM(backward_override=arm)
+    y_ref = op.forward(x.detach(), w.detach(), offs)
+    dx_ref, dw_ref = op.backward(dy)
+    mx.mx_device_error()
+    assert torch.equal(y, y_ref)
+    assert torch.equal(x.grad, dx_ref) and torch.equal(w.grad, dw_ref)
+
+
+def test_grouped_mm_autograd_stride0_grad(mx):
+    """out.sum().backward() hands the backward an expanded (stride-0) gradient."""
+    sizes = [128, 256]
+    x = S.normal_bf16((384, 256), seed=4).cuda().requires_grad_()
+    w = S.normal_bf16((2, 256, 256), 0.02, seed=5).cuda().requires_grad_()
+    offs = S.offsets_from_sizes(sizes).cuda()
+    mx.mxfp8_grouped_mm(x, w, offs).float().sum().backward()
+    mx.mx_device_error()
+    ones = torch.ones(384, 256, dtype=torch.bfloat16)
+    op = mx.MXFP8GroupedMM()
+    op.forward(x.detach(), w.detach(), offs)
+    dx_ref, dw_ref = op.backward(ones.cuda())
+    assert torch.equal(x.grad, dx_ref) and torch.equal(w.grad, dw_ref)
+
+
+def test_linear_autograd_with_cache(mx):
+    x = S.normal_bf16((256, 512), seed=6).cuda().requires_grad_()
+    w = S.normal_bf16((256, 512), 0.02, seed=7).cuda().requires_grad_()
+    dy = S.normal_bf16((256, 256), 0.1, seed=8).cuda()
+    cache = mx.WeightCache()
+    y1 = mx.mxfp8_linear(x, w, cache)
+    y1.backward(dy)
+    g1 = (x.grad.clone(), w.grad.clone())
+    x.grad = None
+    w.grad = None
+    y2 = mx.mxfp8_linear(x, w, cache)                 # cache hit: bitwise the same
+    y2.backward(dy)
+    mx.mx_device_error()
+    assert cache.stats()["hits"] >= 1
+    assert torch.equal(y1, y2) and torch.equal(g1[0], x.grad) and torch.equal(g1[1], w.grad)
+    ref, absref = O.linear_fwd(S.bf16_bits(x.detach().cpu()), S.bf16_bits(w.detach().cpu()))
+    err = np.abs(y1.float().cpu().numpy() - ref)
+    assert np.all(err <= O.gemm_bound(ref, absref))
+    cache.close()
