@@ -65,6 +65,6 @@ def test_linear_autograd_with_cache(mx):
     assert cache.stats()["hits"] >= 1
     assert torch.equal(y1, y2) and torch.equal(g1[0], x.grad) and torch.equal(g1[1], w.grad)
     ref, absref = O.linear_fwd(S.bf16_bits(x.detach().cpu()), S.bf16_bits(w.detach().cpu()))
-    err = np.abs(y1.float().cpu().numpy() - ref)
+    err = np.abs(y1.detach().float().cpu().numpy() - ref)
     assert np.all(err <= O.gemm_bound(ref, absref))
     cache.close()
