@@ -43,6 +43,10 @@ What it computes, and where each step comes from
   dW_g = 0. Computed here in float64 over the dequantized operands.
 * MXFP8 linear forward / dgrad / wgrad ("MXFP8Linear training paths", ao PR
   #4705) composed from the casts above at one group.
+* Backward-override arms (ao backward_override PR, Design notes): the
+  high-precision arm's two bf16 grouped GEMMs over unpadded groups, the
+  dequantized arm's dequantization of the forward's codes to bf16 (round to
+  nearest even), and the grouped dequant that gathers padded rows back.
 
 Where the pages are silent, the readings taken are listed in the repository's
 design notes; each is restated beside the function that depends on it.
