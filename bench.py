@@ -18,7 +18,11 @@ value = 3 * 2*M*N*K FLOPs per step / step time (TFLOP/s, whole job). Inputs
 are seeded synthetic bf16 tensors on the device (512 MB > the 126 MB L2, so
 no explicit flush between steps). The cast bandwidth of the four cast modes
 on the 16384^2 sweep tensor and the [64, 2048, 7168] expert stack is
-reported beside it (L2 flushed between iterations).
+reported beside it (L2 flushed between iterations), and so are the GEMMs
+alone (CUDA-graph replays), the MXFP8 linear at M=4096, N=4096, K=2048, the
+unaligned geometry (casts of a [16384, 576] gradient; the grouped GEMMs at
+G=32, K=7168, N=2048, M=32768 with skewed groups) and the backward-override
+arms.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs the same step on its own GPU (replicas: the
@@ -175,52 +179,62 @@ class L2Flush:
 
 # ------------------------------------------------------------ our step ----
 class MoEStep:
-    """Preallocated buffers and the six launches of one MoE fwd+bwd step."""
+    """Preallocated buffers and the six launches of one MoE fwd+bwd step.
 
-    def __init__(self, mx, device, seed=0):
+    `problem` builds (x, w, dy, offs) for groups G, tokens M, output width N and
+    input width K; the default is the MoE benchmark shape."""
+
+    def __init__(self, mx, device, seed=0, shape=(G, M, N, K), problem=None):
         import torch
         from mxfp8_block_scaled_cast_b200 import synthetic as S
         self.mx, self.torch = mx, torch
-        self.x, self.w, self.dy, offs = S.moe_problem(G, M, N, K, seed=seed, device=device)
+        g, m, n, k = self.G, self.M, self.N, self.K = shape
+        make = problem or S.moe_problem
+        self.x, self.w, self.dy, offs = make(G=g, M=m, N=n, K=k, seed=seed, device=device)
         self.offs = offs.to(device)
-        cap = self.cap = mx.mx_padded_rows_capacity(M, G)
+        cap = self.cap = mx.mx_padded_rows_capacity(m, g)
         u8 = lambda *s: torch.empty(*s, dtype=torch.uint8, device=device)
         bf = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device=device)
-        self.xq, self.xs = u8(cap, K), u8(mx.mx_scale_bytes(cap, K // 32))
-        self.xqt, self.xst = u8(K, cap), u8(mx.mx_scale_bytes(K, cap // 32))
-        self.wq, self.wsf = u8(G, N, K), u8(G * mx.mx_scale_bytes(N, K // 32))
-        self.wsd = u8(G * mx.mx_scale_bytes(K, N // 32))
-        self.dq, self.ds = u8(cap, N), u8(mx.mx_scale_bytes(cap, N // 32))
-        self.dqt, self.dst = u8(N, cap), u8(mx.mx_scale_bytes(N, cap // 32))
-        self.y, self.dx, self.dw = bf(M, N), bf(M, K), bf(G, N, K)
+        self.xq, self.xs = u8(cap, k), u8(mx.mx_scale_bytes(cap, k // 32))
+        self.xqt, self.xst = u8(k, cap), u8(mx.mx_scale_bytes(k, cap // 32))
+        self.wq, self.wsf = u8(g, n, k), u8(g * mx.mx_scale_bytes(n, k // 32))
+        self.wsd = u8(g * mx.mx_scale_bytes(k, n // 32))
+        self.dq, self.ds = u8(cap, n), u8(mx.mx_scale_bytes(cap, n // 32))
+        self.dqt, self.dst = u8(n, cap), u8(mx.mx_scale_bytes(n, cap // 32))
+        self.y, self.dx, self.dw = bf(m, n), bf(m, k), bf(g, n, k)
         self.launches_per_step = 6
+        self.gemm_flops = 2 * m * n * k
         self.gemm_events = []
+
+    def gemms(self):
+        """The three grouped GEMMs of the step, as callables (fwd, dgrad, wgrad)."""
+        mx, g, m, n, k = self.mx, self.G, self.M, self.N, self.K
+        return {
+            "fwd": lambda: mx.mx_grouped_mm(self.xq, self.xs, self.wq, self.wsf, self.offs, g, mx.MX_GROUPS_M,
+                                            self.y, m, n, k, self.cap),
+            "dgrad": lambda: mx.mx_grouped_mm(self.dq, self.ds, self.wq, self.wsd, self.offs, g,
+                                              mx.MX_GROUPS_M_KN, self.dx, m, k, n, self.cap),
+            "wgrad": lambda: mx.mx_grouped_mm(self.dqt, self.dst, self.xqt, self.xst, self.offs, g,
+                                              mx.MX_GROUPS_K, self.dw, m, n, k, self.cap),
+        }
 
     def run(self, timed_gemms=False):
         mx, t = self.mx, self.torch
         mx.mx_cast_2d_grouped(self.x, self.offs, self.cap, self.xq, self.xs, self.xqt, self.xst)
         mx.mx_cast_w32x32(self.w, self.wq, self.wsf, None, self.wsd)
-        gemms = (
-            lambda: mx.mx_grouped_mm(self.xq, self.xs, self.wq, self.wsf, self.offs, G, mx.MX_GROUPS_M, self.y,
-                                     M, N, K, self.cap),
-            None,
-            lambda: mx.mx_grouped_mm(self.dq, self.ds, self.wq, self.wsd, self.offs, G, mx.MX_GROUPS_M_KN,
-                                     self.dx, M, K, N, self.cap),
-            lambda: mx.mx_grouped_mm(self.dqt, self.dst, self.xqt, self.xst, self.offs, G, mx.MX_GROUPS_K,
-                                     self.dw, M, N, K, self.cap),
-        )
-        for i, g in enumerate(gemms):
-            if g is None:
+        calls = self.gemms()
+        for name in ("fwd", None, "dgrad", "wgrad"):
+            if name is None:
                 mx.mx_cast_2d_grouped(self.dy, self.offs, self.cap, self.dq, self.ds, self.dqt, self.dst)
                 continue
             if timed_gemms:
                 a, b = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
                 a.record()
-                g()
+                calls[name]()
                 b.record()
                 self.gemm_events.append((a, b))
             else:
-                g()
+                calls[name]()
 
 
 def cast_sweep(mx, device, flush):
@@ -270,25 +284,17 @@ def cast_sweep(mx, device, flush):
 
 
 def gemm_only(mx, step, peaks, iters=100, runs=5):
-    """The three grouped GEMMs of the step alone, on the step's prequantized
+    """The three grouped GEMMs of a step alone, on the step's prequantized
     operands: each captured as a CUDA graph of `iters` launches and replayed
-    `runs` times; median time per launch. No flush (operands 201-335 MB per
-    launch, above the 126 MB L2)."""
+    `runs` times; median time per launch. No flush (the MoE launches move
+    201-335 MB of operands, above the 126 MB L2)."""
     import torch
     step.run()
     torch.cuda.synchronize()
-    calls = {
-        "fwd": lambda: mx.mx_grouped_mm(step.xq, step.xs, step.wq, step.wsf, step.offs, G, mx.MX_GROUPS_M,
-                                        step.y, M, N, K, step.cap),
-        "dgrad": lambda: mx.mx_grouped_mm(step.dq, step.ds, step.wq, step.wsd, step.offs, G, mx.MX_GROUPS_M_KN,
-                                          step.dx, M, K, N, step.cap),
-        "wgrad": lambda: mx.mx_grouped_mm(step.dqt, step.dst, step.xqt, step.xst, step.offs, G, mx.MX_GROUPS_K,
-                                          step.dw, M, N, K, step.cap),
-    }
     out = {}
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_OVER_BF16
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP8_OVER_BF16
-    for name, fn in calls.items():
+    for name, fn in step.gemms().items():
         fn()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -309,7 +315,7 @@ def gemm_only(mx, step, peaks, iters=100, runs=5):
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b) / iters)
         ts.sort()
-        tf = GEMM_FLOPS / (ts[len(ts) // 2] * 1e-3) / 1e12
+        tf = step.gemm_flops / (ts[len(ts) // 2] * 1e-3) / 1e12
         out[name] = {"us_per_launch": round(ts[len(ts) // 2] * 1e3, 1), "tflops": round(tf, 1),
                      "frac_of_measured_sustained_fp8": round(tf / sustained, 3),
                      "frac_of_measured_burst_fp8": round(tf / burst, 3), "frac_of_4500_spec": round(tf / 4500.0, 3)}
@@ -317,6 +323,54 @@ def gemm_only(mx, step, peaks, iters=100, runs=5):
     mx.mx_device_error()
     out["method"] = (f"CUDA graph of {iters} back-to-back launches (power-capped), median of {runs} replays; "
                      f"fp8 peaks = measured bf16 (sustained, burst) x {FP8_OVER_BF16}")
+    return out
+
+
+def unaligned_bench(mx, device, flush, peaks):
+    """The unaligned geometry: the casts of a [16384, 576] gradient (576 = 18
+    blocks of 32, scale columns padded to 20; L2 flushed between iterations; the
+    tensor is L2-sized, so this is reported, not graded) and the three grouped
+    GEMMs at G=32, K=7168, N=2048, M=32768 with Zipf(1.2) group sizes that are
+    not multiples of 128 and three empty groups (pad path; graph-replayed like
+    the GEMM-only timing)."""
+    import torch
+    from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2] * 1e-3
+
+    out = {}
+    r, c = 16384, 576
+    dy = S.sweep_tensor((r, c), seed=0, device=device)
+    u8 = lambda *s: torch.empty(*s, dtype=torch.uint8, device=device)
+    q, s, qt, st = u8(r, c), u8(mx.mx_scale_bytes(r, c // 32)), u8(c, r), u8(mx.mx_scale_bytes(c, r // 32))
+    modes = {
+        "dim0": (lambda: mx.mx_cast_dim0(dy, q, s), 2 + 1 + 1 / 32),
+        "dim1": (lambda: mx.mx_cast_dim1(dy, qt, st), 2 + 1 + 1 / 32),
+        "2d": (lambda: mx.mx_cast_2d(dy, q, s, qt, st), 2 + 2 + 2 / 32),
+    }
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    for name, (fn, bpe) in modes.items():
+        gbs = r * c * bpe / timed(fn) / 1e9
+        out[f"{name}_{r}x{c}_gbs"] = {"gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm, 3)}
+    del dy, q, s, qt, st
+    step = MoEStep(mx, device, seed=0, shape=(32, 32768, 2048, 7168), problem=S.unaligned_grouped_problem)
+    out["grouped_gemm_G32_K7168_N2048_M32768"] = gemm_only(mx, step, peaks)
+    out["grouped_gemm_G32_K7168_N2048_M32768"]["gflop_per_launch"] = round(step.gemm_flops / 1e9, 1)
+    del step
+    torch.cuda.empty_cache()
     return out
 
 
@@ -547,6 +601,8 @@ def main(argv=None):
     p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
     p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
     p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
+    p.add_argument("--no-unaligned", action="store_true",
+                   help="skip the unaligned geometry ([16384, 576] casts, G=32 skewed grouped GEMMs)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--ref-tokens", type=int, default=512)
     args = p.parse_args(argv)
@@ -669,6 +725,11 @@ def main(argv=None):
     if not args.no_linear:
         flush = L2Flush(dev)
         linear = linear_bench(mx, dev, flush, peaks)
+    unaligned = None
+    if not args.no_unaligned:
+        flush = L2Flush(dev)
+        unaligned = unaligned_bench(mx, dev, flush, peaks)
+        del flush
     arms = None
     if not args.no_arms:
         flush = L2Flush(dev)
@@ -698,6 +759,7 @@ def main(argv=None):
         "backward_overrides": arms,
         "linear": linear,
         "gemm_only": gemm_alone,
+        "unaligned": unaligned,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

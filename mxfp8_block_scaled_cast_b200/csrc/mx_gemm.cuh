@@ -165,7 +165,8 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
 // stores, which then overlap the next tile's main loop. The 32-column subtile
 // shared with the other slot is drained first and released at once
 // (`leader_ovl`), then the rest of the slot (`leader_free`), both barriers of
-// the pair's leader CTA.
+// the pair's leader CTA, with relaxed arrives (the columns are read out, no
+// data is handed over).
 // Stores are coalesced: per 32-column chunk the warp's 32 rows go through a
 // 2 KB shared buffer (16-byte pieces XOR-swizzled by row so both sides are
 // bank-conflict free), then each instruction writes 8 rows x 64 contiguous
@@ -186,7 +187,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot,
   auto release_shared_subtile = [&]() {
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(leader_ovl);
+    if (lane == 0) mbar_arrive_cluster_relaxed(leader_ovl);
   };
   if (slot) {              // shared subtile = chunk 0 of slot 1
     drain(0);
@@ -201,10 +202,12 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot,
   }
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive_cluster(leader_free);
-  const bool valid = dst != nullptr;
-  const uint32_t out_lo = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst)) : 0u;
-  const uint32_t out_hi = valid ? uint32_t(reinterpret_cast<uintptr_t>(dst) >> 32) : 0u;
+  if (lane == 0) mbar_arrive_cluster_relaxed(leader_free);
+  // the rows this lane stores from, gathered once: row i * 8 + lane / 4, i < 4
+  const uint64_t mine = reinterpret_cast<uintptr_t>(dst);
+  uint64_t rows[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) rows[i] = __shfl_sync(0xFFFFFFFFu, mine, i * 8 + (lane >> 2));
 #pragma unroll
   for (int chunk = 0; chunk < kBN / 32; ++chunk) {
 #pragma unroll
@@ -219,11 +222,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot,
     for (int i = 0; i < 4; ++i) {
       const int rr = i * 8 + (lane >> 2);       // row within the warp's 32
       const int k = lane & 3;                   // 16-byte piece within the 64-byte segment
-      const uint32_t lo = __shfl_sync(0xFFFFFFFFu, out_lo, rr);
-      const uint32_t hi = __shfl_sync(0xFFFFFFFFu, out_hi, rr);
       const uint4 val = *reinterpret_cast<const uint4*>(stage_buf + rr * 64 + ((uint32_t(k) ^ ((uint32_t(rr) >> 1) & 3u)) * 16));
-      if (lo | hi) {
-        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>((uint64_t(hi) << 32) | lo);
+      if (rows[i]) {
+        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(rows[i]);
         *reinterpret_cast<uint4*>(d + chunk * 32 + k * 8) = val;
       }
     }

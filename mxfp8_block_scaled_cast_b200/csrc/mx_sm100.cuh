@@ -213,6 +213,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
+// Arrive without release semantics, for a hand-back that carries no data: the
+// epilogue returning accumulator columns whose tcgen05.ld has completed
+// (tcgen05.wait::ld) before the arrive is issued. A cluster-scope release
+// would first wait for every global store the thread has in flight (the
+// previous tile's output rows), about a thousand cycles on the path between
+// one tile's last MMA and the next tile's first.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
 // 2D tiled load into this CTA's shared memory whose completion is counted on
 // an mbarrier that may live in the peer CTA of the pair (no multicast).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
