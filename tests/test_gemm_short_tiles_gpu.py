@@ -1,0 +1,107 @@
+"""The TMEM hand-back between consecutive tiles of a CTA pair, where it is
+exercised hardest: many groups of a few dozen tokens, so that almost every
+tile of the grouped GEMM is one or two 128-deep K steps (K groups) or a
+mostly empty 256-row band (M groups), and the pair moves from tile to tile
+every few hundred cycles.
+
+Each problem is launched four times back to back on one stream (no host
+synchronisation in between) into four outputs: all four must be bitwise
+equal (the kernel is deterministic: no atomics, fixed accumulation order),
+and one is checked against the float64 oracle on the same seeded inputs
+within |gpu - ref| <= 2^-7 |ref| + 1e-3 (|A| |B|^T)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mx_oracle as O
+from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from mxfp8_block_scaled_cast_b200 import mx as _mx
+    _mx.lib()
+    return _mx
+
+
+@pytest.fixture(scope="module")
+def sizes():
+    rng = np.random.default_rng(77)
+    s = rng.integers(1, 161, size=64).astype(np.int64)   # 1..160 tokens per group
+    s[[3, 17, 40]] = 0                                     # and a few empty groups
+    s[9] = 129                                             # one group of two K steps + 1 token
+    return s
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, absref, what):
+    bad = np.abs(got - ref) > O.gemm_bound(ref, absref)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance"
+
+
+def _four_launches(mx, call, out_like):
+    outs = [torch.full_like(out_like, float("nan")) for _ in range(4)]
+    for o in outs:
+        call(o)
+    torch.cuda.synchronize()
+    mx.mx_device_error()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16)), "launches differ"
+    return outs[0]
+
+
+def test_wgrad_many_one_step_groups(mx, sizes):
+    """dW_g = dY_g^T X_g for 64 token groups of 0..160 tokens: 1024 output tiles of one
+    or two K steps each."""
+    G, M, N, K = len(sizes), int(sizes.sum()), 1024, 1024
+    dyb = S.normal_bf16((M, N), 1e-2, seed=31)
+    xb = S.normal_bf16((M, K), 1.0, seed=32)
+    offs_t = S.offsets_from_sizes(sizes)
+    offs = offs_t.numpy()
+    cap = mx.mx_padded_rows_capacity(M, G)
+    dqt, dst = mx.cast_dim1_grouped(dyb.cuda(), offs_t.cuda(), cap)
+    xqt, xst = mx.cast_dim1_grouped(xb.cuda(), offs_t.cuda(), cap)
+    od = offs_t.cuda()
+    like = torch.empty(G, N, K, dtype=torch.bfloat16, device="cuda")
+    dw = _four_launches(mx, lambda o: mx.mx_grouped_mm(dqt, dst, xqt, xst, od, G, mx.MX_GROUPS_K, o, M, N, K, cap),
+                        like)
+    oa, osa = O.cast_dim1_grouped(S.bf16_bits(dyb), offs, cap)
+    ob, osb = O.cast_dim1_grouped(S.bf16_bits(xb), offs, cap)
+    a, b = O.dequant(oa, osa), O.dequant(ob, osb)
+    _close(_f64(dw), O.grouped_mm_k(a, b, offs), O.grouped_mm_k(np.abs(a), np.abs(b), offs), "wgrad")
+    assert not dw[torch.from_numpy(sizes == 0).cuda()].any()
+
+
+def test_forward_and_dgrad_many_small_row_groups(mx, sizes):
+    """Y = X_g W_g^T and dX = dY_g W_g for the same 64 small groups: one mostly empty
+    256-row band per group, two K steps per tile."""
+    G, M, N, K = len(sizes), int(sizes.sum()), 1024, 256
+    xb = S.normal_bf16((M, K), 1.0, seed=33)
+    wb = S.normal_bf16((G, N, K), 0.02, seed=34)
+    dyb = S.normal_bf16((M, N), 1e-2, seed=35)
+    offs_t = S.offsets_from_sizes(sizes)
+    offs = offs_t.numpy()
+    cap = mx.mx_padded_rows_capacity(M, G)
+    od = offs_t.cuda()
+    xq, xs = mx.cast_dim0_grouped(xb.cuda(), od, cap)
+    dq, ds = mx.cast_dim0_grouped(dyb.cuda(), od, cap)
+    wq, wsf, _, wsd = mx.cast_w32x32(wb.cuda(), transposed=False, dgrad_scales=True)
+    y = _four_launches(mx, lambda o: mx.mx_grouped_mm(xq, xs, wq, wsf, od, G, mx.MX_GROUPS_M, o, M, N, K, cap),
+                       torch.empty(M, N, dtype=torch.bfloat16, device="cuda"))
+    dx = _four_launches(mx, lambda o: mx.mx_grouped_mm(dq, ds, wq, wsd, od, G, mx.MX_GROUPS_M_KN, o, M, K, N,
+                                                       cap),
+                        torch.empty(M, K, dtype=torch.bfloat16, device="cuda"))
+    qx, sx = O.cast_dim0_grouped(S.bf16_bits(xb), offs, cap)
+    qd, sd = O.cast_dim0_grouped(S.bf16_bits(dyb), offs, cap)
+    qw, st = O.cast_32x32(S.bf16_bits(wb))
+    s_fwd, s_dgrad = O.w32_scale_views(st)
+    ax, bw = O.dequant(qx, sx), O.dequant(qw, s_fwd)
+    _close(_f64(y), O.grouped_mm_m(ax, bw, offs), O.grouped_mm_m(np.abs(ax), np.abs(bw), offs), "forward")
+    ad = O.dequant(qd, sd)
+    bt = np.ascontiguousarray(np.transpose(bw, (0, 2, 1)))             # W_g^T: [G, K, N]
+    _close(_f64(dx), O.grouped_mm_m(ad, bt, offs), O.grouped_mm_m(np.abs(ad), np.abs(bt), offs), "dgrad")
