@@ -66,3 +66,26 @@ def test_reference_arm_other_ranks_exit_quietly():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                           "--warmup", "0"], capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_profile_traffic_is_null_once_the_kernel_changes(tmp_path, monkeypatch):
+    """`roofline.traffic` comes from a committed ncu summary only while the summary's
+    source hash matches the kernel sources; any edit of them turns it into null."""
+    import hashlib
+    import bench
+    srcs = ["csrc/k.cuh", "csrc/h.cuh"]
+    root = tmp_path / "repo"
+    (root / "csrc").mkdir(parents=True)
+    (root / "profiles").mkdir()
+    (root / srcs[0]).write_text("kernel\n")
+    (root / srcs[1]).write_text("header\n")
+    digest = hashlib.sha256(b"kernel\nheader\n").hexdigest()[:16]
+    (root / "profiles" / "k.txt").write_text(
+        "# a summary\ndram__bytes_read.sum: 1 MB\ntraffic_bytes_per_launch: 12345\n"
+        f"kernel_source_sha256_16: {digest}\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.profile_traffic("k.txt", srcs) == pytest.approx(12345.0)
+    with open(root / srcs[0], "a") as f:
+        f.write("// edited\n")
+    assert bench.profile_traffic("k.txt", srcs) is None
+    assert bench.profile_traffic("missing.txt", srcs) is None
