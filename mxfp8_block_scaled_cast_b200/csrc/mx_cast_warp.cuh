@@ -82,8 +82,6 @@ cast_warp_kernel(const CastArgs a) {
   __shared__ GroupSlot slots[kWarpCastWarps];
   __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
   __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
-  pdl_launch_dependents();
-  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t c0 = int64_t(blockIdx.x) * kCastTile;
   const int64_t r0 = int64_t(blockIdx.y) * kCastTile;

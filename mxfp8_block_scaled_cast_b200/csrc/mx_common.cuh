@@ -24,18 +24,6 @@ enum : unsigned { kErrTimeout = 1u, kErrOffsets = 2u };
 
 __device__ __forceinline__ void flag_error(unsigned bits) { atomicOr(&g_device_error, bits); }
 
-// Programmatic dependent launch. Kernels of the library are launched with
-// programmatic stream serialization: the next kernel in the stream may be
-// scheduled while this one finishes, and runs its set-up meanwhile. Every
-// kernel lets its dependents launch at once (pdl_launch_dependents) and, in
-// every thread, waits for the previous kernel in the stream to complete and
-// its writes to become visible (pdl_wait) before its first global-memory
-// read or write -- unconditionally, so that no grid completes before the one
-// it follows and the ordering stays transitive. Both are no-ops for a launch
-// without the attribute.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t x, int64_t a) { return (x + a - 1) / a; }
 __host__ __device__ __forceinline__ int64_t ceil_to(int64_t x, int64_t a) { return ceil_div(x, a) * a; }
 

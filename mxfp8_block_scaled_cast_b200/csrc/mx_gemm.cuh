@@ -246,7 +246,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  pdl_launch_dependents();
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();      // 0 = leader of the pair
@@ -290,7 +289,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish_pair();
   }
-  pdl_wait();              // global memory from here on: after the previous kernel in the stream
   if (warp == 0) {
     // group table: ends[g], padded starts pstart[0..G], 256-row tile starts tstart[0..G]
     bool bad = false;

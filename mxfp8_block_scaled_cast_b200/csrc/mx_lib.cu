@@ -46,14 +46,6 @@ mx_status cuda_check(const char* what) {
     if (!(cond)) return fail(st, __VA_ARGS__); \
   } while (0)
 
-// Programmatic stream serialization: the kernel may be scheduled while the
-// previous kernel in the stream finishes; each kernel of the library waits for
-// it (griddepcontrol.wait) before touching global memory.
-void set_pdl_attribute(cudaLaunchAttribute& attr) {
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-}
-
 template <int kMode, bool kGrouped>
 mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
                       cudaStream_t stream) {
@@ -63,18 +55,8 @@ mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, i
   MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth <= 65535, MX_ERR_UNSUPPORTED,
              "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles,
              (long long)depth);
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
-  set_pdl_attribute(attr[0]);
-  cfg.gridDim = dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth));
-  cfg.blockDim = dim3(kWarpCastThreads, 1, 1);
-  cfg.dynamicSmemBytes = kWarpCastSmem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, cast_warp_kernel<kMode, kGrouped>, a);
-  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "cast launch: %s", cudaGetErrorString(e));
+  cast_warp_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)),
+                                      kWarpCastThreads, kWarpCastSmem, stream>>>(a);
   return cuda_check("cast launch");
 }
 
@@ -180,7 +162,7 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -199,8 +181,6 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   }
   const int64_t pairs = pair_tiles_ub < max_pairs[dev] ? pair_tiles_ub : max_pairs[dev];
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
-  set_pdl_attribute(attr[1]);
-  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, mx_gemm_kernel<kMode>, ma, mb, msa, msb, ga);
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return cuda_check("gemm launch");
@@ -237,7 +217,7 @@ mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const H
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm smem attribute: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -256,8 +236,6 @@ mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const H
   }
   const int64_t pairs = pair_tiles_ub < max_pairs[dev] ? pair_tiles_ub : max_pairs[dev];
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
-  set_pdl_attribute(attr[1]);
-  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, bf16_gemm_kernel<kMode>, ma, mb, ha);
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm launch: %s", cudaGetErrorString(e));
   return cuda_check("bf16 gemm launch");
