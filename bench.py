@@ -95,7 +95,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period_s=0.02):
+    def __init__(self, index, period_s=0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.index = period_s, index
         self._stop = threading.Event()
@@ -603,7 +603,7 @@ def main(argv=None):
     p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
     p.add_argument("--no-unaligned", action="store_true",
                    help="skip the unaligned geometry ([16384, 576] casts, G=32 skewed grouped GEMMs)")
-    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--e2e-steps", type=int, default=None, help="end-to-end steps (default: --steps)")
     p.add_argument("--ref-tokens", type=int, default=512)
     args = p.parse_args(argv)
     rank, world, local = dist_env()
@@ -648,7 +648,10 @@ def main(argv=None):
     gemm_ms = [a.elapsed_time(b) for a, b in step.gemm_events]
     gemm_avg_s = sum(gemm_ms) / len(gemm_ms) * 1e-3
     gemm_tflops = GEMM_FLOPS / gemm_avg_s / 1e12
-    bf16_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # The timed region is a burst (tens of milliseconds), so the in-step GEMM
+    # rate is held against the burst figure; the sustained figure applies to
+    # the seconds-long back-to-back replays of `gemm_only`.
+    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     fp8_peak = bf16_peak * FP8_OVER_BF16
     traffic = profile_traffic("mx_gemm_kernel_moe_G8_K4096_N4096.txt",
                               ["mxfp8_block_scaled_cast_b200/csrc/mx_gemm.cuh",
@@ -706,11 +709,12 @@ def main(argv=None):
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    e2e_run(args.e2e_steps, start_event=a)
+    e2e_steps = args.steps if args.e2e_steps is None else args.e2e_steps
+    e2e_run(e2e_steps, start_event=a)
     b.record()
     torch.cuda.synchronize()
     mx.mx_device_error()
-    e2e_value, _ = aggregate(a.elapsed_time(b) / args.e2e_steps, args.e2e_steps, world)
+    e2e_value, _ = aggregate(a.elapsed_time(b) / e2e_steps, e2e_steps, world)
     del sets[1]
 
     casts = None
@@ -748,10 +752,12 @@ def main(argv=None):
                    "l2": "inputs 512 MB > 126 MB L2 (no flush between steps)", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel (fwd, dgrad, wgrad launches)",
                      "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
-                     "peak_source": f"{peak_src} bf16 sustained {bf16_peak} x {FP8_OVER_BF16} (nominal fp8/bf16)",
+                     "peak_source": f"{peak_src} bf16 burst {bf16_peak} x {FP8_OVER_BF16} (nominal fp8/bf16); "
+                                    f"burst because the timed region lasts {total_ms:.1f} ms",
                      "frac_of_4500_spec": gemm_tflops / 4500.0, "traffic": traffic,
                      "flops_per_launch": GEMM_FLOPS, "avg_launch_ms": gemm_avg_s * 1e3},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
