@@ -265,13 +265,27 @@ MX_API mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void
  * Weight cache ("Cache quantized weights for full AC", prime-rl PR #3388,
  * Overview): with cache != NULL the 32x32 quantization of w is kept in
  * device memory owned by the cache, keyed by (w address, N, K) and reused
- * while w_version (the caller's in-place update counter of w) is unchanged;
- * a changed version re-quantizes in place. Results are bitwise identical
- * with and without a hit. mx_wcache_clear() frees every entry (call it
- * after backward; it synchronizes the device). The cache is thread-safe;
- * an entry must not be cleared while work that reads it is in flight. */
+ * while w_version is unchanged; a changed version re-quantizes in place.
+ * Results are bitwise identical with and without a hit.
+ * The key is an address, and an allocator may hand a freed weight's address
+ * to a new tensor whose own update counter starts where the old one's did;
+ * a hit would then return the old weight's codes. So w_version must change
+ * whenever the bytes at w change OR w names a different tensor: a caller
+ * either folds a per-tensor identity that is never reused into w_version,
+ * or calls mx_wcache_evict(cache, w) when the tensor at w is freed (before
+ * its memory can be reused). The Python binding does both.
+ * mx_wcache_evict() unbinds the entries of address w without freeing them
+ * (no device synchronization; a later miss of the same N, K reuses the
+ * buffer, stream-ordered after the work already issued on that call's
+ * stream; work on other streams that still reads the entry must be ordered
+ * before that miss). Call it after a weight's backward to drop the entry
+ * ("clear the cache after backward", same page). mx_wcache_clear() frees
+ * every entry, bound or not (it synchronizes the device). The cache is
+ * thread-safe; an entry must not be cleared while work that reads it is in
+ * flight. mx_wcache_stats() counts hits, misses and bound entries. */
 typedef struct mx_wcache mx_wcache;
 MX_API mx_wcache* mx_wcache_create(void);
+MX_API void mx_wcache_evict(mx_wcache* cache, const void* w);
 MX_API void mx_wcache_clear(mx_wcache* cache);
 MX_API void mx_wcache_destroy(mx_wcache* cache);
 MX_API mx_status mx_wcache_stats(mx_wcache* cache, int64_t* hits, int64_t* misses, int64_t* entries);
@@ -304,7 +318,8 @@ MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
  *
  * The first call on a device looks up the array's device address on that
  * device (cudaGetSymbolAddress); make that first call before any stream
- * capture. Every call shares the one array and leaves its contents behind
+ * capture. The address is kept for the life of the process, so a caller
+ * must not reset the device (cudaDeviceReset) after its first call. Every call shares the one array and leaves its contents behind
  * (each call rewrites every byte it reads, so nothing is cleared): calls
  * whose work overlaps on the GPU (other streams, other host threads) race
  * on it, so order them. Same size rules as mx_linear_fwd. */

@@ -474,6 +474,16 @@ void mx_wcache_clear(mx_wcache* c) {
   c->entries.clear();
 }
 
+void mx_wcache_evict(mx_wcache* c, const void* w) {
+  if (c == nullptr) return;
+  std::lock_guard<std::mutex> lk(c->mu);
+  for (auto& e : c->entries)
+    if (e.w == w && w != nullptr) {
+      e.w = nullptr;          // unbound: the buffer waits for a miss of the same shape
+      e.valid = false;
+    }
+}
+
 void mx_wcache_destroy(mx_wcache* c) {
   mx_wcache_clear(c);
   delete c;
@@ -484,7 +494,11 @@ mx_status mx_wcache_stats(mx_wcache* c, int64_t* hits, int64_t* misses, int64_t*
   std::lock_guard<std::mutex> lk(c->mu);
   if (hits) *hits = c->hits;
   if (misses) *misses = c->misses;
-  if (entries) *entries = int64_t(c->entries.size());
+  if (entries) {
+    int64_t bound = 0;
+    for (const auto& e : c->entries) bound += e.w != nullptr;
+    *entries = bound;
+  }
   return MX_OK;
 }
 
@@ -530,6 +544,14 @@ mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, ui
     return MX_OK;
   }
   ++cache->misses;
+  if (e == nullptr) {            // an evicted entry's buffer of the same shape, if any
+    for (auto& x : cache->entries)
+      if (x.w == nullptr && x.N == N && x.K == K) {
+        e = &x;
+        e->w = w;
+        break;
+      }
+  }
   if (e == nullptr) {
     uint8_t* buf = nullptr;
     cudaError_t err = cudaMalloc(&buf, size_t(wq_bytes(N, K)));
@@ -645,6 +667,13 @@ extern "C" mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
   MX_REQUIRE(N % kBN == 0 && K % kBN == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 256");
+  // Bound each factor before any product, so that no size can overflow the
+  // byte count below and slip past the scratch bound.
+  constexpr int64_t kScratch = int64_t(MX_LINEAR_NOALLOC_SCRATCH_BYTES);
+  MX_REQUIRE(M <= kScratch / K && N <= kScratch / K, MX_ERR_UNSUPPORTED,
+             "mx_linear_fwd_noalloc: M=%lld N=%lld K=%lld exceed its static scratch of %lld bytes (use "
+             "mx_linear_fwd with a workspace)",
+             (long long)M, (long long)N, (long long)K, (long long)kScratch);
   const int64_t xq_b = ceil_to(M * K, 256), xs_b = ceil_to(scale_bytes(M, K / kBlock), 256);
   const int64_t wq_b = ceil_to(N * K, 256), ws_b = ceil_to(scale_bytes(N, K / kBlock), 256);
   const int64_t need = xq_b + xs_b + wq_b + ws_b;

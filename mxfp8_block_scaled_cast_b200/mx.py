@@ -10,7 +10,9 @@ is no fallback: if libmx.so is missing or no GPU is present, calls raise.
 from __future__ import annotations
 
 import ctypes
+import itertools
 import os
+import weakref
 
 import torch
 
@@ -34,6 +36,7 @@ _SIGNATURES = {
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
     "mx_wcache_create": (_vp, []),
+    "mx_wcache_evict": (None, [_vp, _vp]),
     "mx_wcache_clear": (None, [_vp]),
     "mx_wcache_destroy": (None, [_vp]),
     "mx_wcache_stats": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
@@ -193,6 +196,12 @@ def mx_linear_fwd_noalloc(x, w, y, stream=None):
     """Linear forward whose scratch is the library's fixed device array (no allocation)."""
     M, K = x.shape
     N = w.shape[0]
+    for name, t in (("x", x), ("w", w), ("y", y)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"mx_linear_fwd_noalloc takes bf16 tensors ({name} is {t.dtype})")
+    if w.dim() != 2 or w.shape[1] != K or tuple(y.shape) != (M, N):
+        raise ValueError(f"shapes must be x [M, K], w [N, K], y [M, N] (got {tuple(x.shape)}, "
+                         f"{tuple(w.shape)}, {tuple(y.shape)})")
     _call("mx_linear_fwd_noalloc", _p(x), _p(w), M, N, K, _p(y), _stream(stream))
 
 
@@ -213,13 +222,58 @@ def mx_scales_unswizzle(s, R, C32, out, stream=None):
     _call("mx_scales_unswizzle", _p(s), R, C32, _p(out), _stream(stream))
 
 
-class WeightCache:
-    """Owner of an mx_wcache: quantized weights reused while their version is unchanged."""
+def _evict_on_free(cache_ref, key, addrs):
+    """Finalizer of a tracked weight: unbind every address it was cached under."""
+    cache = cache_ref()
+    if cache is None:
+        return
+    cache._tracked.pop(key, None)
+    if cache.handle:
+        for a in addrs:
+            lib().mx_wcache_evict(cache.handle, ctypes.c_void_p(a))
 
-    def __init__(self):
+
+class WeightCache:
+    """Owner of an mx_wcache: quantized weights reused while their version is unchanged.
+
+    The library keys an entry by the weight's device address, and torch's
+    caching allocator readily hands a freed weight's block to the next tensor
+    of the same size, whose ``_version`` starts at 0 again. Two guards keep
+    such a tensor from receiving the freed weight's codes ("incorrect cache
+    invalidation could cause silent wrong numerics", prime-rl PR #3388,
+    Note): ``key_version`` folds a serial number that is never reused, one per
+    tensor object, into the version the library compares; and a finalizer on
+    every cached tensor unbinds its entries when it is garbage-collected.
+
+    ``clear_after_backward`` (default on): the MXFP8 linear's backward drops
+    the weight's entry when it has finished, as the page's cache is cleared
+    after backward (same page, Overview); a recompute forward inside the
+    backward (activation checkpointing) still hits.
+    """
+
+    _serials = itertools.count(1)
+
+    def __init__(self, clear_after_backward=True):
         self.handle = ctypes.c_void_p(lib().mx_wcache_create())
         if not self.handle:
             raise MemoryError("mx_wcache_create failed")
+        self.clear_after_backward = clear_after_backward
+        self._tracked = {}           # id(tensor) -> [weakref, serial, addresses, finalizer]
+
+    def key_version(self, w):
+        """The w_version to pass for ``w``: (serial of this tensor object << 32) | w._version."""
+        ent = self._tracked.get(id(w))
+        if ent is None or ent[0]() is not w:
+            addrs = set()
+            fin = weakref.finalize(w, _evict_on_free, weakref.ref(self), id(w), addrs)
+            ent = [weakref.ref(w), next(WeightCache._serials), addrs, fin]
+            self._tracked[id(w)] = ent
+        ent[2].add(w.data_ptr())
+        return (ent[1] << 32) | (w._version & 0xFFFFFFFF)
+
+    def evict(self, w):
+        """Unbind the entry of ``w`` (its buffer is kept for a later miss of the same shape)."""
+        lib().mx_wcache_evict(self.handle, ctypes.c_void_p(w.data_ptr()))
 
     def clear(self):
         lib().mx_wcache_clear(self.handle)
@@ -231,6 +285,9 @@ class WeightCache:
 
     def close(self):
         if self.handle:
+            for ent in list(self._tracked.values()):
+                ent[3].detach()
+            self._tracked.clear()
             lib().mx_wcache_destroy(self.handle)
             self.handle = ctypes.c_void_p(None)
 
@@ -348,14 +405,18 @@ def linear_workspace(M, N, K, device="cuda"):
     return torch.empty(mx_linear_ws_bytes(M, N, K), dtype=torch.uint8, device=device)
 
 
+def _version_of(w, cache):
+    return cache.key_version(w) if cache is not None else w._version
+
+
 def linear_fwd(x, w, cache=None, version=None, ws=None):
-    """y = x w^T through the MXFP8 path; version defaults to w._version."""
+    """y = x w^T through the MXFP8 path; version defaults to the cache's key for w."""
     x, w = _check_bf16(x), _check_bf16(w)
     M, K = x.shape
     N = w.shape[0]
     ws = linear_workspace(M, N, K, x.device) if ws is None else ws
     y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
-    mx_linear_fwd(x, w, cache, w._version if version is None else version, y, ws)
+    mx_linear_fwd(x, w, cache, _version_of(w, cache) if version is None else version, y, ws)
     return y
 
 
@@ -367,7 +428,7 @@ def linear_bwd(dy, x, w, cache=None, version=None, ws=None):
     ws = linear_workspace(M, N, K, x.device) if ws is None else ws
     dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
     dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
-    mx_linear_bwd(dy, x, w, cache, w._version if version is None else version, dx, dw, ws)
+    mx_linear_bwd(dy, x, w, cache, _version_of(w, cache) if version is None else version, dx, dw, ws)
     return dx, dw
 
 
@@ -536,7 +597,7 @@ class _LinearFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, x, w, cache):
         x, w = _check_bf16(x), _check_bf16(w)
-        version = w._version
+        version = _version_of(w, cache)
         M, K = x.shape
         N = w.shape[0]
         ws = linear_workspace(M, N, K, x.device)
@@ -555,6 +616,8 @@ class _LinearFn(torch.autograd.Function):
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
         dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
         mx_linear_bwd(dy, x, w, ctx.cache, ctx.version, dx, dw, ctx.ws)
+        if ctx.cache is not None and ctx.cache.clear_after_backward:
+            ctx.cache.evict(w)
         ctx.ws = None
         return dx, dw, None
 
@@ -562,5 +625,6 @@ class _LinearFn(torch.autograd.Function):
 def mxfp8_linear(x, w, cache=None):
     """y = x @ w^T through the MXFP8 linear, differentiable (ao PR #4705,
     "MXFP8Linear training paths"). With a WeightCache, the 32x32 quantization
-    of w is reused while w's version counter is unchanged."""
+    of w is reused while w is the same tensor with an unchanged version
+    counter, and (by default) dropped once w's backward has run."""
     return _LinearFn.apply(x, w, cache)

@@ -5,6 +5,8 @@ cache tests follow the cases named by "Cache quantized weights for full AC"
 (prime-rl PR #3388, Overview): hit/miss, in-place weight update, per-tensor
 isolation, and bit-identical results with and without a hit.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -133,3 +135,88 @@ def test_stride0_grad_is_materialised(mx):
     assert torch.equal(dx, dx2) and torch.equal(dw, dw2)
     with pytest.raises(ValueError):
         mx.mx_cast_2d(g, *mx.cast_2d(g.contiguous()))  # the raw entry refuses strided views
+
+
+class _DeviceMemory:
+    """A fresh tensor object over existing device memory (its own version counter, at 0)."""
+
+    def __init__(self, ptr, numel):
+        self.__cuda_array_interface__ = {"shape": (numel,), "typestr": "<i2", "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
+def _fresh_view(base, shape):
+    t = torch.as_tensor(_DeviceMemory(base.data_ptr(), base.numel()), device=base.device)
+    return t.view(torch.bfloat16).view(*shape)
+
+
+def test_cache_address_reuse_by_a_new_tensor_is_a_miss(mx):
+    """A weight freed and replaced by a different tensor at the same address, whose
+    _version is 0 again, must not get the freed weight's codes (prime-rl PR #3388,
+    Note: wrong invalidation gives silently wrong numerics)."""
+    x, _, _ = S.linear_problem(M=256, N=512, K=256, seed=9, device="cuda")
+    wa = S.normal_bf16((512 * 256,), 0.02, seed=10, device="cuda")
+    wb = S.normal_bf16((512 * 256,), 0.02, seed=11, device="cuda")
+    base = torch.empty(512 * 256, dtype=torch.bfloat16, device="cuda")
+    cache = mx.WeightCache()
+    base.copy_(wa)
+    w = _fresh_view(base, (512, 256))
+    assert w._version == 0
+    y_a = mx.linear_fwd(x, w, cache)
+    assert torch.equal(y_a, mx.linear_fwd(x, w, cache))            # hit
+    del w                                                           # the tensor is gone ...
+    base.copy_(wb)                                                  # ... its memory gets new bits
+    w2 = _fresh_view(base, (512, 256))                              # and a new tensor at that address
+    assert w2._version == 0
+    y_b = mx.linear_fwd(x, w2, cache)
+    torch.cuda.synchronize()
+    assert torch.equal(y_b, mx.linear_fwd(x, w2))                  # equals the no-cache forward
+    assert not torch.equal(y_b, y_a)
+    st = cache.stats()
+    assert st["hits"] == 1 and st["misses"] == 2
+    # a live alias (a second tensor object over the same memory) is its own entry too
+    w3 = _fresh_view(base, (512, 256))
+    mx.linear_fwd(x, w3, cache)
+    assert cache.stats()["misses"] == 3
+    cache.close()
+
+
+def test_cache_evict_through_the_c_abi(mx):
+    """A C caller that passes the same version for a new tensor at a freed weight's
+    address calls mx_wcache_evict when it frees the weight: the next call misses."""
+    x, _, _ = S.linear_problem(M=128, N=256, K=256, seed=12, device="cuda")
+    base = S.normal_bf16((256, 256), 0.02, seed=13, device="cuda")
+    other = S.normal_bf16((256, 256), 0.02, seed=14, device="cuda")
+    ws = mx.linear_workspace(128, 256, 256)
+    y = torch.empty(128, 256, dtype=torch.bfloat16, device="cuda")
+    cache = mx.WeightCache()
+    mx.mx_linear_fwd(x, base, cache, 0, y, ws)
+    mx.lib().mx_wcache_evict(cache.handle, ctypes.c_void_p(base.data_ptr()))
+    base.copy_(other)
+    mx.mx_linear_fwd(x, base, cache, 0, y, ws)                     # same address, same version: a miss
+    torch.cuda.synchronize()
+    assert torch.equal(y, mx.linear_fwd(x, other))
+    st = cache.stats()
+    assert st["misses"] == 2 and st["hits"] == 0 and st["entries"] == 1
+    cache.close()
+
+
+def test_linear_autograd_clears_the_entry_after_backward(mx):
+    """mxfp8_linear drops the weight's entry once its backward ran (prime-rl PR #3388,
+    Overview: the cache is cleared after backward); a recompute forward before the
+    backward (activation checkpointing) still hits."""
+    x = S.normal_bf16((256, 512), seed=15).cuda().requires_grad_()
+    w = S.normal_bf16((256, 512), 0.02, seed=16).cuda().requires_grad_()
+    dy = S.normal_bf16((256, 256), 0.1, seed=17).cuda()
+    cache = mx.WeightCache()
+    mx.mxfp8_linear(x, w, cache)                      # forward: miss
+    y = mx.mxfp8_linear(x, w, cache)                  # recompute forward: hit
+    assert cache.stats() == {"hits": 1, "misses": 1, "entries": 1}
+    y.backward(dy)                                    # backward: hit, then the entry is dropped
+    st = cache.stats()
+    assert st["hits"] == 2 and st["entries"] == 0
+    keep = mx.WeightCache(clear_after_backward=False)
+    mx.mxfp8_linear(x, w, keep).backward(dy)
+    assert keep.stats()["entries"] == 1
+    cache.close()
+    keep.close()
