@@ -103,6 +103,7 @@ struct GemmArgs {
   const int32_t* offs;         // cumulative group ends, or null for one dense group
   __nv_bfloat16* out;
   int G;
+  int E;                       // experts: group g uses expert g % E (E == G: one expert per group)
   int64_t M, N, K;             // see the mode description above
   int64_t m_cap;               // padded capacity (rows of A in M mode, token columns in K mode)
   int64_t a_sc_tiles;          // 4-column scale tiles (512-byte chunks) per 128-row band of A
@@ -111,9 +112,9 @@ struct GemmArgs {
 };
 
 struct TileInfo {
-  int g;
-  int nk;              // number of 128-deep K steps (0: empty K group)
-  int kt0;             // first K step (in units of 128)
+  int g;               // M modes: the group; K mode: the expert (output matrix)
+  int nk;              // number of 128-deep K steps (0: every K group of the expert is empty)
+  int kt0;             // M modes: first K step (in units of 128)
   int64_t m0;          // first row of A for the pair (M mode: padded row)
   int64_t b_row0;      // first row of B for the pair (global row of the TMA map)
   int64_t b_chunk0;    // scale chunk of B's first 128 rows at K step 0
@@ -125,7 +126,7 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
                                                 const int32_t* pstart, const int32_t* tstart) {
   TileInfo t;
   if (kMode != kGroupsK) {
-    const int64_t nt = a.N / kBN;
+    const int64_t nt = ceil_div(a.N, kBN);
     const int64_t mt = tile / nt;
     t.n0 = (tile % nt) * kBN;
     int lo = 0, hi = a.G;   // largest g with tstart[g] <= mt
@@ -135,25 +136,66 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
     }
     t.g = lo;
     t.m0 = pstart[t.g] + (mt - tstart[t.g]) * kPairM;
-    t.nk = int(a.K / kBK);
+    t.nk = int(ceil_div(a.K, kBK));
     t.kt0 = 0;
-    t.b_row0 = kMode == kGroupsMKn ? int64_t(t.g) * a.K : int64_t(t.g) * a.N + t.n0;
-    t.b_chunk0 = int64_t(t.g) * a.b_sc_group_chunks + (t.n0 / kCtaM) * a.b_sc_tiles;
+    const int64_t we = t.g % a.E;     // the group's expert
+    t.b_row0 = kMode == kGroupsMKn ? we * a.K : we * a.N + t.n0;
+    t.b_chunk0 = we * a.b_sc_group_chunks + (t.n0 / kCtaM) * a.b_sc_tiles;
   } else {
-    const int64_t nt = a.K / kBN, mt = a.N / kPairM;
-    const int64_t per_g = nt * mt;
-    t.g = int(tile / per_g);
-    const int64_t rem = tile % per_g;
+    // output matrix e sums the token steps of groups e, e + E, e + 2E, ...
+    const int64_t nt = ceil_div(a.K, kBN), mt = ceil_div(a.N, kPairM);
+    const int64_t per_e = nt * mt;
+    t.g = int(tile / per_e);
+    const int64_t rem = tile % per_e;
     t.m0 = (rem / nt) * kPairM;
     t.n0 = (rem % nt) * kBN;
-    const int64_t start = t.g ? ends[t.g - 1] : 0;
-    const int64_t size = ends[t.g] - start;
-    t.kt0 = int(pstart[t.g] / kBK);
-    t.nk = int((size + kBK - 1) / kBK);
+    t.kt0 = 0;
+    int64_t nk = 0;
+    for (int g = t.g; g < a.G; g += a.E) {
+      const int64_t start = g ? ends[g - 1] : 0;
+      nk += ceil_div(ends[g] - start, kBK);
+    }
+    t.nk = int(nk);
     t.b_row0 = t.n0;
     t.b_chunk0 = (t.n0 / kCtaM) * a.b_sc_tiles;
   }
   return t;
+}
+
+// The 128-deep K steps of a tile in order: in M modes steps kt0, kt0 + 1, ...;
+// in K mode the padded token steps of groups e, e + E, e + 2E, ... (the groups
+// of expert e, empty ones skipped).
+struct KWalk {
+  int g;          // current group (K mode)
+  int left;       // steps left in it
+  int64_t kk;     // current step
+};
+
+template <int kMode>
+__device__ __forceinline__ KWalk kwalk_begin(const TileInfo& t, const GemmArgs& a) {
+  KWalk w;
+  w.g = kMode == kGroupsK ? t.g - a.E : t.g;
+  w.left = kMode == kGroupsK ? 0 : t.nk;
+  w.kk = t.kt0;
+  return w;
+}
+
+// The step to load now; call only while steps of the tile remain.
+template <int kMode>
+__device__ __forceinline__ int64_t kwalk_step(KWalk& w, const GemmArgs& a, const int32_t* ends,
+                                              const int32_t* pstart) {
+  if (kMode == kGroupsK) {
+    while (w.left == 0) {
+      w.g += a.E;
+      const int64_t start = w.g ? ends[w.g - 1] : 0;
+      w.left = int(ceil_div(ends[w.g] - start, kBK));
+      w.kk = pstart[w.g] / kBK;
+    }
+  }
+  const int64_t kk = w.kk;
+  ++w.kk;
+  --w.left;
+  return kk;
 }
 
 // ------------------------------------------------------------ epilogue ---
@@ -173,7 +215,7 @@ __device__ __forceinline__ TileInfo decode_tile(int64_t tile, const GemmArgs& a,
 // bytes -- whole sectors instead of half-filled ones.
 __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot, __nv_bfloat16* dst,
                                               uint32_t leader_ovl, uint32_t leader_free, uint8_t* stage_buf,
-                                              int lane) {
+                                              int lane, int64_t cols_valid) {
   const uint32_t t_acc = lane_base + (slot ? kAccSlot1 : 0u);
   uint32_t rowv[kBN / 2];
   auto drain = [&](int chunk) {
@@ -210,6 +252,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot,
   for (int i = 0; i < 4; ++i) rows[i] = __shfl_sync(0xFFFFFFFFu, mine, i * 8 + (lane >> 2));
 #pragma unroll
   for (int chunk = 0; chunk < kBN / 32; ++chunk) {
+    if (chunk * 32 >= cols_valid) break;     // columns past the output (N or K not a multiple of 256)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t phys = uint32_t(k) ^ ((uint32_t(lane) >> 1) & 3u);
@@ -232,11 +275,12 @@ __device__ __forceinline__ void epilogue_tile(uint32_t lane_base, uint32_t slot,
   }
 }
 
-// Exact zeros for one 256-column output row (an empty K group), if stored.
-__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
+// Exact zeros for one output row of a 256-column tile (an empty K group), if stored.
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int64_t cols_valid) {
   if (dst) {
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (int c = 0; c < kBN; c += 8) *reinterpret_cast<uint4*>(dst + c) = z;
+    const int n = cols_valid < kBN ? int(cols_valid) : kBN;
+    for (int c = 0; c < n; c += 8) *reinterpret_cast<uint4*>(dst + c) = z;
   }
 }
 
@@ -342,8 +386,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     }
     if (lane == 0) {
       int64_t total;
-      if (kMode != kGroupsK) total = bad ? 0 : int64_t(tstart[G]) * (args.N / kBN);
-      else total = bad ? 0 : int64_t(G) * (args.N / kPairM) * (args.K / kBN);
+      if (kMode != kGroupsK) total = bad ? 0 : int64_t(tstart[G]) * ceil_div(args.N, kBN);
+      else total = bad ? 0 : int64_t(args.offs ? args.E : 1) * ceil_div(args.N, kPairM) * ceil_div(args.K, kBN);
       if (bad && rank == 0) flag_error(kErrOffsets);
       info[0] = total;
     }
@@ -355,7 +399,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const int64_t total_tiles = info[0];
   GemmArgs a = args;
-  if (a.offs == nullptr) a.G = 1;
+  if (a.offs == nullptr) a.G = a.E = 1;
 
   // ----------------------------------------------------------- producer ---
   if (warp == 4) {
@@ -371,9 +415,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         const int32_t b_row = int32_t(t.b_row0 + (kBN / 2) * rank);
         const int64_t sfa_chunk0 = ((t.m0 + kCtaM * rank) / kCtaM) * a.a_sc_tiles;
         bool ok = true;
+        KWalk walk = kwalk_begin<kMode>(t, a);
         for (int kt = 0; kt < t.nk; ++kt) {
           if (!mbar_wait_warp(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
-          const int kk = t.kt0 + kt;
+          const int kk = int(kwalk_step<kMode>(walk, a, ends, pstart));
           const uint32_t fb = full_bar(stage);
           if (elect_one()) {
             if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
@@ -488,21 +533,24 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       const TileInfo t = decode_tile<kMode>(tile, a, ends, pstart, tstart);
       const int64_t row = t.m0 + kCtaM * rank + r;
       __nv_bfloat16* dst = nullptr;
+      int64_t cols_valid;           // output columns of this tile (fewer than 256 at a ragged edge)
       if (kMode != kGroupsK) {
         const int64_t start = t.g ? ends[t.g - 1] : 0;
         const int64_t local = row - pstart[t.g];
         if (local < ends[t.g] - start) dst = a.out + (start + local) * a.N + t.n0;
+        cols_valid = a.N - t.n0;
       } else {
-        dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
+        if (row < a.N) dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
+        cols_valid = a.K - t.n0;
       }
       if (t.nk == 0) {
-        store_zero_row(dst);
+        store_zero_row(dst, cols_valid);
         continue;
       }
       const uint32_t slot = tiles_done & 1u, use = tiles_done >> 1;
       if (!mbar_wait(acc_full0 + 8u * slot, use & 1u, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile(lane_base, slot, dst, leader_ovl, leader_free0 + 8u * slot, stage_buf, lane);
+      epilogue_tile(lane_base, slot, dst, leader_ovl, leader_free0 + 8u * slot, stage_buf, lane, cols_valid);
       ++tiles_done;
     }
   }

@@ -81,7 +81,7 @@ __device__ __forceinline__ HTile decode_tile_bf16(int64_t tile, const HGemmArgs&
                                                   const int32_t* tstart) {
   HTile t;
   if (kMode == kGroupsM) {
-    const int64_t nt = a.N / kBN;
+    const int64_t nt = ceil_div(a.N, kBN);
     const int64_t mt = tile / nt;
     t.n0 = (tile % nt) * kBN;
     int lo = 0, hi = a.G;   // largest g with tstart[g] <= mt
@@ -96,7 +96,7 @@ __device__ __forceinline__ HTile decode_tile_bf16(int64_t tile, const HGemmArgs&
     t.tail = kHBK;
     t.tok0 = 0;
   } else {
-    const int64_t nt = a.K / kBN, mt = a.N / kPairM;
+    const int64_t nt = ceil_div(a.K, kBN), mt = ceil_div(a.N, kPairM);
     const int64_t per_g = nt * mt;
     t.g = int(tile / per_g);
     const int64_t rem = tile % per_g;
@@ -214,8 +214,8 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
     if (lane == 0) {
       int64_t total;
-      if (kMode == kGroupsM) total = bad ? 0 : int64_t(tstart[G]) * (args.N / kBN);
-      else total = bad ? 0 : int64_t(G) * (args.N / kPairM) * (args.K / kBN);
+      if (kMode == kGroupsM) total = bad ? 0 : int64_t(tstart[G]) * ceil_div(args.N, kBN);
+      else total = bad ? 0 : int64_t(G) * ceil_div(args.N, kPairM) * ceil_div(args.K, kBN);
       if (bad && rank == 0) flag_error(kErrOffsets);
       info[0] = total;
     }
@@ -372,19 +372,22 @@ bf16_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
       const HTile t = decode_tile_bf16<kMode>(tile, a, ends, tstart);
       const int64_t row = t.m0 + kCtaM * rank + r;
       __nv_bfloat16* dst = nullptr;
+      int64_t cols_valid;           // output columns of this tile (fewer than 256 at a ragged edge)
       if (kMode == kGroupsM) {
         if (row < ends[t.g]) dst = a.out + row * a.N + t.n0;
+        cols_valid = a.N - t.n0;
       } else {
-        dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
+        if (row < a.N) dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
+        cols_valid = a.K - t.n0;
       }
       if (t.nk == 0) {
-        store_zero_row(dst);
+        store_zero_row(dst, cols_valid);
         continue;
       }
       const uint32_t slot = tiles_done & 1u, use = tiles_done >> 1;
       if (!mbar_wait(acc_full0 + 8u * slot, use & 1u, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile(lane_base, slot, dst, leader_ovl, leader_free0 + 8u * slot, stage_buf, lane);
+      epilogue_tile(lane_base, slot, dst, leader_ovl, leader_free0 + 8u * slot, stage_buf, lane, cols_valid);
       ++tiles_done;
     }
   }

@@ -180,8 +180,8 @@ def test_bf16_gemm_invalid_offsets_and_host_errors(mx):
         mx.mx_device_error()
     assert e.value.status == 6
     assert bool((out == 3.0).all())
-    with pytest.raises(mx.MXError) as e:          # N not a multiple of 256
-        mx.mx_grouped_mm_bf16(a, b, None, 1, mx.MX_GROUPS_M, out, 256, 128, 64)
+    with pytest.raises(mx.MXError) as e:          # N not a multiple of 32
+        mx.mx_grouped_mm_bf16(a, b, None, 1, mx.MX_GROUPS_M, out, 256, 100, 64)
     assert e.value.status == 3
     with pytest.raises(mx.MXError) as e:          # K not a multiple of 8
         mx.mx_grouped_mm_bf16(a, b, None, 1, mx.MX_GROUPS_M, out, 256, 256, 60)
