@@ -178,7 +178,6 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  *   b_q [G, N, K],   b_s G concatenated blocked(N, K/32) buffers
  *   out bf16 [M, N]; rows of the padded layout that are padding are not read
  *       into the output (the unpad is fused into the store).
- *   N a multiple of 256, K a multiple of 128.
  * mode MX_GROUPS_M_KN (dgrad straight from the forward's weight codes): as
  *   MX_GROUPS_M with B codes stored [G, K, N] (N contiguous; read by the MMA
  *   as an MN-major operand, so no transposed copy is needed) and b_s G
@@ -192,7 +191,12 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  *       L = m_cap (padded token columns from mx_cast_dim1_grouped) or M when
  *       offs == NULL (dense, G = 1, M a multiple of 32)
  *   out bf16 [G, N, K]; an empty group gives exact zeros.
- *   N and K multiples of 256.
+ * Sizes: N and K multiples of 32 in every mode, each below 2^31. Sizes that
+ * are not multiples of the 256x256 output tile or of the 128-deep K step
+ * take the pad path of the unaligned geometry (torchtitan PR #5334, review
+ * thread: the 576-wide output gradient): operand tiles past the tensor are
+ * read as zero codes, whose blocked scale bytes are 0x00, so they add
+ * nothing; output rows and columns past the tensor are never written.
  * offs: device int32 [G] cumulative ends (see the pad path above) or NULL.
  * Invalid offsets set the device flag and leave the output unwritten. */
 #define MX_GROUPS_M 0
@@ -201,6 +205,20 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
 MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
                                const int32_t* offs, int32_t G, int32_t mode, void* out,
                                int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
+
+/* The grouped GEMM whose G groups cycle over E experts: group g uses expert
+ * g % E. This is the layout in which an expert-parallel all-to-all delivers
+ * tokens to the rank that holds E experts -- source rank major, expert minor
+ * ("MXFP8 all-to-all", prime-rl PR #3388, Overview, enable_a2a; ao PR #4705,
+ * the expert-parallel pipeline benchmark). E divides G; E == G is exactly
+ * mx_grouped_mm. Operands and sizes as mx_grouped_mm, except:
+ *   MX_GROUPS_M / MX_GROUPS_M_KN: b_q and b_s hold E experts (not G);
+ *   MX_GROUPS_K: out bf16 [E, N, K], out[e] sums the token groups
+ *     e, e + E, e + 2E, ... (an expert with only empty groups gives zeros).
+ * Without offsets G = E = 1. */
+MX_API mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                                       const int32_t* offs, int32_t G, int32_t E, int32_t mode, void* out,
+                                       int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
 
 /* ------------------------------------------- backward-override arms -----
  * ao "[moe training] Add backward_override to the MXFP8 grouped GEMM", Design
@@ -218,10 +236,10 @@ MX_API mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q
  * operand is copied or transposed.
  * mode MX_GROUPS_M (dgrad):  out[rows of g, :] = a[rows of g, :] @ b[g]
  *   a bf16 [M, K], b bf16 [G, K, N], out bf16 [M, N].
- *   N a multiple of 256, K a positive multiple of 8.
+ *   N a multiple of 32, K a positive multiple of 8.
  * mode MX_GROUPS_K (wgrad):  out[g] = a[rows of g, :]^T @ b[rows of g, :]
  *   a bf16 [M, N], b bf16 [M, K], out bf16 [G, N, K]; an empty group gives
- *   exact zeros. N and K multiples of 256.
+ *   exact zeros. N and K multiples of 32.
  * M, N, K < 2^31. Invalid offsets set the device flag and leave the output
  * unwritten. */
 MX_API mx_status mx_grouped_mm_bf16(const void* a, const void* b, const int32_t* offs, int32_t G,
@@ -256,7 +274,8 @@ MX_API mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void
  *   backward dx [M, K] = dy [M, N] w           dy cast 1x32 along N
  *            dw [N, K] = dy^T x                dy and x cast 32x1 along M
  * dy is cast once by the fused rowwise+columnwise cast. All tensors bf16,
- * row-major. M a multiple of 32; N and K multiples of 256.
+ * row-major. M, N and K multiples of 32 (N or K off the 256-wide tile, such
+ * as 576, take the GEMM's pad path).
  * ws: caller-owned device workspace of at least mx_linear_ws_bytes(M, N, K)
  * bytes (holds the quantized activations and gradients and, without a
  * cache, the quantized weight); it must stay untouched until the call's

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include <cudaTypedefs.h>
@@ -119,36 +120,77 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps are kept in a small table keyed by every encode
+// argument, so that launches over the same buffers (every step of a
+// training loop) skip the encode. A map is a pure function of its
+// arguments, so a hit is exactly what a fresh encode would return.
+struct MapKey {
+  const void* base;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  int dtype, rank, swizzle;
+};
+
+constexpr int kMapCacheSize = 64;
+struct MapCacheEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+std::mutex g_map_mu;
+MapCacheEntry g_map_cache[kMapCacheSize];
+int g_map_next = 0;
+
+mx_status encode_tiled(CUtensorMap* m, CUtensorMapDataType dtype, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  for (int i = 0; i < rank; ++i) key.dims[i] = dims[i], key.box[i] = box[i];
+  for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides[i];
+  key.dtype = int(dtype);
+  key.rank = rank;
+  key.swizzle = int(swizzle);
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (auto& e : g_map_cache)
+      if (e.used && memcmp(&e.key, &key, sizeof(key)) == 0) {
+        *m = e.map;
+        return MX_OK;
+      }
+  }
+  auto fn = encode_fn();
+  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], estr[3] = {1u, 1u, 1u};
+  for (int i = 0; i < rank; ++i) d[i] = dims[i], bx[i] = box[i];
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  CUresult r = fn(m, dtype, cuuint32_t(rank), const_cast<void*>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapCacheEntry& e = g_map_cache[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCacheSize;
+  e.key = key;
+  e.map = *m;
+  e.used = true;
+  return MX_OK;
+}
+
 // 2D uint8 tensor map over a row-major [outer, inner] byte matrix, box
 // {128, box_outer}, 128-byte swizzle, zero fill outside the tensor.
 mx_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
-  auto fn = encode_fn();
-  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {128u, box_outer};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
-  return MX_OK;
+  const uint64_t dims[2] = {inner, outer}, strides[1] = {inner};
+  const uint32_t box[2] = {128u, box_outer};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // 2D map over a blocked scale buffer viewed as [chunks, 128] 32-bit words:
 // one box = one 512-byte 128x4 scale tile; rows past the buffer read as zero.
 mx_status make_scale_map(CUtensorMap* m, const void* base, uint64_t chunks) {
-  auto fn = encode_fn();
-  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[2] = {128u, chunks};
-  cuuint64_t strides[1] = {512u};
-  cuuint32_t box[2] = {128u, 1u};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
-  return MX_OK;
+  const uint64_t dims[2] = {128u, chunks}, strides[1] = {512u};
+  const uint32_t box[2] = {128u, 1u};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 template <int kMode>
@@ -158,8 +200,6 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   MX_REQUIRE(e == cudaSuccess && dev < 64, MX_ERR_CUDA, "cudaGetDevice failed");
-  e = cudaFuncSetAttribute(mx_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
-  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
@@ -172,7 +212,9 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs[dev] == 0) {
+  if (max_pairs[dev] == 0) {       // once per device: shared-memory attribute and the resident pairs
+    e = cudaFuncSetAttribute(mx_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
     cfg.gridDim = dim3(2, 1, 1);
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<kMode>, &cfg);
@@ -192,18 +234,11 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
 // box_outer rows (x 1 matrix), 128-byte swizzle, zero fill outside.
 mx_status make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t depth,
                         uint32_t box_outer) {
-  auto fn = encode_fn();
-  MX_REQUIRE(fn != nullptr, MX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint32_t rank = depth > 0 ? 3u : 2u;
-  cuuint64_t dims[3] = {inner, outer, depth};
-  cuuint64_t strides[2] = {inner * 2, inner * outer * 2};
-  cuuint32_t box[3] = {64u, box_outer, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MX_REQUIRE(r == CUDA_SUCCESS, MX_ERR_CUDA, "cuTensorMapEncodeTiled (bf16) failed (%d)", int(r));
-  return MX_OK;
+  const int rank = depth > 0 ? 3 : 2;
+  const uint64_t dims[3] = {inner, outer, depth}, strides[2] = {inner * 2, inner * outer * 2};
+  const uint32_t box[3] = {64u, box_outer, 1u};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int kMode>
@@ -213,8 +248,6 @@ mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const H
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   MX_REQUIRE(e == cudaSuccess && dev < 64, MX_ERR_CUDA, "cudaGetDevice failed");
-  e = cudaFuncSetAttribute(bf16_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kHGemmSmem));
-  MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm smem attribute: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
@@ -227,7 +260,9 @@ mx_status launch_bf16_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const H
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs[dev] == 0) {
+  if (max_pairs[dev] == 0) {       // once per device: shared-memory attribute and the resident pairs
+    e = cudaFuncSetAttribute(bf16_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kHGemmSmem));
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "bf16 gemm smem attribute: %s", cudaGetErrorString(e));
     cfg.gridDim = dim3(2, 1, 1);
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, bf16_gemm_kernel<kMode>, &cfg);
@@ -394,19 +429,20 @@ mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K, const int32_t*
                                         static_cast<cudaStream_t>(stream));
 }
 
-mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
-                        const int32_t* offs, int32_t G, int32_t mode, void* out, int64_t M, int64_t N,
-                        int64_t K, int64_t m_cap, void* stream) {
+mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                                const int32_t* offs, int32_t G, int32_t E, int32_t mode, void* out, int64_t M,
+                                int64_t N, int64_t K, int64_t m_cap, void* stream) {
   MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K || mode == MX_GROUPS_M_KN, MX_ERR_ARG, "unknown mode %d",
              mode);
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   if (offs != nullptr) {
     MX_REQUIRE(G >= 1 && G <= kMaxGroups, MX_ERR_ARG, "G = %d outside [1, %d]", G, kMaxGroups);
+    MX_REQUIRE(E >= 1 && E <= G && G % E == 0, MX_ERR_ARG, "E = %d must divide G = %d", E, G);
     MX_REQUIRE(m_cap >= M && m_cap % 128 == 0 && m_cap < (1ll << 31), MX_ERR_ARG,
                "m_cap = %lld must be a multiple of 128, >= M and < 2^31", (long long)m_cap);
     MX_REQUIRE((reinterpret_cast<uintptr_t>(offs) & 3u) == 0, MX_ERR_ALIGN, "offsets not 4-byte aligned");
   } else {
-    MX_REQUIRE(G == 1, MX_ERR_ARG, "without offsets G must be 1 (dense)");
+    MX_REQUIRE(G == 1 && E == 1, MX_ERR_ARG, "without offsets G and E must be 1 (dense)");
     MX_REQUIRE(M < (1ll << 31), MX_ERR_ARG, "M too large");
   }
   const void* ptrs[5] = {a_q, a_s, b_q, b_s, out};
@@ -417,39 +453,44 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
   ga.offs = offs;
   ga.out = static_cast<__nv_bfloat16*>(out);
   ga.G = G;
+  ga.E = E;
   ga.M = M;
   ga.N = N;
   ga.K = K;
   CUtensorMap map_a, map_b, map_sa, map_sb;
+  // Every size is a multiple of 32 (the block of a scale). A size that is
+  // not a multiple of the tile (256 output columns, 128-deep K steps) is the
+  // pad path: TMA fills operand tiles past the tensor with zero codes (pad
+  // scale bytes are 0x00), so past-the-end K adds nothing; output rows and
+  // 32-column chunks past the tensor are never stored.
+  MX_REQUIRE(N % kBlock == 0 && K % kBlock == 0, MX_ERR_UNSUPPORTED,
+             "N = %lld and K = %lld must be multiples of 32", (long long)N, (long long)K);
+  MX_REQUIRE(N < (1ll << 31) && K < (1ll << 31), MX_ERR_ARG, "N or K is 2^31 or more");
   if (mode != MX_GROUPS_K) {
-    MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
-    MX_REQUIRE(K % kBK == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 128", (long long)K);
     const int64_t rows_a = offs ? m_cap : M;
     ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
     if (rows_a == 0 || M == 0) return MX_OK;
     MX_REQUIRE(a_q && a_s && b_q && b_s && out, MX_ERR_ARG, "null operand");
-    ga.a_sc_tiles = K / kBK;
-    ga.b_sc_tiles = K / kBK;
+    ga.a_sc_tiles = ceil_div(K, kBK);
+    ga.b_sc_tiles = ceil_div(K, kBK);
     ga.b_sc_group_chunks = scale_bytes(N, K / kBlock) / 512;
     MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kCtaM));
     if (mode == MX_GROUPS_M_KN)
-      MX_TRY(make_map(&map_b, b_q, uint64_t(N), uint64_t(G) * uint64_t(K), kBK));
+      MX_TRY(make_map(&map_b, b_q, uint64_t(N), uint64_t(E) * uint64_t(K), kBK));
     else
-      MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(G) * uint64_t(N), kBN / 2));
+      MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(E) * uint64_t(N), kBN / 2));
     MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(rows_a, K / kBlock) / 512)));
-    MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(G) * uint64_t(ga.b_sc_group_chunks)));
-    const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * (N / kBN);
+    MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(E) * uint64_t(ga.b_sc_group_chunks)));
+    const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * ceil_div(N, kBN);
     if (mode == MX_GROUPS_M_KN) return launch_gemm<kGroupsMKn>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
     return launch_gemm<kGroupsM>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
   }
-  MX_REQUIRE(N % kPairM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
-  MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
   MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
   const int64_t len = offs ? m_cap : M;
   MX_REQUIRE(offs || M % kBlock == 0, MX_ERR_UNSUPPORTED, "dense K-groups needs M %% 32 == 0");
   ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
   if (len == 0) {
-    cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
+    cudaError_t e = cudaMemsetAsync(out, 0, size_t(E) * N * K * 2, st);
     MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
     return MX_OK;
   }
@@ -461,8 +502,14 @@ mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const
   MX_TRY(make_map(&map_b, b_q, uint64_t(len), uint64_t(K), kBN / 2));
   MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(N, ceil_div(len, kBlock)) / 512)));
   MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(scale_bytes(K, ceil_div(len, kBlock)) / 512)));
-  const int64_t pair_tiles_ub = int64_t(G) * (N / kPairM) * (K / kBN);
+  const int64_t pair_tiles_ub = int64_t(E) * ceil_div(N, kPairM) * ceil_div(K, kBN);
   return launch_gemm<kGroupsK>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
+}
+
+mx_status mx_grouped_mm(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                        const int32_t* offs, int32_t G, int32_t mode, void* out, int64_t M, int64_t N,
+                        int64_t K, int64_t m_cap, void* stream) {
+  return mx_grouped_mm_experts(a_q, a_s, b_q, b_s, offs, G, G, mode, out, M, N, K, m_cap, stream);
 }
 
 mx_wcache* mx_wcache_create(void) { return new (std::nothrow) mx_wcache(); }
@@ -519,7 +566,7 @@ namespace {
 mx_status check_linear(int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes) {
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
-  MX_REQUIRE(N % kBN == 0 && K % kBN == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 256");
+  MX_REQUIRE(N % kBlock == 0 && K % kBlock == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 32");
   MX_REQUIRE(ws_bytes >= mx_linear_ws_bytes(M, N, K), MX_ERR_ARG, "workspace too small (%zu < %zu bytes)",
              ws_bytes, mx_linear_ws_bytes(M, N, K));
   MX_REQUIRE(ws != nullptr && aligned16(ws), MX_ERR_ALIGN, "workspace null or not 16-byte aligned");
@@ -666,7 +713,7 @@ extern "C" mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t
                                            void* stream) {
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
-  MX_REQUIRE(N % kBN == 0 && K % kBN == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 256");
+  MX_REQUIRE(N % kBlock == 0 && K % kBlock == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 32");
   // Bound each factor before any product, so that no size can overflow the
   // byte count below and slip past the scratch bound.
   constexpr int64_t kScratch = int64_t(MX_LINEAR_NOALLOC_SCRATCH_BYTES);
@@ -751,17 +798,17 @@ extern "C" mx_status mx_grouped_mm_bf16(const void* a, const void* b, const int3
   ha.K = K;
   CUtensorMap map_a, map_b;
   if (mode == MX_GROUPS_M) {
-    MX_REQUIRE(N % kBN == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
+    MX_REQUIRE(N % 32 == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 32", (long long)N);
     MX_REQUIRE(K % 8 == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 8 (16-byte rows)", (long long)K);
     if (M == 0) return MX_OK;
     MX_REQUIRE(a && b && out, MX_ERR_ARG, "null operand");
     MX_TRY(make_map_bf16(&map_a, a, uint64_t(K), uint64_t(M), 0, kCtaM));
     MX_TRY(make_map_bf16(&map_b, b, uint64_t(N), uint64_t(K), uint64_t(G), 64));
-    const int64_t pair_tiles_ub = (ceil_div(M, kPairM) + (offs ? G : 0)) * (N / kBN);
+    const int64_t pair_tiles_ub = (ceil_div(M, kPairM) + (offs ? G : 0)) * ceil_div(N, kBN);
     return launch_bf16_gemm<kGroupsM>(map_a, map_b, ha, pair_tiles_ub, st);
   }
-  MX_REQUIRE(N % kPairM == 0, MX_ERR_UNSUPPORTED, "N = %lld is not a multiple of 256", (long long)N);
-  MX_REQUIRE(K % kBN == 0, MX_ERR_UNSUPPORTED, "K = %lld is not a multiple of 256", (long long)K);
+  MX_REQUIRE(N % 32 == 0 && K % 32 == 0, MX_ERR_UNSUPPORTED, "N = %lld and K = %lld must be multiples of 32",
+             (long long)N, (long long)K);
   MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
   if (M == 0) {
     cudaError_t e = cudaMemsetAsync(out, 0, size_t(G) * N * K * 2, st);
@@ -771,7 +818,7 @@ extern "C" mx_status mx_grouped_mm_bf16(const void* a, const void* b, const int3
   MX_REQUIRE(a && b, MX_ERR_ARG, "null operand");
   MX_TRY(make_map_bf16(&map_a, a, uint64_t(N), uint64_t(M), 0, 64));
   MX_TRY(make_map_bf16(&map_b, b, uint64_t(K), uint64_t(M), 0, 64));
-  const int64_t pair_tiles_ub = int64_t(G) * (N / kPairM) * (K / kBN);
+  const int64_t pair_tiles_ub = int64_t(G) * ceil_div(N, kPairM) * ceil_div(K, kBN);
   return launch_bf16_gemm<kGroupsK>(map_a, map_b, ha, pair_tiles_ub, st);
 }
 

@@ -35,6 +35,8 @@ _SIGNATURES = {
     "mx_cast_dim1_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
+    "mx_grouped_mm_experts": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
+                                             _i64, _vp]),
     "mx_wcache_create": (_vp, []),
     "mx_wcache_evict": (None, [_vp, _vp]),
     "mx_wcache_clear": (None, [_vp]),
@@ -92,9 +94,17 @@ def exported_names():
     return list(_SIGNATURES)
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_raw_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    """cudaStream_t of `stream`, or of the current stream (read without building a Stream object)."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    if _raw_stream is not None and _raw_device is not None:
+        return ctypes.c_void_p(_raw_stream(_raw_device()))
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
 def _p(t):
@@ -171,6 +181,11 @@ def mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st, stream=None):
 
 def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream=None):
     _call("mx_grouped_mm", _p(a_q), _p(a_s), _p(b_q), _p(b_s), _p(offs), G, mode, _p(out), M, N, K,
+          m_cap, _stream(stream))
+
+
+def mx_grouped_mm_experts(a_q, a_s, b_q, b_s, offs, G, E, mode, out, M, N, K, m_cap, stream=None):
+    _call("mx_grouped_mm_experts", _p(a_q), _p(a_s), _p(b_q), _p(b_s), _p(offs), G, E, mode, _p(out), M, N, K,
           m_cap, _stream(stream))
 
 

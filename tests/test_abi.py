@@ -83,10 +83,14 @@ def test_host_argument_checks_return_before_any_launch():
     assert L.mx_cast_dim1(ok16, 48, 64, ok16, ok16, None) == 3          # R not a multiple of 32
     assert L.mx_cast_ex(ok16, 64, 64, 3, 7, ok16, ok16, ok16, ok16, None) == 1   # unknown rule
     assert L.mx_grouped_mm(ok16, ok16, ok16, ok16, None, 1, 5, ok16, 128, 256, 128, 0, None) == 1  # mode
-    assert L.mx_grouped_mm(ok16, ok16, ok16, ok16, None, 1, 0, ok16, 128, 200, 128, 0, None) == 3  # N % 256
+    assert L.mx_grouped_mm(ok16, ok16, ok16, ok16, None, 1, 0, ok16, 128, 200, 128, 0, None) == 3  # N % 32
     assert L.mx_grouped_mm_bf16(ok16, ok16, None, 1, 0, ok16, 128, 256, 60, None) == 3      # K % 8
     assert L.mx_grouped_mm_bf16(ok16, ok16, ok16, 0, 0, ok16, 128, 256, 64, None) == 1      # G = 0
     assert L.mx_dequant_dim0(ok16, ok16, 1, 4, 40, ok16, None) == 3     # C not a multiple of 32
+    assert L.mx_grouped_mm_experts(ok16, ok16, ok16, ok16, ok16, 6, 4, 0, ok16, 128, 256, 128, 1024,
+                                   None) == 1                           # E does not divide G
+    assert L.mx_grouped_mm_experts(ok16, ok16, ok16, ok16, None, 1, 2, 0, ok16, 128, 256, 128, 0,
+                                   None) == 1                           # dense needs E = 1
     assert L.mx_scales_unswizzle(odd, 4, 4, ok16, None) == 2
     msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
     assert b"not a multiple of 32" in msg
