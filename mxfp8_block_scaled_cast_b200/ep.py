@@ -1,0 +1,246 @@
+"""Expert-parallel MoE grouped GEMM with the MXFP8 all-to-all.
+
+With expert parallelism each of W ranks holds E of the W*E experts, and an
+all-to-all moves every token to the rank of its expert and its output back.
+The "MXFP8 all-to-all" (prime-rl PR #3388, Overview: MXFP8Config.enable_a2a,
+with notes on when it helps and when it hurts; ao PR #4705, the two-GPU
+expert-parallel pipeline benchmark) carries the dispatched tokens as MXFP8 --
+one E4M3 byte per element plus one E8M0 byte per 32 -- instead of two bf16
+bytes.
+
+Layout (this implementation's reading; the pages describe no layout):
+  * The sender casts its tokens rowwise (1x32 along K) straight into the
+    padded group layout of the pad path with one group per global expert,
+    ordered by destination rank. Each destination's groups are then one
+    contiguous run of whole 128-row tiles: its codes are a row range of the
+    code buffer and its scales a range of whole 512-byte blocked scale tiles,
+    so each piece is one slice of the all-to-all.
+  * The receiver's buffer is therefore the padded grouped operand of groups
+    (source rank, local expert), source major -- exactly what the grouped
+    GEMM reads, with group g using local expert g % E
+    (mx_grouped_mm_experts). No unpack or rearrangement pass runs. The
+    rowwise cast is per row, so the received codes are bitwise the codes the
+    receiver would compute from the bf16 tokens.
+  * Outputs return in bf16 by the reverse all-to-all (the combine), in the
+    sender's token order.
+  * Backward: dY goes to the experts in bf16 (the combine's reverse), the
+    receiver casts it (rowwise for dX, columnwise per group for dW), and the
+    wgrad's columnwise cast of the activations reads the received codes
+    dequantized to bf16 -- the receiver never sees the bf16 activations;
+    that double rounding is what the MXFP8 dispatch trades for bandwidth.
+    dW of expert e sums its groups from every source rank in one GEMM.
+
+Everything that moves data is torch.distributed.all_to_all_single (NCCL over
+NVLink on GPUs); every arithmetic step is a libmx kernel.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import mx
+
+BLOCK_ROWS = 128          # rows of a blocked scale tile: the pad path's group alignment
+
+
+def _pad(n):
+    return -(-int(n) // BLOCK_ROWS) * BLOCK_ROWS
+
+
+def scale_band_bytes(K: int) -> int:
+    """Bytes of the blocked scales of one 128-row band of a [rows, K] rowwise cast."""
+    return mx_scale_bytes_host(BLOCK_ROWS, K // 32)
+
+
+def mx_scale_bytes_host(rows: int, cols: int) -> int:
+    """ceil(rows/128)*128 * ceil(cols/4)*4: the blocked layout's size (host arithmetic)."""
+    if rows <= 0 or cols <= 0:
+        return 0
+    return _pad(rows) * (-(-int(cols) // 4) * 4)
+
+
+@dataclass
+class ExchangePlan:
+    """Sizes of one rank's all-to-alls, from the token counts.
+
+    send_counts[j]: tokens this rank sends to global expert j (W*E entries;
+    rank r holds experts r*E .. r*E + E - 1); recv_counts[s, e]: tokens rank s
+    sends to this rank's local expert e."""
+    W: int
+    E: int
+    send_counts: np.ndarray
+    recv_counts: np.ndarray
+
+    def __post_init__(self):
+        self.send_counts = np.asarray(self.send_counts, dtype=np.int64).reshape(-1)
+        self.recv_counts = np.asarray(self.recv_counts, dtype=np.int64).reshape(self.W, self.E)
+        assert self.send_counts.size == self.W * self.E
+        assert (self.send_counts >= 0).all() and (self.recv_counts >= 0).all()
+        pad = np.array([_pad(c) for c in self.send_counts], dtype=np.int64).reshape(self.W, self.E)
+        rpad = np.array([_pad(c) for c in self.recv_counts.reshape(-1)], dtype=np.int64).reshape(self.W, self.E)
+        self.M = int(self.send_counts.sum())                          # tokens sent
+        self.m_cap_send = int(pad.sum())                              # padded rows of the send buffer
+        self.send_rows = pad.sum(axis=1)                              # padded rows to each rank
+        self.send_tokens = self.send_counts.reshape(self.W, self.E).sum(axis=1)
+        self.M_recv = int(self.recv_counts.sum())                     # tokens received
+        self.m_cap_recv = int(rpad.sum())
+        self.recv_rows = rpad.sum(axis=1)                             # padded rows from each rank
+        self.recv_tokens = self.recv_counts.sum(axis=1)
+
+    def offs_send(self) -> np.ndarray:
+        """Cumulative group ends of the send layout (one group per global expert)."""
+        return np.cumsum(self.send_counts).astype(np.int32)
+
+    def offs_recv(self) -> np.ndarray:
+        """Cumulative group ends of the receive layout: groups (source rank, local expert)."""
+        return np.cumsum(self.recv_counts.reshape(-1)).astype(np.int32)
+
+    @property
+    def G_recv(self) -> int:
+        return self.W * self.E
+
+
+def exchange_counts(send_counts, W: int, E: int, a2a, device) -> np.ndarray:
+    """recv_counts [W, E] from every rank's send_counts (one small all-to-all)."""
+    send = torch.as_tensor(np.asarray(send_counts, dtype=np.int64), device=device)
+    recv = torch.empty(W * E, dtype=torch.int64, device=device)
+    a2a(recv, send, [E] * W, [E] * W)
+    return recv.cpu().numpy().reshape(W, E)
+
+
+def _splits(rows):
+    return [int(r) for r in rows]
+
+
+def dist_all_to_all(group=None):
+    """all_to_all_single over `group` (output, input, output splits, input splits), in rows."""
+    import torch.distributed as dist
+
+    def a2a(out, inp, out_splits, in_splits):
+        dist.all_to_all_single(out, inp, out_splits, in_splits, group=group)
+    return a2a
+
+
+# ----------------------------------------------------------- the pieces --
+def pack_mxfp8(x, plan: ExchangePlan):
+    """Rowwise cast of x [M, K] (tokens ordered by global expert) into the send
+    layout: codes [m_cap_send, K] and blocked scales viewed as [bands, band bytes]."""
+    M, K = x.shape
+    offs = torch.as_tensor(plan.offs_send(), device=x.device)
+    q = torch.empty(plan.m_cap_send, K, dtype=torch.uint8, device=x.device)
+    s = torch.empty(mx.mx_scale_bytes(plan.m_cap_send, K // 32), dtype=torch.uint8, device=x.device)
+    if plan.m_cap_send:
+        mx.mx_cast_dim0_grouped(x, offs, plan.m_cap_send, q, s)
+    return q, s.view(plan.m_cap_send // BLOCK_ROWS, scale_band_bytes(K))
+
+
+def dispatch_mxfp8(q, s, plan: ExchangePlan, a2a):
+    """The MXFP8 dispatch: codes by padded rows, scales by whole 128-row bands."""
+    K = q.shape[1]
+    rq = torch.empty(plan.m_cap_recv, K, dtype=torch.uint8, device=q.device)
+    rs = torch.empty(plan.m_cap_recv // BLOCK_ROWS, s.shape[1], dtype=torch.uint8, device=q.device)
+    a2a(rq, q, _splits(plan.recv_rows), _splits(plan.send_rows))
+    a2a(rs, s, _splits(plan.recv_rows // BLOCK_ROWS), _splits(plan.send_rows // BLOCK_ROWS))
+    return rq, rs
+
+
+def expert_forward(rq, rs, wq, wsf, plan: ExchangePlan):
+    """y_recv [M_recv, N] bf16 = each received group times its local expert (g % E)."""
+    N, K = wq.shape[1], wq.shape[2]
+    y = torch.empty(plan.M_recv, N, dtype=torch.bfloat16, device=rq.device)
+    if plan.M_recv:
+        offs = torch.as_tensor(plan.offs_recv(), device=rq.device)
+        mx.mx_grouped_mm_experts(rq, rs, wq, wsf, offs, plan.G_recv, plan.E, mx.MX_GROUPS_M, y, plan.M_recv, N, K,
+                                 plan.m_cap_recv)
+    return y
+
+
+def combine(y_recv, plan: ExchangePlan, a2a):
+    """Outputs back to their senders (bf16), in the sender's token order."""
+    y = torch.empty(plan.M, y_recv.shape[1], dtype=y_recv.dtype, device=y_recv.device)
+    a2a(y, y_recv, _splits(plan.send_tokens), _splits(plan.recv_tokens))
+    return y
+
+
+def dispatch_bf16(t, plan: ExchangePlan, a2a):
+    """A bf16 tensor in the sender's token order to the experts' ranks (dY in backward)."""
+    out = torch.empty(plan.M_recv, t.shape[1], dtype=t.dtype, device=t.device)
+    a2a(out, t, _splits(plan.recv_tokens), _splits(plan.send_tokens))
+    return out
+
+
+def expert_backward(dy_recv, rq, rs, wq, wsd, plan: ExchangePlan):
+    """(dx_recv [M_recv, K], dw [E, N, K]) of the received groups.
+
+    dX = dY W_e (dY cast rowwise along N, W's forward codes read MN-major);
+    dW_e = sum over the groups of expert e of dY_g^T X_g, both cast columnwise
+    per group, X from the received codes dequantized to bf16."""
+    E, N, K = wq.shape
+    dev = dy_recv.device
+    dw = torch.empty(E, N, K, dtype=torch.bfloat16, device=dev)
+    dx = torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
+    if plan.M_recv == 0:
+        dw.zero_()
+        return dx, dw
+    offs = torch.as_tensor(plan.offs_recv(), device=dev)
+    G, cap = plan.G_recv, plan.m_cap_recv
+    dq, ds, dqt, dst = mx.cast_2d_grouped(dy_recv, offs, cap)
+    mx.mx_grouped_mm_experts(dq, ds, wq, wsd, offs, G, E, mx.MX_GROUPS_M_KN, dx, plan.M_recv, K, N, cap)
+    x_deq = torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
+    mx.mx_dequant_dim0_grouped(rq, rs.reshape(-1), offs, plan.M_recv, K, cap, x_deq)
+    xqt, xst = mx.cast_dim1_grouped(x_deq, offs, cap)
+    mx.mx_grouped_mm_experts(dqt, dst, xqt, xst, offs, G, E, mx.MX_GROUPS_K, dw, plan.M_recv, N, K, cap)
+    return dx, dw
+
+
+def return_grad(dx_recv, plan: ExchangePlan, a2a):
+    """dX back to the senders (bf16), in the sender's token order."""
+    return combine(dx_recv, plan, a2a)
+
+
+# ------------------------------------------------------------- the layer --
+class MXFP8ExpertParallelMM:
+    """y[tokens of expert j] = x[tokens of expert j] @ w_j^T with the experts
+    sharded over the ranks of `group` and the dispatch in MXFP8.
+
+    forward(x [M, K] bf16 ordered by global expert, send_counts [W*E] tokens
+    per global expert, w [E, N, K] bf16 local experts) -> y [M, N];
+    backward(dy [M, N]) -> (dx [M, K], dw [E, N, K]). `a2a` defaults to
+    torch.distributed.all_to_all_single over `group`."""
+
+    def __init__(self, group=None, a2a=None):
+        import torch.distributed as dist
+        self.group = group
+        self.W = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.a2a = a2a if a2a is not None else dist_all_to_all(group)
+        self._saved = None
+
+    def forward(self, x, send_counts, w):
+        for name, t in (("x", x), ("w", w)):
+            if t.dtype != torch.bfloat16:
+                raise TypeError(f"MXFP8ExpertParallelMM takes bf16 operands ({name} is {t.dtype})")
+        x, w = x.contiguous(), w.contiguous()
+        E = w.shape[0]
+        if int(np.sum(send_counts)) != x.shape[0]:
+            raise ValueError("send_counts must sum to the number of tokens")
+        recv = exchange_counts(send_counts, self.W, E, self.a2a, x.device)
+        plan = ExchangePlan(self.W, E, send_counts, recv)
+        q, s = pack_mxfp8(x, plan)
+        rq, rs = dispatch_mxfp8(q, s, plan, self.a2a)
+        wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
+        y = combine(expert_forward(rq, rs, wq, wsf, plan), plan, self.a2a)
+        self._saved = (plan, rq, rs, wq, wsd)
+        return y
+
+    def backward(self, dy):
+        if self._saved is None:
+            raise RuntimeError("backward before forward")
+        if dy.dtype != torch.bfloat16:
+            raise TypeError("MXFP8ExpertParallelMM takes a bf16 gradient")
+        plan, rq, rs, wq, wsd = self._saved
+        self._saved = None
+        dy_recv = dispatch_bf16(dy.contiguous(), plan, self.a2a)
+        dx_recv, dw = expert_backward(dy_recv, rq, rs, wq, wsd, plan)
+        return return_grad(dx_recv, plan, self.a2a), dw

@@ -47,6 +47,12 @@ What it computes, and where each step comes from
   high-precision arm's two bf16 grouped GEMMs over unpadded groups, the
   dequantized arm's dequantization of the forward's codes to bf16 (round to
   nearest even), and the grouped dequant that gathers padded rows back.
+* Expert parallelism with the MXFP8 all-to-all ("Cache quantized weights for
+  full AC", prime-rl PR #3388, Overview: enable_a2a; ao PR #4705, the
+  expert-parallel pipeline benchmark): the expert-side forward and backward
+  over received groups (source rank, local expert), group g served by local
+  expert g % E, the wgrad's activations cast columnwise from their
+  dequantized values, dW of an expert summed over its groups.
 
 Where the pages are silent, the readings taken are listed in the repository's
 design notes; each is restated beside the function that depends on it.
@@ -603,3 +609,73 @@ def moe_backward_dequantized(x_bits, w_bits, dy_bits, offs):
     dy = bf16_to_f64(dy_bits)
     return (hp_grouped_mm_m(dy, wd, offs), hp_grouped_mm_m(np.abs(dy), np.abs(wd), offs),
             hp_grouped_mm_k(dy, xd, offs), hp_grouped_mm_k(np.abs(dy), np.abs(xd), offs))
+
+
+# --------------------------------------------------------------------------
+# Expert parallelism with the MXFP8 all-to-all (prime-rl PR #3388, Overview:
+# MXFP8Config.enable_a2a; ao PR #4705, the expert-parallel pipeline
+# benchmark). The rank that holds E experts receives the tokens of every
+# source rank as groups (source, local expert), source major, so group g is
+# served by local expert g % E. Reading: the dispatch carries the rowwise
+# (1x32) cast of the tokens, so the forward and dgrad operands are those of
+# the plain grouped GEMM; the wgrad casts the received activations
+# columnwise from their dequantized (bf16) values, since the bf16 tokens
+# never reach the expert's rank; dW of expert e sums its groups.
+# --------------------------------------------------------------------------
+def ep_expert_forward(x_bits, w_bits, offs, E):
+    """Y[rows of g] = dim0(X)[rows of g] @ 32x32(W[g % E])^T.
+
+    x [M, K] received tokens (bf16 bits) in groups `offs` (G = len(offs), a
+    multiple of E); w [E, N, K]. Returns (Y, |A| |B|^T), float64.
+    """
+    qx, sx = cast_dim0(x_bits)
+    a = dequant(qx, sx)
+    qw, st = cast_32x32(w_bits)
+    s_fwd, _ = w32_scale_views(st)
+    b = dequant(qw, s_fwd)
+    starts, ends = group_bounds(offs)
+    E_, N, _ = b.shape
+    if E_ != E or len(starts) % E:
+        raise ValueError("G must be a multiple of E and w must hold E experts")
+    y = np.zeros((a.shape[0], N))
+    ya = np.zeros((a.shape[0], N))
+    for g in range(len(starts)):
+        r = slice(starts[g], ends[g])
+        y[r] = mm(a[r], b[g % E])
+        ya[r] = mm(np.abs(a[r]), np.abs(b[g % E]))
+    return y, ya
+
+
+def ep_expert_backward(x_bits, w_bits, dy_bits, offs, E):
+    """(dX, |dX| bound, dW, |dW| bound) of the received groups, float64.
+
+    dX[rows of g] = dim0(dY)[rows of g] @ W[g % E] with W's 32x32 codes and
+    their dgrad scale view; dW[e] = sum over groups g = e, e + E, ... of
+    dim1_g(dY)^T dim1_g(X~), dim1_g the per-group columnwise cast and
+    X~ = bf16(dequant(dim0(X))).
+    """
+    starts, ends = group_bounds(offs)
+    G = len(starts)
+    if G % E:
+        raise ValueError("G must be a multiple of E")
+    qd, sd = cast_dim0(dy_bits)
+    da = dequant(qd, sd)
+    qw, st = cast_32x32(w_bits)
+    _, s_dg = w32_scale_views(st)
+    wt = dequant(np.ascontiguousarray(np.swapaxes(qw, 1, 2)), s_dg)          # [E, K, N]
+    dx = np.zeros((da.shape[0], wt.shape[1]))
+    dxa = np.zeros_like(dx)
+    for g in range(G):
+        r = slice(starts[g], ends[g])
+        dx[r] = mm(da[r], wt[g % E])
+        dxa[r] = mm(np.abs(da[r]), np.abs(wt[g % E]))
+    qx, sx = cast_dim0(x_bits)
+    x_deq = f64_to_bf16_bits(dequant_bf16(qx, sx))
+    cap = int(padded_group_starts(offs)[-1])
+    qa, sa = cast_dim1_grouped(dy_bits, offs, cap)
+    qb, sb = cast_dim1_grouped(x_deq, offs, cap)
+    a, b = dequant(qa, sa), dequant(qb, sb)
+    per_group, per_group_abs = grouped_mm_k(a, b, offs), grouped_mm_k(np.abs(a), np.abs(b), offs)
+    dw = per_group.reshape(G // E, E, *per_group.shape[1:]).sum(axis=0)
+    dwa = per_group_abs.reshape(G // E, E, *per_group.shape[1:]).sum(axis=0)
+    return dx, dxa, dw, dwa

@@ -1,0 +1,160 @@
+"""Expert-parallel MoE layer with the MXFP8 all-to-all, on one GPU.
+
+1. The expert side alone: received groups (source rank, local expert) through
+   mx_grouped_mm_experts (group g uses expert g % E) in all three modes,
+   against the oracle's ep_expert_forward / ep_expert_backward.
+2. Two ranks emulated in one process (one stream; nothing waits on another
+   kernel): every rank packs its tokens with the CUDA cast, a host-side copy
+   stands in for the all-to-all (the same slices NCCL would move), the
+   expert GEMMs run per rank, and each rank's y, dx and dw are checked
+   against the oracle.
+3. The module itself over a one-rank NCCL group (the all-to-all is a
+   loopback through NCCL).
+
+GEMM tolerance: |gpu - ref| <= 2^-7 |ref| + 1e-3 (|A| |B|^T).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mx_oracle as O
+from mxfp8_block_scaled_cast_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from mxfp8_block_scaled_cast_b200 import mx as _mx
+    _mx.lib()
+    return _mx
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got, ref, absref, what):
+    bad = ~(np.abs(got - ref) <= O.gemm_bound(ref, absref))
+    assert not bad.any(), f"{what}: {int(bad.sum())} of {bad.size} outside tolerance"
+
+
+@pytest.mark.parametrize("W,E,N,K", [(3, 2, 512, 256), (2, 4, 576, 96)])
+def test_expert_side_groups_cycle_over_experts(mx, W, E, N, K):
+    from mxfp8_block_scaled_cast_b200 import ep
+    rng = np.random.default_rng(W * E + K)
+    recv = rng.integers(0, 300, size=(W, E))
+    recv[0, 1] = 0
+    plan = ep.ExchangePlan(W, E, recv.reshape(-1), recv)        # the send side is not used here
+    M = plan.M_recv
+    xb = S.normal_bf16((M, K), seed=1)
+    wb = S.normal_bf16((E, N, K), 0.02, seed=2)
+    dyb = S.normal_bf16((M, N), 0.1, seed=3)
+    offs = torch.as_tensor(plan.offs_recv()).cuda()
+    rq, rs = mx.cast_dim0_grouped(xb.cuda(), offs, plan.m_cap_recv)
+    wq, wsf, _, wsd = mx.cast_w32x32(wb.cuda(), transposed=False, dgrad_scales=True)
+    rs = rs.view(plan.m_cap_recv // 128, ep.scale_band_bytes(K))
+    y = ep.expert_forward(rq, rs, wq, wsf, plan)
+    dx, dw = ep.expert_backward(dyb.cuda(), rq, rs, wq, wsd, plan)
+    mx.mx_device_error()
+    xbits, wbits, dbits = S.bf16_bits(xb), S.bf16_bits(wb), S.bf16_bits(dyb)
+    of = plan.offs_recv()
+    _close(_f64(y), *O.ep_expert_forward(xbits, wbits, of, E), "forward")
+    dx_ref, dx_abs, dw_ref, dw_abs = O.ep_expert_backward(xbits, wbits, dbits, of, E)
+    _close(_f64(dx), dx_ref, dx_abs, "dgrad")
+    _close(_f64(dw), dw_ref, dw_abs, "wgrad (each expert sums its groups over sources)")
+
+
+def _virtual_a2a(ins, in_splits, out_splits):
+    """What an all-to-all delivers: rank d receives chunk d of every rank's
+    input (chunks cut by that rank's input splits), in rank order."""
+    W = len(ins)
+    starts = [np.concatenate([[0], np.cumsum(sp)]) for sp in in_splits]
+    outs = []
+    for d in range(W):
+        parts = [ins[s][int(starts[s][d]):int(starts[s][d + 1])] for s in range(W)]
+        assert [p.shape[0] for p in parts] == [int(v) for v in out_splits[d]]
+        outs.append(torch.cat(parts) if parts else ins[d][:0])
+    return outs
+
+
+def test_two_ranks_emulated_end_to_end(mx):
+    from mxfp8_block_scaled_cast_b200 import ep
+    W, E, N, K = 2, 3, 256, 576
+    rng = np.random.default_rng(7)
+    counts = [rng.integers(0, 260, size=W * E) for _ in range(W)]
+    counts[1][2] = 0
+    xs = [S.normal_bf16((int(c.sum()), K), seed=10 + r) for r, c in enumerate(counts)]
+    ws = [S.normal_bf16((E, N, K), 0.02, seed=20 + r) for r in range(W)]      # rank r's local experts
+    dys = [S.normal_bf16((int(c.sum()), N), 0.1, seed=30 + r) for r, c in enumerate(counts)]
+    plans = [ep.ExchangePlan(W, E, counts[r], np.stack([counts[s][r * E:(r + 1) * E] for s in range(W)]))
+             for r in range(W)]
+    packed = [ep.pack_mxfp8(xs[r].cuda(), plans[r]) for r in range(W)]
+    rq = _virtual_a2a([p[0] for p in packed], [pl.send_rows for pl in plans], [pl.recv_rows for pl in plans])
+    rs = _virtual_a2a([p[1] for p in packed], [pl.send_rows // 128 for pl in plans],
+                      [pl.recv_rows // 128 for pl in plans])
+    wc = [mx.cast_w32x32(w.cuda(), transposed=False, dgrad_scales=True) for w in ws]
+    y_recv = [ep.expert_forward(rq[r], rs[r], wc[r][0], wc[r][1], plans[r]) for r in range(W)]
+    ys = _virtual_a2a(y_recv, [pl.recv_tokens for pl in plans], [pl.send_tokens for pl in plans])
+    dy_recv = _virtual_a2a([d.cuda() for d in dys], [pl.send_tokens for pl in plans],
+                           [pl.recv_tokens for pl in plans])
+    back = [ep.expert_backward(dy_recv[r], rq[r], rs[r], wc[r][0], wc[r][3], plans[r]) for r in range(W)]
+    dxs = _virtual_a2a([b[0] for b in back], [pl.recv_tokens for pl in plans], [pl.send_tokens for pl in plans])
+    mx.mx_device_error()
+    # the oracle, from each sender's view: token rows of global expert j use expert j % E of rank j // E
+    for r in range(W):
+        wall = np.concatenate([S.bf16_bits(w) for w in ws])                    # [W*E, N, K], global order
+        of = np.cumsum(counts[r])
+        xbits, dbits = S.bf16_bits(xs[r]), S.bf16_bits(dys[r])
+        y_ref, y_abs = O.ep_expert_forward(xbits, wall, of, W * E)
+        _close(_f64(ys[r]), y_ref, y_abs, f"y of rank {r}")
+        dx_ref, dx_abs, _, _ = O.ep_expert_backward(xbits, wall, dbits, of, W * E)
+        _close(_f64(dxs[r]), dx_ref, dx_abs, f"dx of rank {r}")
+    # dW from each expert's view: its received groups, source major
+    for r in range(W):
+        ends = [np.cumsum(c) for c in counts]
+        xr = np.concatenate([S.bf16_bits(xs[s])[(ends[s][j - 1] if j else 0):ends[s][j]]
+                             for s in range(W) for j in range(r * E, (r + 1) * E)])
+        dr = np.concatenate([S.bf16_bits(dys[s])[(ends[s][j - 1] if j else 0):ends[s][j]]
+                             for s in range(W) for j in range(r * E, (r + 1) * E)])
+        _, _, dw_ref, dw_abs = O.ep_expert_backward(xr, S.bf16_bits(ws[r]), dr, plans[r].offs_recv(), E)
+        _close(_f64(back[r][1]), dw_ref, dw_abs, f"dw of rank {r}")
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def test_module_over_a_one_rank_nccl_group(mx):
+    import torch.distributed as dist
+    from mxfp8_block_scaled_cast_b200 import ep
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        E, N, K = 4, 512, 256
+        counts = np.array([100, 0, 333, 129])
+        x = S.normal_bf16((int(counts.sum()), K), seed=40)
+        w = S.normal_bf16((E, N, K), 0.02, seed=41)
+        dy = S.normal_bf16((int(counts.sum()), N), 0.1, seed=42)
+        layer = ep.MXFP8ExpertParallelMM()
+        y = layer.forward(x.cuda(), counts, w.cuda())
+        dx, dw = layer.backward(dy.cuda())
+        mx.mx_device_error()
+        xb, wb, db, of = S.bf16_bits(x), S.bf16_bits(w), S.bf16_bits(dy), np.cumsum(counts)
+        _close(_f64(y), *O.ep_expert_forward(xb, wb, of, E), "y")
+        dx_ref, dx_abs, dw_ref, dw_abs = O.ep_expert_backward(xb, wb, db, of, E)
+        _close(_f64(dx), dx_ref, dx_abs, "dx")
+        _close(_f64(dw), dw_ref, dw_abs, "dw")
+    finally:
+        dist.destroy_process_group()

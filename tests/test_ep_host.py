@@ -1,0 +1,128 @@
+"""Expert-parallel MXFP8 all-to-all on CPU: two gloo ranks, the exchange layout.
+
+The MXFP8 dispatch (prime-rl PR #3388, Overview, enable_a2a) sends each
+rank's tokens, cast rowwise into the padded group layout ordered by
+destination rank, as codes and whole 128-row blocked scale tiles. Here the
+oracle does the cast on each rank (no GPU), the library's own exchange
+functions (ExchangePlan, exchange_counts, dispatch_mxfp8, combine,
+dispatch_bf16) move the bytes over a real two-rank gloo group, and every
+receiver checks that its buffer is bitwise the oracle's padded grouped
+operand of the tokens it should hold -- groups (source rank, local expert),
+source major -- and that the combine returns every row to its sender in
+order.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+W, E, K = 2, 3, 96          # ranks, experts per rank, hidden size (not a multiple of 128)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _counts(rank):
+    rng = np.random.default_rng(200 + rank)
+    c = rng.integers(0, 300, size=W * E)
+    c[rank] = 0                               # an empty group
+    c[-1] = 128 * (rank + 1)                  # and an exact multiple of the tile
+    return c
+
+
+def _tokens(rank):
+    from mxfp8_block_scaled_cast_b200 import synthetic as S
+    return S.bf16_bits(S.normal_bf16((int(_counts(rank).sum()), K), seed=100 + rank))
+
+
+def _worker(rank, port, q):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        import torch
+        import torch.distributed as dist
+        from oracle import mx_oracle as O
+        from mxfp8_block_scaled_cast_b200 import ep
+        dist.init_process_group("gloo", rank=rank, world_size=W)
+        a2a = ep.dist_all_to_all()
+        counts = [_counts(r) for r in range(W)]
+        xs = [_tokens(r) for r in range(W)]
+
+        recv = ep.exchange_counts(counts[rank], W, E, a2a, "cpu")
+        assert np.array_equal(recv, np.stack([counts[s][rank * E:(rank + 1) * E] for s in range(W)]))
+        plan = ep.ExchangePlan(W, E, counts[rank], recv)
+
+        # pack (the oracle's rowwise cast into the send layout) and dispatch
+        qs, ss = O.cast_dim0_grouped(xs[rank], plan.offs_send(), plan.m_cap_send)
+        sb = O.swizzle(ss)
+        assert sb.size == plan.m_cap_send // 128 * ep.scale_band_bytes(K)
+        q_t = torch.from_numpy(qs)
+        s_t = torch.from_numpy(sb).view(plan.m_cap_send // 128, ep.scale_band_bytes(K))
+        rq, rs = ep.dispatch_mxfp8(q_t, s_t, plan, a2a)
+
+        # what this rank must hold: source s's tokens of global experts rank*E + e, source major
+        ends = [np.cumsum(c) for c in counts]
+        rows, origin = [], []
+        for s in range(W):
+            for e in range(E):
+                j = rank * E + e
+                lo = ends[s][j - 1] if j else 0
+                rows.append(xs[s][lo:ends[s][j]])
+                origin += [(s, i) for i in range(lo, ends[s][j])]
+        x_recv = np.concatenate(rows)
+        assert x_recv.shape[0] == plan.M_recv
+        qe, se = O.cast_dim0_grouped(x_recv, plan.offs_recv(), plan.m_cap_recv)
+        assert np.array_equal(rq.numpy(), qe), "received codes differ from the padded grouped operand"
+        assert np.array_equal(rs.numpy().reshape(-1), O.swizzle(se)), "received scale tiles differ"
+
+        # combine: each received row carries its origin, and must come back to it in order
+        y_recv = torch.tensor([s * 1e6 + i for s, i in origin], dtype=torch.float64).reshape(-1, 1).repeat(1, 4)
+        y = ep.combine(y_recv, plan, a2a)
+        want = rank * 1e6 + np.arange(plan.M, dtype=np.float64)
+        assert np.array_equal(y[:, 0].numpy(), want) and np.array_equal(y[:, 3].numpy(), want)
+
+        # dispatch of a bf16 gradient follows the same rows as the tokens
+        dy = torch.from_numpy(xs[rank].astype(np.int16)).view(torch.bfloat16)
+        dy_recv = ep.dispatch_bf16(dy, plan, a2a)
+        assert np.array_equal(dy_recv.view(torch.int16).numpy().view(np.uint16), x_recv)
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except Exception as exc:  # reported to the parent
+        import traceback
+        q.put((rank, traceback.format_exc()))
+        raise SystemExit(1) from exc
+
+
+def test_mxfp8_dispatch_layout_and_combine_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, port, q)) for r in range(W)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+    assert res == {0: "ok", 1: "ok"}, res
+    assert all(p.exitcode == 0 for p in procs)
+
+
+def test_plan_sizes_on_the_host():
+    from mxfp8_block_scaled_cast_b200 import ep
+    send = np.array([0, 5, 128, 129, 1, 0])            # W = 2, E = 3
+    recv = np.array([[3, 0, 200], [128, 7, 0]])
+    p = ep.ExchangePlan(2, 3, send, recv)
+    assert p.M == 263 and p.m_cap_send == 0 + 128 + 128 + 256 + 128 + 0
+    assert list(p.send_rows) == [256, 384] and list(p.send_tokens) == [133, 130]
+    assert p.M_recv == 338 and p.m_cap_recv == 128 + 0 + 256 + 128 + 128 + 0
+    assert list(p.recv_rows) == [384, 256] and list(p.recv_tokens) == [203, 135]
+    assert list(p.offs_recv()) == [3, 3, 203, 331, 338, 338] and p.G_recv == 6
+    assert ep.scale_band_bytes(96) == 128 * 4 and ep.scale_band_bytes(4096) == 128 * 128

@@ -548,3 +548,98 @@ def test_planted_padded_starts_in_hp_wgrad_is_caught(monkeypatch):
     monkeypatch.setattr(O, "hp_grouped_mm_k", slip)
     with pytest.raises(AssertionError):
         test_hp_grouped_mm_k_brute_force_and_empty_group()
+
+
+# ------------------------------------------ expert parallelism (MXFP8 a2a) --
+def _torch_deq(codes, scale_bytes):
+    """Values of E4M3 codes [R, C] with per-32 scale bytes [R, C/32], via torch's float8 type."""
+    v = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return v * np.repeat(2.0 ** (np.asarray(scale_bytes, np.float64) - 127.0), 32, axis=-1)
+
+
+def _ep_case(seed=3):
+    rng = np.random.default_rng(seed)
+    E, W, K, N = 2, 3, 64, 64
+    counts = rng.integers(0, 40, size=W * E)
+    counts[1] = 0                                    # an empty (source, expert) group
+    offs = np.cumsum(counts)
+    M = int(offs[-1])
+    x = S.bf16_bits(S.normal_bf16((M, K), seed=seed))
+    w = S.bf16_bits(S.normal_bf16((E, N, K), 0.1, seed=seed + 1))
+    dy = S.bf16_bits(S.normal_bf16((M, N), 0.1, seed=seed + 2))
+    return E, W, K, N, offs, x, w, dy
+
+
+def test_ep_expert_forward_brute_force_uses_expert_g_mod_e():
+    """Each row of group g times expert g % E, entry by entry, from codes decoded by torch."""
+    E, W, K, N, offs, x, w, _ = _ep_case()
+    y, _ = O.ep_expert_forward(x, w, offs, E)
+    qx, sx = O.cast_dim0(x)
+    xv = _torch_deq(qx, sx)
+    starts, ends = O.group_bounds(offs)
+    for e in range(E):
+        qw, st = O.cast_32x32(w[e])
+        wv = _torch_deq(qw, O.w32_scale_views(st)[0])
+        for g in range(e, W * E, E):
+            for i in range(starts[g], ends[g]):
+                for n in range(0, N, 7):
+                    assert y[i, n] == pytest.approx(sum(xv[i, k] * wv[n, k] for k in range(K)), rel=1e-12, abs=1e-300)
+
+
+def test_ep_expert_backward_dx_brute_force():
+    E, W, K, N, offs, x, w, dy = _ep_case(4)
+    dx, _, _, _ = O.ep_expert_backward(x, w, dy, offs, E)
+    qd, sd = O.cast_dim0(dy)
+    dv = _torch_deq(qd, sd)
+    starts, ends = O.group_bounds(offs)
+    for g in range(W * E):
+        qw, st = O.cast_32x32(w[g % E])
+        wtv = _torch_deq(np.ascontiguousarray(qw.T), O.w32_scale_views(st)[1])    # [K, N]
+        for i in range(starts[g], ends[g], 5):
+            for k in range(0, K, 9):
+                assert dx[i, k] == pytest.approx(sum(dv[i, n] * wtv[k, n] for n in range(N)), rel=1e-12, abs=1e-300)
+
+
+def test_ep_expert_backward_dw_sums_each_experts_groups_over_sources():
+    """dW[e] is the sum over sources of the per-group wgrad of group (source, e), each
+    computed alone by the pinned single-group path (a swapped sum order fails)."""
+    E, W, K, N, offs, x, w, dy = _ep_case(5)
+    _, _, dw, _ = O.ep_expert_backward(x, w, dy, offs, E)
+    qx, sx = O.cast_dim0(x)
+    x_deq = O.f64_to_bf16_bits(O.dequant_bf16(qx, sx))
+    starts, ends = O.group_bounds(offs)
+    for e in range(E):
+        want = np.zeros((N, K))
+        for g in range(e, W * E, E):
+            n = ends[g] - starts[g]
+            if n == 0:
+                continue
+            one = np.array([n])
+            cap = O.padded_rows_capacity(n, 1)
+            qa, sa = O.cast_dim1_grouped(dy[starts[g]:ends[g]], one, cap)
+            qb, sb = O.cast_dim1_grouped(x_deq[starts[g]:ends[g]], one, cap)
+            want += _torch_deq(qa, sa) @ _torch_deq(qb, sb).T
+        np.testing.assert_allclose(dw[e], want, rtol=1e-12, atol=1e-300)
+
+
+def test_ep_one_rank_mx_exact_inputs_equal_the_plain_layer():
+    """With one rank (G == E) and activations that are exact MX values, the expert-side
+    backward is the plain grouped layer's: dequantizing the dispatched codes is exact."""
+    E, K, N = 3, 64, 64
+    sizes = [40, 0, 70]
+    offs = np.cumsum(sizes)
+    M = int(offs[-1])
+    x0 = S.bf16_bits(S.normal_bf16((M, K), seed=9))
+    qx, sx = O.cast_dim0(x0)
+    x = O.f64_to_bf16_bits(O.dequant_bf16(qx, sx))                   # an exact MX tensor
+    w = S.bf16_bits(S.normal_bf16((E, N, K), 0.1, seed=10))
+    dy = S.bf16_bits(S.normal_bf16((M, N), 0.1, seed=11))
+    y, _ = O.ep_expert_forward(x, w, offs, E)
+    cap = O.padded_rows_capacity(M, E)
+    q, s = O.cast_dim0_grouped(x, offs, cap)
+    qw, st = O.cast_32x32(w)
+    np.testing.assert_array_equal(y, O.grouped_mm_m(O.dequant(q, s), O.dequant(qw, O.w32_scale_views(st)[0]), offs))
+    _, _, dw, _ = O.ep_expert_backward(x, w, dy, offs, E)
+    qa, sa = O.cast_dim1_grouped(dy, offs, cap)
+    qb, sb = O.cast_dim1_grouped(x, offs, cap)
+    np.testing.assert_array_equal(dw, O.grouped_mm_k(O.dequant(qa, sa), O.dequant(qb, sb), offs))
