@@ -106,31 +106,39 @@ struct GroupSlot {
 __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ offs, int G,
                                                   long long m_total, long long m_cap,
                                                   long long row0, GroupSlot* out) {
+  // Valid offsets keep every running sum below m_cap, which the launch bounds
+  // to 65535 tiles of 128 rows, so the scan runs in 32-bit arithmetic
+  // (unsigned, so that invalid offsets wrap instead of overflowing; they are
+  // flagged below whatever the sums come to).
   const unsigned full = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
-  long long carry = 0, prev_end = 0;
+  const unsigned r0 = unsigned(row0);
+  unsigned carry = 0u;
+  int prev_end = 0;
   bool bad = false;
-  long long f_src = 0, f_live = 0;
+  unsigned f_src = 0u;
+  long long f_live = 0;
   int f_group = -1;
   for (int base = 0; base < G; base += 32) {
     const int g = base + lane;
     const bool in = g < G;
-    long long e = in ? (long long)__ldg(offs + g) : 0;
-    long long s = __shfl_up_sync(full, e, 1);
+    const int e = in ? __ldg(offs + g) : 0;
+    int s = __shfl_up_sync(full, e, 1);
     if (lane == 0) s = prev_end;
-    long long size = in ? e - s : 0;
-    if (in && size < 0) bad = true;
-    long long pad = size > 0 ? ((size + 127) / 128) * 128 : 0;
-    long long incl = pad;
+    const bool neg = in && (e < s || e < 0);
+    if (neg) bad = true;
+    const unsigned size = (in && !neg) ? unsigned(e - s) : 0u;
+    const unsigned pad = (size + 127u) & ~127u;
+    unsigned incl = pad;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      long long t = __shfl_up_sync(full, incl, o);
+      const unsigned t = __shfl_up_sync(full, incl, o);
       if (lane >= o) incl += t;
     }
-    const long long pend = carry + incl, pbeg = pend - pad;
-    if (in && pad > 0 && row0 >= pbeg && row0 < pend) {
-      f_src = s + (row0 - pbeg);
-      f_live = size - (row0 - pbeg);
+    const unsigned pend = carry + incl, pbeg = pend - pad;
+    if (in && pad > 0u && r0 >= pbeg && r0 < pend) {
+      f_src = unsigned(s) + (r0 - pbeg);
+      f_live = (long long)size - (long long)(r0 - pbeg);
       f_group = g;
     }
     const int last = min(31, G - 1 - base);
@@ -138,7 +146,8 @@ __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ of
     prev_end = __shfl_sync(full, e, last);
   }
   bad = __any_sync(full, bad);
-  if (prev_end != m_total || carry > m_cap) bad = true;
+  // a total past the capacity (or one that wrapped) is invalid too
+  if ((long long)prev_end != m_total || (long long)carry > m_cap || carry < unsigned(prev_end)) bad = true;
   const unsigned hit = __ballot_sync(full, f_group >= 0);
   if (lane == 0) {
     if (bad) {
@@ -149,7 +158,7 @@ __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ of
     }
   }
   if (!bad && hit != 0u && lane == __ffs(hit) - 1) {
-    out->src0 = f_src; out->live = f_live; out->group = f_group;
+    out->src0 = (long long)f_src; out->live = f_live; out->group = f_group;
   }
 }
 
