@@ -274,6 +274,20 @@ def cast_sweep(mx, device, flush):
             sec = timed(fn)
             out[f"{name}_{n}x{n}_gbs"] = round(E * bpe / sec / 1e9, 1)
     del x, q, s, qt, st
+    # the pad-path launch of the MoE step: the fused cast of X [16384, 4096] into
+    # the padded groups of the Dirichlet(1) sizes (bytes: X read, both padded code
+    # copies and both blocked scale buffers written)
+    xm, wm, dym, offs = S.moe_problem(seed=0, device=device)
+    del wm, dym
+    offs = offs.to(device)
+    mm, km = xm.shape
+    cap = mx.mx_padded_rows_capacity(mm, offs.numel())
+    gq, gs = u8(cap, km), u8(mx.mx_scale_bytes(cap, km // 32))
+    gqt, gst = u8(km, cap), u8(mx.mx_scale_bytes(km, cap // 32))
+    sec = timed(lambda: mx.mx_cast_2d_grouped(xm, offs, cap, gq, gs, gqt, gst))
+    nbytes = mm * km * 2 + 2 * cap * km + gs.numel() + gst.numel()
+    out["2d_grouped_moe_16384x4096_gbs"] = round(nbytes / sec / 1e9, 1)
+    del xm, gq, gs, gqt, gst
     g3, n3, k3 = 64, 2048, 7168
     w = S.sweep_tensor((g3, n3, k3), seed=0, device=device)
     wq = u8(g3, n3, k3)
@@ -281,6 +295,34 @@ def cast_sweep(mx, device, flush):
     sec = timed(lambda: mx.mx_cast_w32x32(w, wq, sf, None, sd), reps=5)
     out["32x32_64x2048x7168_gbs"] = round(g3 * n3 * k3 * (2 + 1 + 2 / 32) / sec / 1e9, 1)
     return out
+
+
+def graph_time(fn, iters=100, runs=5):
+    """Seconds per call of `fn`: a CUDA graph of `iters` back-to-back calls, replayed
+    `runs` times, median."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+            for _ in range(iters):
+                fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(runs):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / iters)
+    ts.sort()
+    del g
+    return ts[len(ts) // 2] * 1e-3
 
 
 def gemm_only(mx, step, peaks, iters=100, runs=5):
@@ -366,11 +408,50 @@ def unaligned_bench(mx, device, flush, peaks):
         gbs = r * c * bpe / timed(fn) / 1e9
         out[f"{name}_{r}x{c}_gbs"] = {"gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm, 3)}
     del dy, q, s, qt, st
+    out["kva_linear_M16384_N576_K7168"] = kva_gemms(mx, device, peaks)
     step = MoEStep(mx, device, seed=0, shape=(32, 32768, 2048, 7168), problem=S.unaligned_grouped_problem)
     out["grouped_gemm_G32_K7168_N2048_M32768"] = gemm_only(mx, step, peaks)
     out["grouped_gemm_G32_K7168_N2048_M32768"]["gflop_per_launch"] = round(step.gemm_flops / 1e9, 1)
     del step
     torch.cuda.empty_cache()
+    return out
+
+
+def kva_gemms(mx, device, peaks, Mk=16384, Nk=576, Kk=7168):
+    """The GEMMs around the 576-wide output gradient (torchtitan PR #5334, review
+    thread: the KV-A projection, y [16384, 576] = x [16384, 7168] w [576, 7168]^T):
+    forward (576 output columns: two full 256-column tiles and a 64-column one),
+    dgrad (contraction over 576: four 128-deep K steps and a half one) and wgrad
+    (576 output rows), on the pad path, each timed alone as graph replays."""
+    import torch
+    from mxfp8_block_scaled_cast_b200 import synthetic as S
+    x, w, _ = S.linear_problem(Mk, Nk, Kk, seed=0, device=device)
+    dy = S.sweep_tensor((Mk, Nk), seed=0, device=device)
+    u8 = lambda *sh: torch.empty(*sh, dtype=torch.uint8, device=device)
+    bf = lambda *sh: torch.empty(*sh, dtype=torch.bfloat16, device=device)
+    xq, xs = u8(Mk, Kk), u8(mx.mx_scale_bytes(Mk, Kk // 32))
+    xqt, xst = u8(Kk, Mk), u8(mx.mx_scale_bytes(Kk, Mk // 32))
+    wq, wsf, wsd = u8(Nk, Kk), u8(mx.mx_scale_bytes(Nk, Kk // 32)), u8(mx.mx_scale_bytes(Kk, Nk // 32))
+    dq, ds = u8(Mk, Nk), u8(mx.mx_scale_bytes(Mk, Nk // 32))
+    dqt, dst = u8(Nk, Mk), u8(mx.mx_scale_bytes(Nk, Mk // 32))
+    mx.mx_cast_2d(x, xq, xs, xqt, xst)
+    mx.mx_cast_w32x32(w, wq, wsf, None, wsd)
+    mx.mx_cast_2d(dy, dq, ds, dqt, dst)
+    y, dx, dw = bf(Mk, Nk), bf(Mk, Kk), bf(Nk, Kk)
+    calls = {
+        "fwd": lambda: mx.mx_grouped_mm(xq, xs, wq, wsf, None, 1, mx.MX_GROUPS_M, y, Mk, Nk, Kk, 0),
+        "dgrad": lambda: mx.mx_grouped_mm(dq, ds, wq, wsd, None, 1, mx.MX_GROUPS_M_KN, dx, Mk, Kk, Nk, 0),
+        "wgrad": lambda: mx.mx_grouped_mm(dqt, dst, xqt, xst, None, 1, mx.MX_GROUPS_K, dw, Mk, Nk, Kk, 0),
+    }
+    flops = 2 * Mk * Nk * Kk
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP8_OVER_BF16
+    out = {"gflop_per_launch": round(flops / 1e9, 1)}
+    for name, fn in calls.items():
+        sec = graph_time(fn, iters=50)
+        tf = flops / sec / 1e12
+        out[name] = {"us_per_launch": round(sec * 1e6, 1), "tflops": round(tf, 1),
+                     "frac_of_measured_burst_fp8": round(tf / burst, 3), "frac_of_4500_spec": round(tf / 4500.0, 3)}
+    mx.mx_device_error()
     return out
 
 
@@ -717,6 +798,15 @@ def main(argv=None):
     e2e_value, _ = aggregate(a.elapsed_time(b) / e2e_steps, e2e_steps, world)
     del sets[1]
 
+    # The linear runs first after the step: its GEMMs are short, so its figures
+    # move with the power state the seconds-long GEMM replays below leave behind.
+    linear = None
+    if not args.no_linear:
+        flush = L2Flush(dev)
+        with ClockSampler(local) as lin_clocks:
+            linear = linear_bench(mx, dev, flush, peaks)
+        linear["clocks"] = lin_clocks.summary()
+        del flush
     casts = None
     if not args.no_sweep:
         flush = L2Flush(dev)
@@ -725,10 +815,6 @@ def main(argv=None):
         casts = {k: {"gbs": v, "frac_of_measured_hbm": round(v / hbm, 3), "frac_of_8tbs_spec": round(v / 8000, 3)}
                  for k, v in casts.items()}
     gemm_alone = None if args.no_gemm_only else gemm_only(mx, step, peaks)
-    linear = None
-    if not args.no_linear:
-        flush = L2Flush(dev)
-        linear = linear_bench(mx, dev, flush, peaks)
     unaligned = None
     if not args.no_unaligned:
         flush = L2Flush(dev)
