@@ -126,3 +126,19 @@ def test_plan_sizes_on_the_host():
     assert list(p.recv_rows) == [384, 256] and list(p.recv_tokens) == [203, 135]
     assert list(p.offs_recv()) == [3, 3, 203, 331, 338, 338] and p.G_recv == 6
     assert ep.scale_band_bytes(96) == 128 * 4 and ep.scale_band_bytes(4096) == 128 * 128
+
+
+def test_module_rejects_bad_arguments_before_any_exchange():
+    """Host-side checks of the layer run before any collective or kernel."""
+    import pytest
+    import torch
+    from mxfp8_block_scaled_cast_b200 import ep
+    layer = ep.MXFP8ExpertParallelMM(a2a=lambda *a: pytest.fail("no exchange expected"))
+    x = torch.zeros(10, 64, dtype=torch.bfloat16)
+    w = torch.zeros(2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        layer.forward(x.float(), [5, 5], w)
+    with pytest.raises(ValueError):
+        layer.forward(x, [5, 4], w)                 # counts must cover every token
+    with pytest.raises(RuntimeError):
+        layer.backward(torch.zeros(10, 64, dtype=torch.bfloat16))
