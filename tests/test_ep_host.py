@@ -142,3 +142,43 @@ def test_module_rejects_bad_arguments_before_any_exchange():
         layer.forward(x, [5, 4], w)                 # counts must cover every token
     with pytest.raises(RuntimeError):
         layer.backward(torch.zeros(10, 64, dtype=torch.bfloat16))
+
+
+def _dead_peer_worker(rank, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    import torch.distributed as dist
+    from mxfp8_block_scaled_cast_b200 import ep
+    dist.init_process_group("gloo", rank=rank, world_size=2, timeout=timedelta(seconds=5))
+    if rank == 1:
+        q.put((1, "left"))
+        q.close()
+        q.join_thread()                          # the message is out before the process goes
+        os._exit(0)                              # dies between steps, nothing in flight
+    import time
+    t0 = time.monotonic()
+    try:
+        ep.exchange_counts(np.array([1, 2, 3, 4]), 2, 2, ep.dist_all_to_all(), "cpu")
+        q.put((0, "no error"))
+    except Exception as exc:                     # the collective must end with an error
+        q.put((0, f"error after {time.monotonic() - t0:.0f} s: {type(exc).__name__}"))
+
+
+def test_exchange_with_a_dead_peer_ends_with_an_error():
+    """A rank that leaves between steps: the other rank's all-to-all of the token counts
+    (the first exchange of a step) ends with an error within the group's timeout instead
+    of waiting for good."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dead_peer_worker, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res
