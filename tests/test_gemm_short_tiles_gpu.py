@@ -105,3 +105,29 @@ def test_forward_and_dgrad_many_small_row_groups(mx, sizes):
     ad = O.dequant(qd, sd)
     bt = np.ascontiguousarray(np.transpose(bw, (0, 2, 1)))             # W_g^T: [G, K, N]
     _close(_f64(dx), O.grouped_mm_m(ad, bt, offs), O.grouped_mm_m(np.abs(ad), np.abs(bt), offs), "dgrad")
+
+
+def test_wgrad_launches_on_two_streams_at_once(mx, sizes):
+    """Two wgrad launches running at the same time on two streams (persistent grids
+    sharing the GPU's SMs) give exactly the bits they give one after the other."""
+    M, G = int(sizes.sum()), len(sizes)
+    offs_t = S.offsets_from_sizes(sizes).cuda()
+    cap = mx.mx_padded_rows_capacity(M, G)
+    ops = []
+    for seed in (21, 22):
+        dyb = S.normal_bf16((M, 512), 1e-2, seed=seed, device="cuda")
+        xb = S.normal_bf16((M, 768), 1.0, seed=seed + 10, device="cuda")
+        ops.append((*mx.cast_dim1_grouped(dyb, offs_t, cap), *mx.cast_dim1_grouped(xb, offs_t, cap)))
+    torch.cuda.synchronize()
+    serial = [mx.grouped_mm_wgrad(a, sa, b, sb, offs_t, M) for a, sa, b, sb in ops]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.full_like(serial[0], float("nan")) for _ in ops]
+    for _ in range(3):
+        for s, (a, sa, b, sb), o in zip(streams, ops, outs):
+            with torch.cuda.stream(s):
+                mx.mx_grouped_mm(a, sa, b, sb, offs_t, G, mx.MX_GROUPS_K, o, M, 512, 768, cap)
+        torch.cuda.synchronize()
+        mx.mx_device_error()
+        for o, ref in zip(outs, serial):
+            assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
