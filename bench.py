@@ -243,7 +243,7 @@ def cast_sweep(mx, device, flush):
     import torch
     from mxfp8_block_scaled_cast_b200 import synthetic as S
 
-    def timed(fn, reps=10):
+    def timed(fn, reps=20):
         for _ in range(3):
             fn()
         ts = []
