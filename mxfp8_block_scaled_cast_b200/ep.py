@@ -43,6 +43,7 @@ import torch
 from . import mx
 
 BLOCK_ROWS = 128          # rows of a blocked scale tile: the pad path's group alignment
+MAX_GROUPS = 1024         # groups the grouped casts and GEMMs take (include/mx.h)
 
 
 def _pad(n):
@@ -51,14 +52,7 @@ def _pad(n):
 
 def scale_band_bytes(K: int) -> int:
     """Bytes of the blocked scales of one 128-row band of a [rows, K] rowwise cast."""
-    return mx_scale_bytes_host(BLOCK_ROWS, K // 32)
-
-
-def mx_scale_bytes_host(rows: int, cols: int) -> int:
-    """ceil(rows/128)*128 * ceil(cols/4)*4: the blocked layout's size (host arithmetic)."""
-    if rows <= 0 or cols <= 0:
-        return 0
-    return _pad(rows) * (-(-int(cols) // 4) * 4)
+    return mx.mx_scale_bytes(BLOCK_ROWS, K // 32)
 
 
 @dataclass
@@ -75,9 +69,14 @@ class ExchangePlan:
 
     def __post_init__(self):
         self.send_counts = np.asarray(self.send_counts, dtype=np.int64).reshape(-1)
-        self.recv_counts = np.asarray(self.recv_counts, dtype=np.int64).reshape(self.W, self.E)
-        assert self.send_counts.size == self.W * self.E
-        assert (self.send_counts >= 0).all() and (self.recv_counts >= 0).all()
+        self.recv_counts = np.asarray(self.recv_counts, dtype=np.int64)
+        if self.send_counts.size != self.W * self.E or self.recv_counts.size != self.W * self.E:
+            raise ValueError(f"token counts must hold W*E = {self.W * self.E} entries")
+        self.recv_counts = self.recv_counts.reshape(self.W, self.E)
+        if (self.send_counts < 0).any() or (self.recv_counts < 0).any():
+            raise ValueError("token counts must be >= 0")
+        if self.W * self.E > MAX_GROUPS:
+            raise ValueError(f"W*E = {self.W * self.E} groups exceed the grouped kernels' {MAX_GROUPS}")
         pad = np.array([_pad(c) for c in self.send_counts], dtype=np.int64).reshape(self.W, self.E)
         rpad = np.array([_pad(c) for c in self.recv_counts.reshape(-1)], dtype=np.int64).reshape(self.W, self.E)
         self.M = int(self.send_counts.sum())                          # tokens sent

@@ -182,3 +182,14 @@ def test_exchange_with_a_dead_peer_ends_with_an_error():
             p.kill()
     assert res[1] == "left"
     assert res[0].startswith("error"), res
+
+
+def test_plan_rejects_inconsistent_counts():
+    import pytest
+    from mxfp8_block_scaled_cast_b200 import ep
+    with pytest.raises(ValueError):
+        ep.ExchangePlan(2, 2, [1, 2, 3], [[1, 1], [1, 1]])          # send counts not W*E
+    with pytest.raises(ValueError):
+        ep.ExchangePlan(2, 2, [1, 2, 3, -1], [[1, 1], [1, 1]])      # negative count
+    with pytest.raises(ValueError):
+        ep.ExchangePlan(64, 17, [0] * (64 * 17), [[0] * 17] * 64)   # more groups than the kernels take
