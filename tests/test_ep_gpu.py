@@ -3,8 +3,8 @@
 1. The expert side alone: received groups (source rank, local expert) through
    mx_grouped_mm_experts (group g uses expert g % E) in all three modes,
    against the oracle's ep_expert_forward / ep_expert_backward.
-2. Two ranks emulated in one process (one stream; nothing waits on another
-   kernel): every rank packs its tokens with the CUDA cast, a host-side copy
+2. Two and four ranks emulated in one process (one stream; nothing waits on
+   another kernel): every rank packs its tokens with the CUDA cast, a host-side copy
    stands in for the all-to-all (the same slices NCCL would move), the
    expert GEMMs run per rank, and each rank's y, dx and dw are checked
    against the oracle.
@@ -81,10 +81,10 @@ def _virtual_a2a(ins, in_splits, out_splits):
     return outs
 
 
-def test_two_ranks_emulated_end_to_end(mx):
+@pytest.mark.parametrize("W,E,N,K", [(2, 3, 256, 576), (4, 2, 512, 256)])
+def test_ranks_emulated_end_to_end(mx, W, E, N, K):
     from mxfp8_block_scaled_cast_b200 import ep
-    W, E, N, K = 2, 3, 256, 576
-    rng = np.random.default_rng(7)
+    rng = np.random.default_rng(7 + W)
     counts = [rng.integers(0, 260, size=W * E) for _ in range(W)]
     counts[1][2] = 0
     xs = [S.normal_bf16((int(c.sum()), K), seed=10 + r) for r, c in enumerate(counts)]

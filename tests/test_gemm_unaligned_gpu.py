@@ -172,3 +172,45 @@ def test_sizes_not_a_multiple_of_32_are_rejected(mx):
     with pytest.raises(mx.MXError) as e:
         mx.linear_fwd(x, w)
     assert e.value.status == 3
+
+
+def test_kva_gemms_full_size_sampled(mx):
+    """The three GEMMs around the 576-wide gradient at the size bench.py times them
+    (M=16384 tokens, N=576, K=7168; dense, as the linear runs them): sampled rows of
+    the forward and dgrad (one in every 256-row tile, 32-column slabs in every
+    256-column tile) and sampled 32-column slices of dW, against the oracle."""
+    Mk, Nk, Kk = 16384, 576, 7168
+    x, w, _ = S.linear_problem(Mk, Nk, Kk, seed=0, device="cuda")
+    dy = S.sweep_tensor((Mk, Nk), seed=0, device="cuda")
+    xq, xs, xqt, xst = mx.cast_2d(x)
+    wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
+    dq, ds, dqt, dst = mx.cast_2d(dy)
+    y, dx, dw = _nan(Mk, Nk), _nan(Mk, Kk), _nan(Nk, Kk)
+    mx.mx_grouped_mm(xq, xs, wq, wsf, None, 1, mx.MX_GROUPS_M, y, Mk, Nk, Kk, 0)
+    mx.mx_grouped_mm(dq, ds, wq, wsd, None, 1, mx.MX_GROUPS_M_KN, dx, Mk, Kk, Nk, 0)
+    mx.mx_grouped_mm(dqt, dst, xqt, xst, None, 1, mx.MX_GROUPS_K, dw, Mk, Nk, Kk, 0)
+    mx.mx_device_error()
+    rng = np.random.default_rng(5)
+    rows = np.array([t * 256 + int(rng.integers(256)) for t in range(Mk // 256)] + [0, Mk - 1])
+    xb, wb, db = S.bf16_bits(x), S.bf16_bits(w), S.bf16_bits(dy)
+    # forward: rows x every 32-column slab of the 576 outputs (the third column tile is 64 wide)
+    qx, sx = O.cast_dim0(xb[rows])
+    qw, st = O.cast_32x32(wb)
+    a, b = O.dequant(qx, sx), O.dequant(qw, O.w32_scale_views(st)[0])
+    _assert_close(_f64(y[torch.as_tensor(rows, device="cuda")]), O.mm(a, b), O.mm(np.abs(a), np.abs(b)), "kva forward")
+    # dgrad: contraction over the 576 (four full K steps and a half one), one slab per 256 columns
+    qd, sd = O.cast_dim0(db[rows])
+    ad = O.dequant(qd, sd)
+    for t in range(Kk // 256):
+        k0 = t * 256 + 32 * int(rng.integers(8))
+        qws, sts = O.cast_32x32(wb[:, k0:k0 + 32])
+        bt = O.dequant(np.ascontiguousarray(qws.T), O.w32_scale_views(sts)[1])
+        got = _f64(dx[torch.as_tensor(rows, device="cuda")][:, k0:k0 + 32])
+        _assert_close(got, O.mm(ad, bt), O.mm(np.abs(ad), np.abs(bt)), f"kva dgrad cols {k0}")
+    # wgrad: all 576 rows of dW on sampled 32-column slices (the second row tile is half empty)
+    qa, sa = O.cast_dim1(db)
+    aw = O.dequant(qa, sa)                                                   # [576, Mk]
+    for k0 in (0, 32 * int(rng.integers(1, Kk // 32 - 1)), Kk - 32):
+        qb, sb = O.cast_dim1(xb[:, k0:k0 + 32])
+        bw = O.dequant(qb, sb)
+        _assert_close(_f64(dw[:, k0:k0 + 32]), O.mm(aw, bw), O.mm(np.abs(aw), np.abs(bw)), f"kva wgrad cols {k0}")
