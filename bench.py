@@ -17,8 +17,9 @@ cast and GEMM of the path:
 value = 3 * 2*M*N*K FLOPs per step / step time (TFLOP/s, whole job). Inputs
 are seeded synthetic bf16 tensors on the device (512 MB > the 126 MB L2, so
 no explicit flush between steps). The cast bandwidth of the four cast modes
-on the 16384^2 sweep tensor and the [64, 2048, 7168] expert stack is
-reported beside it (L2 flushed between iterations), and so are the GEMMs
+on the 1024^2 ... 16384^2 sweep tensors and the [64, 2048, 7168] expert stack
+is reported beside it (L2 flushed before every launch; in-stream and isolated
+launch timings), and so are the GEMMs
 alone (CUDA-graph replays), the MXFP8 linear at M=4096, N=4096, K=2048, the
 unaligned geometry (casts of a [16384, 576] gradient; the grouped GEMMs at
 G=32, K=7168, N=2048, M=32768 with skewed groups) and the backward-override
@@ -237,28 +238,91 @@ class MoEStep:
                 calls[name]()
 
 
-def cast_sweep(mx, device, flush):
+def flushed_time(fn, flush, reps=20, pairs=40, runs=15):
+    """Seconds per launch of `fn` with the L2 flushed before it, measured two ways.
+
+    isolated   CUDA events around one launch issued after a flush, median of `reps`.
+               The stream has drained when the start event fires, so this includes the
+               latency of a launch into an idle stream (about 5 us here), which dominates
+               tensors of a few MB.
+    in_stream  a CUDA graph of `pairs` (flush, launch) pairs minus a graph of `pairs`
+               flushes alone, replayed alternately `runs` times, median difference per
+               launch: the launch queued behind other work, as inside a training step;
+               the write-back of its dirty lines during the next flush is charged to it.
+    """
+    import torch
+    iso = isolated_time(fn, flush, reps)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    with torch.cuda.stream(s):
+        for with_fn in (True, False):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                for _ in range(pairs):
+                    flush.zero_()
+                    if with_fn:
+                        fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def replay(g):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    for g in graphs:
+        replay(g)
+    diffs = sorted((replay(graphs[0]) - replay(graphs[1])) / pairs for _ in range(runs))
+    del graphs
+    return iso, max(diffs[len(diffs) // 2], 1e-6) * 1e-3
+
+
+def isolated_time(fn, flush, reps=20):
+    """Seconds per launch of `fn`: CUDA events around one launch issued after an
+    L2 flush, median of `reps` (3 unflushed warm-up launches first)."""
+    import torch
+    for _ in range(3):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ts.sort()
+    return ts[len(ts) // 2] * 1e-3
+
+
+CAST_METHOD = ("gbs: in-stream, a CUDA graph of 40 (L2 flush, cast) pairs minus 40 flushes alone, "
+               "median of 15 alternating replays; gbs_isolated: CUDA events around one launch after a "
+               "flush, median of 20 (includes about 5 us of launch latency into an idle stream)")
+
+
+def cast_rates(nbytes, times, hbm):
+    """GB/s of a cast moving `nbytes`, in-stream and isolated, with the in-stream
+    figure's fractions of the measured copy bandwidth and of the 8 TB/s spec."""
+    iso, ins = times
+    gbs = nbytes / ins / 1e9
+    return {"gbs": round(gbs, 1), "gbs_isolated": round(nbytes / iso / 1e9, 1),
+            "frac_of_measured_hbm": round(gbs / hbm, 3), "frac_of_8tbs_spec": round(gbs / 8000, 3)}
+
+
+def cast_sweep(mx, device, flush, hbm):
     """GB/s of each cast mode on the 1024^2 ... 16384^2 sweep tensors and the expert
-    stack (L2 flushed between iterations; 8192^2, 16384^2 and the stack exceed L2)."""
+    stack, L2 flushed before every launch (8192^2, 16384^2 and the stack also
+    exceed the L2); bytes are the tensor read plus codes and scales written."""
     import torch
     from mxfp8_block_scaled_cast_b200 import synthetic as S
 
-    def timed(fn, reps=20):
-        for _ in range(3):
-            fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ts.sort()
-        return ts[len(ts) // 2] * 1e-3
-
-    out = {}
+    out = {"method": CAST_METHOD}
     for n in (1024, 4096, 8192, 16384):
         x = S.sweep_tensor((n, n), seed=0, device=device)
         u8 = lambda *s: torch.empty(*s, dtype=torch.uint8, device=device)
@@ -271,8 +335,8 @@ def cast_sweep(mx, device, flush):
             "32x32": (lambda: mx.mx_cast_w32x32(x, q, s, None, st), 2 + 1 + 2 / 32),
         }
         for name, (fn, bpe) in modes.items():
-            sec = timed(fn)
-            out[f"{name}_{n}x{n}_gbs"] = round(E * bpe / sec / 1e9, 1)
+            pairs = 40 if n < 16384 else 10
+            out[f"{name}_{n}x{n}_gbs"] = cast_rates(E * bpe, flushed_time(fn, flush, pairs=pairs), hbm)
     del x, q, s, qt, st
     # the pad-path launch of the MoE step: the fused cast of X [16384, 4096] into
     # the padded groups of the Dirichlet(1) sizes (bytes: X read, both padded code
@@ -284,16 +348,17 @@ def cast_sweep(mx, device, flush):
     cap = mx.mx_padded_rows_capacity(mm, offs.numel())
     gq, gs = u8(cap, km), u8(mx.mx_scale_bytes(cap, km // 32))
     gqt, gst = u8(km, cap), u8(mx.mx_scale_bytes(km, cap // 32))
-    sec = timed(lambda: mx.mx_cast_2d_grouped(xm, offs, cap, gq, gs, gqt, gst))
     nbytes = mm * km * 2 + 2 * cap * km + gs.numel() + gst.numel()
-    out["2d_grouped_moe_16384x4096_gbs"] = round(nbytes / sec / 1e9, 1)
+    out["2d_grouped_moe_16384x4096_gbs"] = cast_rates(
+        nbytes, flushed_time(lambda: mx.mx_cast_2d_grouped(xm, offs, cap, gq, gs, gqt, gst), flush), hbm)
     del xm, gq, gs, gqt, gst
     g3, n3, k3 = 64, 2048, 7168
     w = S.sweep_tensor((g3, n3, k3), seed=0, device=device)
     wq = u8(g3, n3, k3)
     sf, sd = u8(g3 * mx.mx_scale_bytes(n3, k3 // 32)), u8(g3 * mx.mx_scale_bytes(k3, n3 // 32))
-    sec = timed(lambda: mx.mx_cast_w32x32(w, wq, sf, None, sd), reps=5)
-    out["32x32_64x2048x7168_gbs"] = round(g3 * n3 * k3 * (2 + 1 + 2 / 32) / sec / 1e9, 1)
+    out["32x32_64x2048x7168_gbs"] = cast_rates(
+        g3 * n3 * k3 * (2 + 1 + 2 / 32),
+        flushed_time(lambda: mx.mx_cast_w32x32(w, wq, sf, None, sd), flush, reps=5, pairs=5, runs=5), hbm)
     return out
 
 
@@ -378,21 +443,6 @@ def unaligned_bench(mx, device, flush, peaks):
     import torch
     from mxfp8_block_scaled_cast_b200 import synthetic as S
 
-    def timed(fn, reps=10):
-        for _ in range(3):
-            fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ts.sort()
-        return ts[len(ts) // 2] * 1e-3
-
     out = {}
     r, c = 16384, 576
     dy = S.sweep_tensor((r, c), seed=0, device=device)
@@ -405,8 +455,7 @@ def unaligned_bench(mx, device, flush, peaks):
     }
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for name, (fn, bpe) in modes.items():
-        gbs = r * c * bpe / timed(fn) / 1e9
-        out[f"{name}_{r}x{c}_gbs"] = {"gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm, 3)}
+        out[f"{name}_{r}x{c}_gbs"] = cast_rates(r * c * bpe, flushed_time(fn, flush), hbm)
     del dy, q, s, qt, st
     out["kva_linear_M16384_N576_K7168"] = kva_gemms(mx, device, peaks)
     step = MoEStep(mx, device, seed=0, shape=(32, 32768, 2048, 7168), problem=S.unaligned_grouped_problem)
@@ -538,27 +587,13 @@ def override_arms(mx, step, flush, peaks):
     """
     import torch
 
-    def timed(fn, reps=10):
-        for _ in range(3):
-            fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ts.sort()
-        return ts[len(ts) // 2] * 1e-3
-
     dev = step.x.device
     dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
     dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=dev)
     xd = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
     wd = torch.empty(G, N, K, dtype=torch.bfloat16, device=dev)
     step.run()     # the forward codes of this step are what the dequantized arm reads
+    timed = lambda fn: isolated_time(fn, flush, reps=10)
     t_dgrad = timed(lambda: mx.mx_grouped_mm_bf16(step.dy, step.w, step.offs, G, mx.MX_GROUPS_M, dx, M, K, N))
     t_wgrad = timed(lambda: mx.mx_grouped_mm_bf16(step.dy, step.x, step.offs, G, mx.MX_GROUPS_K, dw, M, N, K))
     t_dqx = timed(lambda: mx.mx_dequant_dim0_grouped(step.xq, step.xs, step.offs, M, K, step.cap, xd))
@@ -814,10 +849,8 @@ def main(argv=None):
     casts = None
     if not args.no_sweep:
         flush = L2Flush(dev)
-        casts = cast_sweep(mx, dev, flush)
-        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        casts = {k: {"gbs": v, "frac_of_measured_hbm": round(v / hbm, 3), "frac_of_8tbs_spec": round(v / 8000, 3)}
-                 for k, v in casts.items()}
+        casts = cast_sweep(mx, dev, flush, peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        del flush
     gemm_alone = None if args.no_gemm_only else gemm_only(mx, step, peaks)
     unaligned = None
     if not args.no_unaligned:
