@@ -22,8 +22,9 @@ is reported beside it (L2 flushed before every launch; in-stream and isolated
 launch timings), and so are the GEMMs
 alone (CUDA-graph replays), the MXFP8 linear at M=4096, N=4096, K=2048, the
 unaligned geometry (casts of a [16384, 576] gradient; the grouped GEMMs at
-G=32, K=7168, N=2048, M=32768 with skewed groups) and the backward-override
-arms.
+G=32, K=7168, N=2048, M=32768 with skewed groups), the backward-override
+arms, and (one GPU only) the same GEMMs through cuBLASLt's MXFP8 kernel,
+timed interleaved with this library's as context.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs the same step on its own GPU (replicas: the
@@ -433,6 +434,97 @@ def gemm_only(mx, step, peaks, iters=100, runs=5):
     return out
 
 
+def library_mxfp8(mx, step, device, iters=(20, 10), rounds=8):
+    """The same GEMMs through cuBLASLt's MXFP8 kernel (torch._scaled_mm with E8M0
+    scales in the blocked layout this library writes), timed interleaved with this
+    library's kernel in one process (CUDA graphs, order flipped each round, median),
+    so both see the same power state. Dense 8192^3, and the MoE forward as one
+    cuBLASLt call per group (its padded rows; the library has no grouped MXFP8 GEMM)
+    against the one grouped launch. Outputs are compared bitwise."""
+    import torch
+    from mxfp8_block_scaled_cast_b200 import synthetic as S
+    f8, e8 = torch.float8_e4m3fn, torch.float8_e8m0fnu
+
+    def capture(fn, n):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                for _ in range(n):
+                    fn()
+        torch.cuda.synchronize()
+        return g
+
+    def replay_ms(g):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    def interleaved(f_ours, f_lib, n, flops):
+        ga, gb = capture(f_ours, n), capture(f_lib, n)
+        replay_ms(ga)
+        replay_ms(gb)
+        t = {0: [], 1: []}
+        for r in range(rounds):
+            for k in ((0, 1) if r % 2 == 0 else (1, 0)):
+                t[k].append(replay_ms((ga, gb)[k]) / n)
+        del ga, gb
+        med = [sorted(v)[len(v) // 2] for v in (t[0], t[1])]
+        return {"ours_tflops": round(flops / med[0] / 1e9, 1), "cublaslt_tflops": round(flops / med[1] / 1e9, 1),
+                "ours_over_cublaslt": round(med[1] / med[0], 4)}
+
+    out = {"method": "CUDA graphs of back-to-back launches (power-capped), this library and cuBLASLt "
+                     f"alternating over {rounds} rounds, median per launch"}
+    try:
+        n = 8192
+        x = S.normal_bf16((n, n), 1.0, seed=1, device=device)
+        w = S.normal_bf16((n, n), 0.02, seed=2, device=device)
+        xq, xs = mx.cast_dim0(x)
+        wq, wsf, _, _ = mx.cast_w32x32(w, transposed=False)
+        del x, w
+        y = torch.empty(n, n, dtype=torch.bfloat16, device=device)
+        ours = lambda: mx.mx_grouped_mm(xq, xs, wq, wsf, None, 1, mx.MX_GROUPS_M, y, n, n, n, 0)
+        a8, b8, sa, sb = xq.view(f8), wq.view(f8), xs.view(e8), wsf.view(e8)
+        lib = lambda: torch._scaled_mm(a8, b8.t(), sa, sb, out_dtype=torch.bfloat16)
+        ours()
+        same = bool(torch.equal(lib(), y))
+        out["dense_8192"] = dict(interleaved(ours, lib, iters[0], 2 * n ** 3), bitwise_equal=same)
+        del xq, xs, wq, wsf, y, a8, b8, sa, sb
+
+        offs = step.offs.cpu().tolist()
+        sizes = [offs[0]] + [offs[i] - offs[i - 1] for i in range(1, len(offs))]
+        pads = [(v + 127) // 128 * 128 for v in sizes]
+        starts = [sum(pads[:i]) for i in range(len(pads))]
+        band = mx.mx_scale_bytes(128, step.K // 32)            # one 128-row scale band of X
+        per_w = mx.mx_scale_bytes(step.N, step.K // 32)        # one expert's forward scales
+        y_pad = torch.empty(sum(pads), step.N, dtype=torch.bfloat16, device=device)
+        calls = [(step.xq[p:p + m].view(f8), step.wq[g].view(f8),
+                  step.xs[p // 128 * band:(p + m) // 128 * band].view(e8),
+                  step.wsf[g * per_w:(g + 1) * per_w].view(e8), y_pad[p:p + m])
+                 for g, (p, m) in enumerate(zip(starts, pads)) if m]
+
+        def lib_moe():
+            for a8_, b8_, sa_, sb_, yv in calls:
+                torch._scaled_mm(a8_, b8_.t(), sa_, sb_, out_dtype=torch.bfloat16, out=yv)
+        fwd = step.gemms()["fwd"]
+        fwd()
+        lib_moe()
+        same = all(torch.equal(y_pad[p:p + v], step.y[o - v:o]) for p, v, o in zip(starts, sizes, offs) if v)
+        out["moe_fwd_per_group"] = dict(interleaved(fwd, lib_moe, iters[1], step.gemm_flops), bitwise_equal=same,
+                                        library_calls=len(calls))
+        del y_pad, calls
+    except Exception as exc:          # reported, not fatal: the comparison is context
+        out["error"] = repr(exc)[:300]
+    mx.mx_device_error()
+    torch.cuda.empty_cache()
+    return out
+
+
 def unaligned_bench(mx, device, flush, peaks):
     """The unaligned geometry: the casts of a [16384, 576] gradient (576 = 18
     blocks of 32, scale columns padded to 20; L2 flushed between iterations; the
@@ -717,6 +809,8 @@ def main(argv=None):
     p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
     p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
     p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
+    p.add_argument("--no-library", action="store_true",
+                   help="skip the interleaved comparison with cuBLASLt's MXFP8 GEMM")
     p.add_argument("--no-unaligned", action="store_true",
                    help="skip the unaligned geometry ([16384, 576] casts, G=32 skewed grouped GEMMs)")
     p.add_argument("--e2e-steps", type=int, default=None, help="end-to-end steps (default: --steps)")
@@ -852,6 +946,8 @@ def main(argv=None):
         casts = cast_sweep(mx, dev, flush, peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         del flush
     gemm_alone = None if args.no_gemm_only else gemm_only(mx, step, peaks)
+    # a library's kernel is context, measured on a single GPU only
+    library = None if (args.no_library or world > 1) else library_mxfp8(mx, step, dev)
     unaligned = None
     if not args.no_unaligned:
         flush = L2Flush(dev)
@@ -888,6 +984,7 @@ def main(argv=None):
         "backward_overrides": arms,
         "linear": linear,
         "gemm_only": gemm_alone,
+        "library_mxfp8_cublaslt": library,
         "unaligned": unaligned,
     }
     print(json.dumps(line), flush=True)
