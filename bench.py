@@ -670,12 +670,14 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
 
 
 def override_arms(mx, step, flush, peaks):
-    """Backward of the same MoE layer under the two backward overrides.
+    """Backward of the same MoE layer under the two backward overrides and
+    wgrad_with_hp.
 
     high_precision: dX = dY_g W_g and dW_g = dY_g^T X_g as bf16 grouped GEMMs
     on the bf16 operands; dequantized: the same GEMMs on the forward's codes
-    dequantized to bf16 (X from the padded dim0 codes, W from the 32x32 codes).
-    Times are medians of 10 L2-flushed repetitions of each launch.
+    dequantized to bf16 (X from the padded dim0 codes, W from the 32x32 codes);
+    wgrad_with_hp: the rowwise cast of dY and the MXFP8 dgrad, with the bf16
+    wgrad. Times are medians of 10 L2-flushed repetitions of each launch.
     """
     import torch
 
@@ -690,6 +692,9 @@ def override_arms(mx, step, flush, peaks):
     t_wgrad = timed(lambda: mx.mx_grouped_mm_bf16(step.dy, step.x, step.offs, G, mx.MX_GROUPS_K, dw, M, N, K))
     t_dqx = timed(lambda: mx.mx_dequant_dim0_grouped(step.xq, step.xs, step.offs, M, K, step.cap, xd))
     t_dqw = timed(lambda: mx.mx_dequant_dim0(step.wq, step.wsf, G, N, K, wd))
+    # wgrad_with_hp: dY cast rowwise only, the MXFP8 dgrad, and the bf16 wgrad above
+    t_dyc = timed(lambda: mx.mx_cast_dim0_grouped(step.dy, step.offs, step.cap, step.dq, step.ds))
+    t_mxd = timed(step.gemms()["dgrad"])
     mx.mx_device_error()
     bf16_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -706,6 +711,12 @@ def override_arms(mx, step, flush, peaks):
             "dequant_x_gbs": deq_gbs(M * K, t_dqx),
             "dequant_w_gbs": deq_gbs(G * N * K, t_dqw),
             "dequant_frac_of_measured_hbm": round(deq_gbs(G * N * K, t_dqw) / hbm, 3),
+        },
+        "wgrad_with_hp": {
+            "backward_ms": round((t_dyc + t_mxd + t_wgrad) * 1e3, 4),
+            "dy_dim0_cast_ms": round(t_dyc * 1e3, 4),
+            "dgrad_mxfp8_tflops": round(GEMM_FLOPS / t_mxd / 1e12, 1),
+            "wgrad_bf16_tflops": round(GEMM_FLOPS / t_wgrad / 1e12, 1),
         },
     }
 

@@ -519,14 +519,23 @@ class MXFP8GroupedMM:
     "high_precision" uses bf16 grouped GEMMs on the saved bf16 x and w;
     "dequantized" uses the same bf16 GEMMs on the forward's codes turned back
     into bf16 (the gradient of the function the quantized forward computes).
+    ``wgrad_with_hp`` (same page, Known follow-ups: the existing knob that
+    "high_precision" extends to both gradients) keeps the MXFP8 dgrad and
+    takes dw from a bf16 grouped GEMM on the saved bf16 x; under
+    "high_precision" it changes nothing, and with "dequantized" it is
+    rejected (the two would take dw from different operands).
     Only bf16 operands are accepted; a strided dy is made contiguous first.
     """
 
-    def __init__(self, backward_override=None):
+    def __init__(self, backward_override=None, wgrad_with_hp=False):
         if backward_override not in BACKWARD_OVERRIDES:
             raise ValueError(f"backward_override must be one of {BACKWARD_OVERRIDES}, "
                              f"got {backward_override!r}")
         self.backward_override = None if backward_override == "quantized" else backward_override
+        if wgrad_with_hp and self.backward_override == "dequantized":
+            raise ValueError("wgrad_with_hp takes dw from the bf16 activations, the dequantized arm from the "
+                             "forward's codes: set one of them")
+        self.wgrad_with_hp = bool(wgrad_with_hp) and self.backward_override is None
         self._saved = None
 
     def forward(self, x, w, offs):
@@ -569,6 +578,11 @@ class MXFP8GroupedMM:
         x, wq, wsd, offs, m_cap = saved
         M, K = x.shape
         G, N, _ = wq.shape
+        if self.wgrad_with_hp:
+            dq, ds = cast_dim0_grouped(dy, offs, m_cap)
+            dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
+            mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
+            return dx, grouped_mm_bf16_wgrad(dy, x, offs)
         dq, ds, dqt, dst = cast_2d_grouped(dy, offs, m_cap)
         xqt, xst = cast_dim1_grouped(x, offs, m_cap)
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
@@ -583,8 +597,8 @@ class _GroupedMMFn(torch.autograd.Function):
     """Autograd wrapper of MXFP8GroupedMM: forward and backward are its calls."""
 
     @staticmethod
-    def forward(ctx, x, w, offs, backward_override):
-        op = MXFP8GroupedMM(backward_override=backward_override)
+    def forward(ctx, x, w, offs, backward_override, wgrad_with_hp):
+        op = MXFP8GroupedMM(backward_override=backward_override, wgrad_with_hp=wgrad_with_hp)
         y = op.forward(x, w, offs)
         ctx.op = op
         return y
@@ -593,17 +607,18 @@ class _GroupedMMFn(torch.autograd.Function):
     def backward(ctx, dy):
         dx, dw = ctx.op.backward(dy)
         ctx.op = None
-        return dx, dw, None, None
+        return dx, dw, None, None, None
 
 
-def mxfp8_grouped_mm(x, w, offs, backward_override=None):
+def mxfp8_grouped_mm(x, w, offs, backward_override=None, wgrad_with_hp=False):
     """y[rows of g] = x[rows of g] @ w[g]^T through the MXFP8 path, differentiable.
 
     x bf16 [M, K], w bf16 [G, N, K], offs int32 [G] on the device (cumulative
-    group ends). ``backward_override`` as in MXFP8GroupedMM (ao "[moe
-    training] Add backward_override to the MXFP8 grouped GEMM", Design notes).
+    group ends). ``backward_override`` and ``wgrad_with_hp`` as in
+    MXFP8GroupedMM (ao "[moe training] Add backward_override to the MXFP8
+    grouped GEMM", Design notes and Known follow-ups).
     """
-    return _GroupedMMFn.apply(x, w, offs, backward_override)
+    return _GroupedMMFn.apply(x, w, offs, backward_override, wgrad_with_hp)
 
 
 class _LinearFn(torch.autograd.Function):

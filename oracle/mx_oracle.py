@@ -46,7 +46,10 @@ What it computes, and where each step comes from
 * Backward-override arms (ao backward_override PR, Design notes): the
   high-precision arm's two bf16 grouped GEMMs over unpadded groups, the
   dequantized arm's dequantization of the forward's codes to bf16 (round to
-  nearest even), and the grouped dequant that gathers padded rows back.
+  nearest even), and the grouped dequant that gathers padded rows back; and
+  wgrad_with_hp (same PR, Known follow-ups: the existing knob that
+  "high_precision" extends to both gradients), the MXFP8 dgrad beside the
+  bf16 wgrad.
 * Expert parallelism with the MXFP8 all-to-all ("Cache quantized weights for
   full AC", prime-rl PR #3388, Overview: enable_a2a; ao PR #4705, the
   expert-parallel pipeline benchmark): the expert-side forward and backward
@@ -609,6 +612,30 @@ def moe_backward_dequantized(x_bits, w_bits, dy_bits, offs):
     dy = bf16_to_f64(dy_bits)
     return (hp_grouped_mm_m(dy, wd, offs), hp_grouped_mm_m(np.abs(dy), np.abs(wd), offs),
             hp_grouped_mm_k(dy, xd, offs), hp_grouped_mm_k(np.abs(dy), np.abs(xd), offs))
+
+
+def moe_backward_wgrad_hp(x_bits, w_bits, dy_bits, offs):
+    """wgrad_with_hp: the weight gradient in high precision, the input gradient MXFP8.
+
+    The MXFP8 knob that the "high_precision" override extends to both
+    gradients (ao "[moe training] Add backward_override to the MXFP8 grouped
+    GEMM", Known follow-ups). dX_g = dY_g W_g with dY cast rowwise (1x32, along
+    N) into the padded group layout and W cast in 32x32 tiles, read through
+    its dgrad scale view; dW_g = dY_g^T X_g on the bf16 operands. Returns what
+    moe_backward_high_precision returns.
+    """
+    dy_bits = np.asarray(dy_bits, dtype=np.uint16)
+    M = dy_bits.shape[0]
+    G = np.asarray(w_bits).shape[0]
+    m_cap = padded_rows_capacity(M, G)
+    qd, sd = cast_dim0_grouped(dy_bits, offs, m_cap)
+    qw, st = cast_32x32(w_bits)
+    _, s_dgrad = w32_scale_views(st)
+    a = dequant(qd, sd)                                              # [m_cap, N]
+    b = dequant(np.ascontiguousarray(np.swapaxes(qw, 1, 2)), s_dgrad)   # [G, K, N]
+    x, dy = bf16_to_f64(x_bits), bf16_to_f64(dy_bits)
+    return (grouped_mm_m(a, b, offs), grouped_mm_m(np.abs(a), np.abs(b), offs),
+            hp_grouped_mm_k(dy, x, offs), hp_grouped_mm_k(np.abs(dy), np.abs(x), offs))
 
 
 # --------------------------------------------------------------------------

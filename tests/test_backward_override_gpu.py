@@ -239,6 +239,42 @@ def test_stride0_grad_through_every_arm(mx):
     _assert_close(_f64(grads[1][1]), ref[2], ref[3], "hp dw, stride-0 dy")
 
 
+def test_wgrad_with_hp_matches_oracle_and_composes(mx):
+    """wgrad_with_hp: dx is the MXFP8 dgrad (bitwise the default backward's), dw the
+    bf16 wgrad (bitwise the high-precision arm's); with "high_precision" the flag
+    changes nothing. Also through autograd and with a stride-0 dy."""
+    x, w, dy, offs_t = _moe_small(9)
+    out = {}
+    for name, kw in (("mixed", dict(wgrad_with_hp=True)), ("quantized", {}),
+                     ("hp", dict(backward_override="high_precision")),
+                     ("hp_flag", dict(backward_override="high_precision", wgrad_with_hp=True))):
+        op = mx.MXFP8GroupedMM(**kw)
+        op.forward(x.cuda(), w.cuda(), offs_t.cuda())
+        out[name] = op.backward(dy.cuda())
+    mx.mx_device_error()
+    rdx, adx, rdw, adw = O.moe_backward_wgrad_hp(S.bf16_bits(x), S.bf16_bits(w), S.bf16_bits(dy), offs_t.numpy())
+    _assert_close(_f64(out["mixed"][0]), rdx, adx, "wgrad_with_hp dx")
+    _assert_close(_f64(out["mixed"][1]), rdw, adw, "wgrad_with_hp dw")
+    assert torch.equal(out["mixed"][0], out["quantized"][0])
+    assert torch.equal(out["mixed"][1], out["hp"][1])
+    assert torch.equal(out["hp_flag"][0], out["hp"][0]) and torch.equal(out["hp_flag"][1], out["hp"][1])
+
+    xa = x.cuda().requires_grad_(True)
+    wa = w.cuda().requires_grad_(True)
+    mx.mxfp8_grouped_mm(xa, wa, offs_t.cuda(), wgrad_with_hp=True).backward(dy.cuda())
+    assert torch.equal(xa.grad, out["mixed"][0]) and torch.equal(wa.grad, out["mixed"][1])
+
+    ones = torch.ones(1, 1, dtype=torch.bfloat16, device="cuda").expand(x.shape[0], w.shape[1])
+    op = mx.MXFP8GroupedMM(wgrad_with_hp=True)
+    op.forward(x.cuda(), w.cuda(), offs_t.cuda())
+    dx1, dw1 = op.backward(ones)
+    mx.mx_device_error()
+    r = O.moe_backward_wgrad_hp(S.bf16_bits(x), S.bf16_bits(w),
+                                S.bf16_bits(torch.ones(x.shape[0], w.shape[1], dtype=torch.bfloat16)), offs_t.numpy())
+    _assert_close(_f64(dx1), r[0], r[1], "wgrad_with_hp dx, stride-0 dy")
+    _assert_close(_f64(dw1), r[2], r[3], "wgrad_with_hp dw, stride-0 dy")
+
+
 def test_override_validation(mx):
     with pytest.raises(ValueError):
         mx.MXFP8GroupedMM(backward_override="fp32")

@@ -523,6 +523,34 @@ def test_dequantized_arm_equals_high_precision_arm_on_mx_exact_operands():
                               O.moe_backward_dequantized(xg, wb, db, offs)[2])
 
 
+def test_wgrad_hp_arm_on_mx_exact_and_generic_operands():
+    """wgrad_with_hp: with dY MX-exact in 1x32 blocks along N and W MX-exact in
+    32x32 tiles, the MXFP8 dgrad loses nothing, so dX is the plain float64
+    product per group (a torch matmul, to summation order); dW is always the
+    bf16 product, so it
+    equals the high-precision arm's; for a generic dY the dgrad is quantized
+    and differs from the high-precision arm's."""
+    rng = np.random.default_rng(34)
+    offs = np.array([40, 96])                       # groups of 40 and 56 tokens (pad path)
+    db = _mx_exact_bits((96, 64), rng, (1, 32))
+    wb = np.stack([_mx_exact_bits((64, 128), rng, (32, 32)) for _ in range(2)])   # [G, N=64, K=128]
+    xb = S.bf16_bits(S.normal_bf16((96, 128), seed=10))
+    dx, adx, dw, _ = O.moe_backward_wgrad_hp(xb, wb, db, offs)
+    dy_f, w_f, x_f = O.bf16_to_f64(db), O.bf16_to_f64(wb), O.bf16_to_f64(xb)
+    for g, (lo, hi) in enumerate([(0, 40), (40, 96)]):
+        want = (torch.from_numpy(dy_f[lo:hi]) @ torch.from_numpy(w_f[g])).numpy()
+        assert np.allclose(dx[lo:hi], want, rtol=1e-12, atol=1e-300)
+        want = (torch.from_numpy(dy_f[lo:hi]).T @ torch.from_numpy(x_f[lo:hi])).numpy()
+        assert np.allclose(dw[g], want, rtol=1e-12, atol=1e-300)
+    assert np.all(adx >= np.abs(dx))
+    hp = O.moe_backward_high_precision(xb, wb, db, offs)
+    assert np.array_equal(dw, hp[2])
+    dg = S.bf16_bits(S.normal_bf16((96, 64), seed=11))
+    mixed, full = O.moe_backward_wgrad_hp(xb, wb, dg, offs), O.moe_backward_high_precision(xb, wb, dg, offs)
+    assert np.array_equal(mixed[2], full[2])
+    assert not np.array_equal(mixed[0], full[0])
+
+
 def test_dequant_grouped_gathers_padded_rows():
     x = S.normal_bf16((300, 64), seed=9)
     xb = S.bf16_bits(x)
