@@ -74,21 +74,20 @@ __device__ __forceinline__ uint32_t warp_max_u16x2(uint32_t v) {
   return v;
 }
 
+// One 128x128 tile (column tile bx, row tile by, expert bz of a stack) of one
+// cast; every thread of the CTA calls it. `wsmem` holds the four warps'
+// slices, `s_row` / `s_col` the tile's two 512-byte scale tiles.
 template <int kMode, bool kGrouped>
-__global__ void __launch_bounds__(kWarpCastThreads)
-cast_warp_kernel(const CastArgs a) {
+__device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32_t by, uint32_t bz, uint8_t* wsmem,
+                                          GroupSlot* slots, uint8_t* s_row, uint8_t* s_col) {
   constexpr bool kRow = (kMode & kModeRow) != 0;
   constexpr bool kCol = (kMode & kModeCol) != 0;
   constexpr bool kSq = (kMode & kModeSquare) != 0;
   static_assert(!(kSq && (kRow || kCol || kGrouped)), "the 32x32 cast is its own mode");
-  extern __shared__ __align__(128) uint8_t wsmem[];
-  __shared__ GroupSlot slots[kWarpCastWarps];
-  __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
-  __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t c0 = int64_t(blockIdx.x) * kCastTile;
-  const int64_t r0 = int64_t(blockIdx.y) * kCastTile;
-  const int64_t z = blockIdx.z;                       // expert of a 32x32 stack
+  const int64_t c0 = int64_t(bx) * kCastTile;
+  const int64_t r0 = int64_t(by) * kCastTile;
+  const int64_t z = bz;                               // expert of a 32x32 stack
   const uint16_t* __restrict__ x = a.x + z * a.x_stride;
   uint8_t* const q = a.q ? a.q + z * a.q_stride : nullptr;
   uint8_t* const s = a.s ? a.s + z * a.s_stride : nullptr;
@@ -143,8 +142,8 @@ cast_warp_kernel(const CastArgs a) {
 
   const int64_t col_tiles_row = ceil_div(ceil_div(a.C, kBlock), 4);          // of blocked(rows_out, C/32)
   const int64_t col_tiles_col = ceil_div(ceil_div(a.rows_out, kBlock), 4);   // of blocked(C, rows_out/32)
-  const int64_t chunk_row = int64_t(blockIdx.y) * col_tiles_row + blockIdx.x;
-  const int64_t chunk_col = int64_t(blockIdx.x) * col_tiles_col + blockIdx.y;
+  const int64_t chunk_row = int64_t(by) * col_tiles_row + bx;
+  const int64_t chunk_col = int64_t(bx) * col_tiles_col + by;
   const bool rows_out_ok = r0 + rw < a.rows_out;       // the warp's 32 output rows exist
   // row and column code offsets are multiples of 32 bytes, so 256-bit stores
   // only need 32-byte aligned base pointers (the ABI promises 16)
@@ -279,6 +278,58 @@ cast_warp_kernel(const CastArgs a) {
     if ((kCol || kSq) && st != nullptr)
       *reinterpret_cast<uint4*>(st + chunk_col * 512 + (threadIdx.x - 32) * 16) =
           *reinterpret_cast<const uint4*>(s_col + (threadIdx.x - 32) * 16);
+  }
+}
+
+template <int kMode, bool kGrouped>
+__global__ void __launch_bounds__(kWarpCastThreads)
+cast_warp_kernel(const CastArgs a) {
+  extern __shared__ __align__(128) uint8_t wsmem[];
+  __shared__ GroupSlot slots[kWarpCastWarps];
+  __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
+  __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
+  cast_tile<kMode, kGrouped>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col);
+}
+
+// Up to three independent dense casts in one launch (the linear's weight and
+// activation casts): CTAs [0, n0) take cast 0's tiles, the next n1 cast 1's,
+// then cast 2's, each in its own launch order (column tile fastest, then row
+// tile, then expert). One launch instead of several lets the casts' partial
+// last waves share the SMs and drops the gaps between launches; every tile is
+// computed exactly as its own launch would, so the output bits are the same.
+// A mode of -1 marks an unused slot.
+struct CastJobs {
+  CastArgs a[3];
+  uint32_t gx[3], gy[3], gz[3];   // each cast's tile grid (column, row, expert)
+};
+
+template <int kM0, int kM1, int kM2>
+__global__ void __launch_bounds__(kWarpCastThreads)
+cast_multi_kernel(const __grid_constant__ CastJobs j) {
+  extern __shared__ __align__(128) uint8_t wsmem[];
+  __shared__ GroupSlot slots[kWarpCastWarps];
+  __shared__ __align__(16) uint8_t s_row[512];
+  __shared__ __align__(16) uint8_t s_col[512];
+  uint32_t id = blockIdx.x;
+  const uint32_t n0 = j.gx[0] * j.gy[0] * j.gz[0];
+  const uint32_t n1 = kM1 < 0 ? 0u : j.gx[1] * j.gy[1] * j.gz[1];
+  int k = 0;
+  if (id >= n0) {
+    id -= n0;
+    k = 1;
+    if (id >= n1) {
+      id -= n1;
+      k = 2;
+    }
+  }
+  const uint32_t gx = j.gx[k], gy = j.gy[k];
+  const uint32_t bx = id % gx, by = (id / gx) % gy, bz = id / (gx * gy);
+  if (k == 0) {
+    cast_tile<kM0, false>(j.a[0], bx, by, bz, wsmem, slots, s_row, s_col);
+  } else if (k == 1) {
+    if constexpr (kM1 >= 0) cast_tile<kM1, false>(j.a[1], bx, by, bz, wsmem, slots, s_row, s_col);
+  } else {
+    if constexpr (kM2 >= 0) cast_tile<kM2, false>(j.a[2], bx, by, bz, wsmem, slots, s_row, s_col);
   }
 }
 

@@ -108,6 +108,142 @@ mx_status check_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs
   return MX_OK;
 }
 
+// A dense cast whose arguments have been checked: what its own launch would
+// get. The public cast entry points prepare and launch one; the linear
+// launches its weight and activation casts together (cast_multi_kernel).
+struct PreparedCast {
+  CastArgs a;
+  int mode = -1;                  // kModeRow, kModeCol, kModeRowCol or kModeSquare
+  int64_t gx = 0, gy = 0, gz = 0;  // tiles along columns, rows, experts
+};
+
+mx_status prepare_dim0(const void* x, int64_t R, int64_t C, void* q, void* s, PreparedCast* p) {
+  MX_TRY(check_cast_geometry(x, R, C, false));
+  MX_TRY(check_out(q, R > 0, "q"));
+  MX_TRY(check_out(s, R > 0, "s"));
+  p->a = make_args(x, R, C, R);
+  p->a.q = static_cast<uint8_t*>(q);
+  p->a.s = static_cast<uint8_t*>(s);
+  p->mode = kModeRow;
+  p->gx = ceil_div(C, kCastTile);
+  p->gy = ceil_div(R, kCastTile);
+  p->gz = 1;
+  return MX_OK;
+}
+
+mx_status prepare_dim1(const void* x, int64_t R, int64_t C, void* qt, void* st, PreparedCast* p) {
+  MX_TRY(check_cast_geometry(x, R, C, true));
+  MX_TRY(check_out(qt, R > 0, "qt"));
+  MX_TRY(check_out(st, R > 0, "st"));
+  p->a = make_args(x, R, C, R);
+  p->a.qt = static_cast<uint8_t*>(qt);
+  p->a.st = static_cast<uint8_t*>(st);
+  p->mode = kModeCol;
+  p->gx = ceil_div(C, kCastTile);
+  p->gy = ceil_div(R, kCastTile);
+  p->gz = 1;
+  return MX_OK;
+}
+
+mx_status prepare_2d(const void* x, int64_t R, int64_t C, void* q, void* s, void* qt, void* st, PreparedCast* p) {
+  MX_TRY(check_cast_geometry(x, R, C, true));
+  MX_TRY(check_out(q, R > 0, "q"));
+  MX_TRY(check_out(s, R > 0, "s"));
+  MX_TRY(check_out(qt, R > 0, "qt"));
+  MX_TRY(check_out(st, R > 0, "st"));
+  p->a = make_args(x, R, C, R);
+  p->a.q = static_cast<uint8_t*>(q);
+  p->a.s = static_cast<uint8_t*>(s);
+  p->a.qt = static_cast<uint8_t*>(qt);
+  p->a.st = static_cast<uint8_t*>(st);
+  p->mode = kModeRowCol;
+  p->gx = ceil_div(C, kCastTile);
+  p->gy = ceil_div(R, kCastTile);
+  p->gz = 1;
+  return MX_OK;
+}
+
+mx_status prepare_w32x32(const void* w, int64_t G, int64_t N, int64_t K, void* q, void* s_fwd, void* qt,
+                         void* s_dgrad, PreparedCast* p) {
+  MX_REQUIRE(G >= 0, MX_ERR_ARG, "G must be >= 0");
+  MX_TRY(check_cast_geometry(w, N, K, true));
+  MX_REQUIRE(N > 0, MX_ERR_ARG, "N must be > 0");
+  MX_TRY(check_out(q, G > 0, "q"));
+  MX_TRY(check_out(s_fwd, G > 0, "s_fwd"));
+  MX_TRY(check_out(qt, false, "qt"));
+  MX_TRY(check_out(s_dgrad, false, "s_dgrad"));
+  p->a = make_args(w, N, K, N);
+  p->a.q = static_cast<uint8_t*>(q);
+  p->a.s = static_cast<uint8_t*>(s_fwd);
+  p->a.qt = static_cast<uint8_t*>(qt);
+  p->a.st = static_cast<uint8_t*>(s_dgrad);
+  p->a.x_stride = N * K;
+  p->a.q_stride = N * K;
+  p->a.qt_stride = N * K;
+  p->a.s_stride = scale_bytes(N, K / kBlock);
+  p->a.st_stride = scale_bytes(K, N / kBlock);
+  p->mode = kModeSquare;
+  p->gx = ceil_div(K, kCastTile);
+  p->gy = ceil_div(N, kCastTile);
+  p->gz = G;
+  return MX_OK;
+}
+
+mx_status launch_prepared(const PreparedCast& p, cudaStream_t st) {
+  switch (p.mode) {
+    case kModeRow: return launch_cast<kModeRow, false>(p.a, p.gx, p.gy, p.gz, st);
+    case kModeCol: return launch_cast<kModeCol, false>(p.a, p.gx, p.gy, p.gz, st);
+    case kModeRowCol: return launch_cast<kModeRowCol, false>(p.a, p.gx, p.gy, p.gz, st);
+    case kModeSquare: return launch_cast<kModeSquare, false>(p.a, p.gx, p.gy, p.gz, st);
+    default: return fail(MX_ERR_ARG, "internal: unprepared cast");
+  }
+}
+
+// Launches the prepared casts `ps[0..n)` (in order) as one grid when their
+// modes are one of the linear's combinations -- (32x32, rowwise),
+// (fused, columnwise), (32x32, fused, columnwise) -- and one at a time
+// otherwise. Empty casts are dropped.
+mx_status launch_casts(const PreparedCast* ps, int n, cudaStream_t st) {
+  const PreparedCast* c[3];
+  int m = 0;
+  for (int i = 0; i < n; ++i)
+    if (ps[i].gx > 0 && ps[i].gy > 0 && ps[i].gz > 0) {
+      MX_REQUIRE(m < 3, MX_ERR_ARG, "internal: more than three casts in one launch");
+      c[m++] = &ps[i];
+    }
+  if (m == 0) return MX_OK;
+  if (m == 1) return launch_prepared(*c[0], st);
+  CastJobs j;
+  memset(&j, 0, sizeof(j));
+  int64_t total = 0;
+  for (int i = 0; i < m; ++i) {
+    MX_REQUIRE(c[i]->gx < (1ll << 31) && c[i]->gy <= 65535 && c[i]->gz <= 65535, MX_ERR_UNSUPPORTED,
+               "cast grid too large (%lld x %lld x %lld tiles)", (long long)c[i]->gx, (long long)c[i]->gy,
+               (long long)c[i]->gz);
+    j.a[i] = c[i]->a;
+    j.gx[i] = uint32_t(c[i]->gx);
+    j.gy[i] = uint32_t(c[i]->gy);
+    j.gz[i] = uint32_t(c[i]->gz);
+    total += c[i]->gx * c[i]->gy * c[i]->gz;
+  }
+  if (total >= (1ll << 31)) {     // beyond one 1-D grid: each cast on its own
+    for (int i = 0; i < m; ++i) MX_TRY(launch_prepared(*c[i], st));
+    return MX_OK;
+  }
+  const dim3 grid{unsigned(total), 1u, 1u}, block{unsigned(kWarpCastThreads), 1u, 1u};
+  if (m == 2 && c[0]->mode == kModeSquare && c[1]->mode == kModeRow)
+    cast_multi_kernel<kModeSquare, kModeRow, -1><<<grid, block, kWarpCastSmem, st>>>(j);
+  else if (m == 2 && c[0]->mode == kModeRowCol && c[1]->mode == kModeCol)
+    cast_multi_kernel<kModeRowCol, kModeCol, -1><<<grid, block, kWarpCastSmem, st>>>(j);
+  else if (m == 3 && c[0]->mode == kModeSquare && c[1]->mode == kModeRowCol && c[2]->mode == kModeCol)
+    cast_multi_kernel<kModeSquare, kModeRowCol, kModeCol><<<grid, block, kWarpCastSmem, st>>>(j);
+  else {
+    for (int i = 0; i < m; ++i) MX_TRY(launch_prepared(*c[i], st));
+    return MX_OK;
+  }
+  return cuda_check("cast launch");
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -323,64 +459,29 @@ mx_status mx_device_error(void* stream) {
 }
 
 mx_status mx_cast_dim0(const void* x, int64_t R, int64_t C, void* q, void* s, void* stream) {
-  MX_TRY(check_cast_geometry(x, R, C, false));
-  MX_TRY(check_out(q, R > 0, "q"));
-  MX_TRY(check_out(s, R > 0, "s"));
-  CastArgs a = make_args(x, R, C, R);
-  a.q = static_cast<uint8_t*>(q);
-  a.s = static_cast<uint8_t*>(s);
-  return launch_cast<kModeRow, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
-                                      static_cast<cudaStream_t>(stream));
+  PreparedCast p;
+  MX_TRY(prepare_dim0(x, R, C, q, s, &p));
+  return launch_prepared(p, static_cast<cudaStream_t>(stream));
 }
 
 mx_status mx_cast_dim1(const void* x, int64_t R, int64_t C, void* qt, void* st, void* stream) {
-  MX_TRY(check_cast_geometry(x, R, C, true));
-  MX_TRY(check_out(qt, R > 0, "qt"));
-  MX_TRY(check_out(st, R > 0, "st"));
-  CastArgs a = make_args(x, R, C, R);
-  a.qt = static_cast<uint8_t*>(qt);
-  a.st = static_cast<uint8_t*>(st);
-  return launch_cast<kModeCol, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
-                                      static_cast<cudaStream_t>(stream));
+  PreparedCast p;
+  MX_TRY(prepare_dim1(x, R, C, qt, st, &p));
+  return launch_prepared(p, static_cast<cudaStream_t>(stream));
 }
 
 mx_status mx_cast_2d(const void* x, int64_t R, int64_t C, void* q, void* s, void* qt, void* st,
                      void* stream) {
-  MX_TRY(check_cast_geometry(x, R, C, true));
-  MX_TRY(check_out(q, R > 0, "q"));
-  MX_TRY(check_out(s, R > 0, "s"));
-  MX_TRY(check_out(qt, R > 0, "qt"));
-  MX_TRY(check_out(st, R > 0, "st"));
-  CastArgs a = make_args(x, R, C, R);
-  a.q = static_cast<uint8_t*>(q);
-  a.s = static_cast<uint8_t*>(s);
-  a.qt = static_cast<uint8_t*>(qt);
-  a.st = static_cast<uint8_t*>(st);
-  return launch_cast<kModeRowCol, false>(a, ceil_div(C, kCastTile), ceil_div(R, kCastTile), 1,
-                                         static_cast<cudaStream_t>(stream));
+  PreparedCast p;
+  MX_TRY(prepare_2d(x, R, C, q, s, qt, st, &p));
+  return launch_prepared(p, static_cast<cudaStream_t>(stream));
 }
 
 mx_status mx_cast_w32x32(const void* w, int64_t G, int64_t N, int64_t K, void* q, void* s_fwd, void* qt,
                          void* s_dgrad, void* stream) {
-  MX_REQUIRE(G >= 0, MX_ERR_ARG, "G must be >= 0");
-  MX_TRY(check_cast_geometry(w, N, K, true));
-  MX_REQUIRE(N > 0, MX_ERR_ARG, "N must be > 0");
-  MX_TRY(check_out(q, G > 0, "q"));
-  MX_TRY(check_out(s_fwd, G > 0, "s_fwd"));
-  MX_TRY(check_out(qt, false, "qt"));
-  MX_TRY(check_out(s_dgrad, false, "s_dgrad"));
-  CastArgs a = make_args(w, N, K, N);
-  a.q = static_cast<uint8_t*>(q);
-  a.s = static_cast<uint8_t*>(s_fwd);
-  a.qt = static_cast<uint8_t*>(qt);
-  a.st = static_cast<uint8_t*>(s_dgrad);
-  a.x_stride = N * K;
-  a.q_stride = N * K;
-  a.qt_stride = N * K;
-  a.s_stride = scale_bytes(N, K / kBlock);
-  a.st_stride = scale_bytes(K, N / kBlock);
-  return launch_cast<kModeSquare, false>(a, ceil_div(K, kCastTile), ceil_div(N, kCastTile), G,
-                                         static_cast<cudaStream_t>(stream));
+  PreparedCast p;
+  MX_TRY(prepare_w32x32(w, G, N, K, q, s_fwd, qt, s_dgrad, &p));
+  return launch_prepared(p, static_cast<cudaStream_t>(stream));
 }
 
 mx_status mx_cast_dim0_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
@@ -573,21 +674,31 @@ mx_status check_linear(int64_t M, int64_t N, int64_t K, void* ws, size_t ws_byte
   return MX_OK;
 }
 
-// The 32x32 quantization of W: from the cache (hit), re-cast into the cache
-// (miss or stale version), or cast into the workspace tail (no cache).
-mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, uint64_t version, uint8_t* ws_tail,
-                       WeightView* out, cudaStream_t st) {
+// Where this call's 32x32 quantization of W comes from: the cache (hit), a
+// re-cast into the cache (miss or stale version), or a cast into the
+// workspace tail (no cache). A cast to run is returned prepared (`cast.mode`
+// >= 0), so that it can share a launch with the activation casts; a cache
+// entry being refilled is marked invalid here and valid by commit_weight once
+// its cast is launched. The caller holds the cache's lock from plan to commit.
+struct WeightPlan {
+  WeightView view;
+  PreparedCast cast;
+  mx_wcache::Entry* entry = nullptr;
+  uint64_t version = 0;
+};
+
+mx_status plan_weight(const void* w, int64_t N, int64_t K, mx_wcache* cache, uint64_t version, uint8_t* ws_tail,
+                      WeightPlan* out) {
   if (cache == nullptr) {
-    *out = carve_weight(ws_tail, N, K);
-    return mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, nullptr, out->s_dgrad, st);
+    out->view = carve_weight(ws_tail, N, K);
+    return prepare_w32x32(w, 1, N, K, out->view.q, out->view.s_fwd, nullptr, out->view.s_dgrad, &out->cast);
   }
-  std::lock_guard<std::mutex> lk(cache->mu);
   mx_wcache::Entry* e = nullptr;
   for (auto& x : cache->entries)
     if (x.w == w && x.N == N && x.K == K) e = &x;
   if (e != nullptr && e->valid && e->version == version) {
     ++cache->hits;
-    *out = carve_weight(e->q, N, K);
+    out->view = carve_weight(e->q, N, K);
     return MX_OK;
   }
   ++cache->misses;
@@ -610,12 +721,23 @@ mx_status weight_codes(const void* w, int64_t N, int64_t K, mx_wcache* cache, ui
     e->K = K;
     e->q = buf;
   }
-  *out = carve_weight(e->q, N, K);
+  out->view = carve_weight(e->q, N, K);
   e->valid = false;
-  MX_TRY(mx_cast_w32x32(w, 1, N, K, out->q, out->s_fwd, nullptr, out->s_dgrad, st));
-  e->version = version;
-  e->valid = true;
+  MX_TRY(prepare_w32x32(w, 1, N, K, out->view.q, out->view.s_fwd, nullptr, out->view.s_dgrad, &out->cast));
+  out->entry = e;
+  out->version = version;
   return MX_OK;
+}
+
+void commit_weight(const WeightPlan& p) {
+  if (p.entry != nullptr) {
+    p.entry->version = p.version;
+    p.entry->valid = true;
+  }
+}
+
+std::unique_lock<std::mutex> lock_cache(mx_wcache* cache) {
+  return cache ? std::unique_lock<std::mutex>(cache->mu) : std::unique_lock<std::mutex>();
 }
 
 }  // namespace
@@ -631,10 +753,18 @@ mx_status mx_linear_fwd(const void* x, const void* w, int64_t M, int64_t N, int6
   uint8_t* xq = p;
   uint8_t* xs = xq + ceil_to(M * K, 256);
   uint8_t* tail = p + (mx_linear_ws_bytes(M, N, K) - wq_bytes(N, K));
-  WeightView wv;
-  MX_TRY(weight_codes(w, N, K, cache, w_version, tail, &wv, st));
+  // the weight's cast (on a miss) and X's rowwise cast go out as one launch
+  std::unique_lock<std::mutex> lk = lock_cache(cache);
+  WeightPlan wp;
+  MX_TRY(plan_weight(w, N, K, cache, w_version, tail, &wp));
+  PreparedCast casts[2];
+  casts[0] = wp.cast;
+  if (M > 0) MX_TRY(prepare_dim0(x, M, K, xq, xs, &casts[1]));
+  MX_TRY(launch_casts(casts, 2, st));
+  commit_weight(wp);
+  if (lk.owns_lock()) lk.unlock();
   if (M == 0) return MX_OK;
-  MX_TRY(mx_cast_dim0(x, M, K, xq, xs, stream));
+  const WeightView& wv = wp.view;
   return mx_grouped_mm(xq, xs, wv.q, wv.s_fwd, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
 }
 
@@ -651,15 +781,26 @@ mx_status mx_linear_bwd(const void* dy, const void* x, const void* w, int64_t M,
   uint8_t* xqt = dyst + ceil_to(scale_bytes(N, M / kBlock), 256);  // [K, M]
   uint8_t* xst = xqt + ceil_to(K * M, 256);                      // blocked(K, M/32)
   uint8_t* tail = p + (mx_linear_ws_bytes(M, N, K) - wq_bytes(N, K));
-  WeightView wv;
-  MX_TRY(weight_codes(w, N, K, cache, w_version, tail, &wv, st));
+  // the weight's cast (on a miss), dY's fused cast and X's columnwise cast
+  // go out as one launch
+  std::unique_lock<std::mutex> lk = lock_cache(cache);
+  WeightPlan wp;
+  MX_TRY(plan_weight(w, N, K, cache, w_version, tail, &wp));
+  PreparedCast casts[3];
+  casts[0] = wp.cast;
+  if (M > 0) {
+    MX_TRY(prepare_2d(dy, M, N, dyq, dys, dyqt, dyst, &casts[1]));
+    MX_TRY(prepare_dim1(x, M, K, xqt, xst, &casts[2]));
+  }
+  MX_TRY(launch_casts(casts, 3, st));
+  commit_weight(wp);
+  if (lk.owns_lock()) lk.unlock();
   if (M == 0) {
     cudaError_t e = cudaMemsetAsync(dw, 0, size_t(N) * K * 2, st);
     MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
     return MX_OK;
   }
-  MX_TRY(mx_cast_2d(dy, M, N, dyq, dys, dyqt, dyst, stream));
-  MX_TRY(mx_cast_dim1(x, M, K, xqt, xst, stream));
+  const WeightView& wv = wp.view;
   MX_TRY(mx_grouped_mm(dyq, dys, wv.q, wv.s_dgrad, nullptr, 1, MX_GROUPS_M_KN, dx, M, K, N, 0, stream));
   return mx_grouped_mm(dyqt, dyst, xqt, xst, nullptr, 1, MX_GROUPS_K, dw, M, N, K, 0, stream);
 }
@@ -737,9 +878,11 @@ extern "C" mx_status mx_linear_fwd_noalloc(const void* x, const void* w, int64_t
   // Every scratch byte the GEMM reads is written by the two casts of this
   // call (codes and every scale byte, pads included), so nothing needs
   // clearing between calls.
-  MX_TRY(mx_cast_w32x32(w, 1, N, K, wq, wsf, nullptr, nullptr, stream));
+  PreparedCast casts[2];
+  MX_TRY(prepare_w32x32(w, 1, N, K, wq, wsf, nullptr, nullptr, &casts[0]));
+  if (M > 0) MX_TRY(prepare_dim0(x, M, K, xq, xs, &casts[1]));
+  MX_TRY(launch_casts(casts, 2, static_cast<cudaStream_t>(stream)));
   if (M == 0) return MX_OK;
-  MX_TRY(mx_cast_dim0(x, M, K, xq, xs, stream));
   return mx_grouped_mm(xq, xs, wq, wsf, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
 }
 
