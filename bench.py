@@ -886,8 +886,9 @@ def main(argv=None):
     # the device for the optimizer. Two device buffer sets let the copies
     # overlap the compute: while step i runs, the inputs of step i + 1 arrive
     # and the outputs of step i - 1 leave, on their own streams (PCIe is full
-    # duplex). Each step waits for its own inputs; a buffer set is refilled
-    # only after its previous outputs have been copied out.
+    # duplex). A set's inputs are refilled once the step that read them has
+    # run; a step runs once its own inputs have arrived and the outputs its
+    # set held before have left.
     pin = lambda t: t.cpu().pin_memory()
     hx, hw, hdy, hoffs = pin(step.x), pin(step.w), pin(step.dy), pin(step.offs)
     sets = [step, MoEStep(mx, dev, seed=1)]
@@ -901,23 +902,27 @@ def main(argv=None):
 
     def e2e_run(n, start_event=None):
         ev_out = [None, None]
+        ev_used = [None, None]          # the last step that read each set's inputs
         for i in range(n):
             b = i % 2
             st = sets[b]
             with torch.cuda.stream(s_in):
                 if start_event is not None and i == 0:
                     s_in.wait_event(start_event)
-                if ev_out[b] is not None:
-                    s_in.wait_event(ev_out[b])
+                if ev_used[b] is not None:
+                    s_in.wait_event(ev_used[b])
                 st.x.copy_(hx, non_blocking=True)
                 st.dy.copy_(hdy, non_blocking=True)
                 st.offs.copy_(hoffs, non_blocking=True)
                 ev_in = torch.cuda.Event()
                 ev_in.record(s_in)
             comp.wait_event(ev_in)
+            if ev_out[b] is not None:
+                comp.wait_event(ev_out[b])
             st.run()
             ev_comp = torch.cuda.Event()
             ev_comp.record(comp)
+            ev_used[b] = ev_comp
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp)
                 for h, d in zip(hout[b], (st.y, st.dx)):
