@@ -273,9 +273,11 @@ MX_API mx_status mx_scales_unswizzle(const void* s, int64_t R, int64_t C32, void
  *   forward  y  [M, N] = x [M, K] w [N, K]^T   x cast 1x32 (dim0), w 32x32
  *   backward dx [M, K] = dy [M, N] w           dy cast 1x32 along N
  *            dw [N, K] = dy^T x                dy and x cast 32x1 along M
- * dy is cast once by the fused rowwise+columnwise cast. All tensors bf16,
- * row-major. M, N and K multiples of 32 (N or K off the 256-wide tile, such
- * as 576, take the GEMM's pad path).
+ * dy is cast once by the fused rowwise+columnwise cast. The casts of one
+ * call (the weight's, when it is quantized, with x's in the forward; with
+ * dy's and x's in the backward) go out as one kernel launch, followed by the
+ * GEMMs. All tensors bf16, row-major. M, N and K multiples of 32 (N or K off
+ * the 256-wide tile, such as 576, take the GEMM's pad path).
  * ws: caller-owned device workspace of at least mx_linear_ws_bytes(M, N, K)
  * bytes (holds the quantized activations and gradients and, without a
  * cache, the quantized weight); it must stay untouched until the call's
