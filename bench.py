@@ -23,8 +23,9 @@ launch timings), and so are the GEMMs
 alone (CUDA-graph replays), the MXFP8 linear at M=4096, N=4096, K=2048, the
 unaligned geometry (casts of a [16384, 576] gradient; the grouped GEMMs at
 G=32, K=7168, N=2048, M=32768 with skewed groups), the backward-override
-arms, and (one GPU only) the same GEMMs through cuBLASLt's MXFP8 kernel,
-timed interleaved with this library's as context.
+arms, and (one GPU only) the same GEMMs through cuBLASLt's MXFP8 kernel and
+the high-precision arm's through torch._grouped_mm, timed interleaved with
+this library's as context.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs the same step on its own GPU (replicas: the
@@ -525,6 +526,65 @@ def library_mxfp8(mx, step, device, iters=(20, 10), rounds=8):
     return out
 
 
+def library_bf16(mx, step, iters=10, rounds=8):
+    """The high-precision arm's bf16 grouped GEMMs against torch._grouped_mm (a
+    library grouped GEMM) on the same bf16 operands: dX_g = dY_g W_g over row
+    groups and dW_g = dY_g^T X_g over token groups, interleaved CUDA graphs as
+    in library_mxfp8, outputs compared bitwise."""
+    import torch
+    G_, M_, N_, K_ = step.G, step.M, step.N, step.K
+    dx = torch.empty(M_, K_, dtype=torch.bfloat16, device=step.dy.device)
+    dw = torch.empty(G_, N_, K_, dtype=torch.bfloat16, device=step.dy.device)
+    ours = {"dgrad": (lambda: mx.mx_grouped_mm_bf16(step.dy, step.w, step.offs, G_, mx.MX_GROUPS_M, dx, M_, K_, N_), dx),
+            "wgrad": (lambda: mx.mx_grouped_mm_bf16(step.dy, step.x, step.offs, G_, mx.MX_GROUPS_K, dw, M_, N_, K_), dw)}
+    out = {"method": f"CUDA graphs of {iters} launches, this library and torch._grouped_mm alternating over "
+                     f"{rounds} rounds, median per launch"}
+    try:
+        lib = {"dgrad": lambda: torch._grouped_mm(step.dy, step.w, offs=step.offs, out_dtype=torch.bfloat16),
+               "wgrad": lambda: torch._grouped_mm(step.dy.t(), step.x, offs=step.offs, out_dtype=torch.bfloat16)}
+
+        def capture(fn):
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
+                    for _ in range(iters):
+                        fn()
+            torch.cuda.synchronize()
+            return g
+
+        def replay_ms(g):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b)
+
+        for name in ("dgrad", "wgrad"):
+            fn, res = ours[name]
+            fn()
+            same = bool(torch.equal(lib[name](), res))
+            ga, gb = capture(fn), capture(lib[name])
+            replay_ms(ga)
+            replay_ms(gb)
+            t = {0: [], 1: []}
+            for r in range(rounds):
+                for k in ((0, 1) if r % 2 == 0 else (1, 0)):
+                    t[k].append(replay_ms((ga, gb)[k]) / iters)
+            del ga, gb
+            med = [sorted(v)[len(v) // 2] for v in (t[0], t[1])]
+            out[name] = {"ours_tflops": round(GEMM_FLOPS / med[0] / 1e9, 1),
+                         "torch_grouped_mm_tflops": round(GEMM_FLOPS / med[1] / 1e9, 1),
+                         "ours_over_torch": round(med[1] / med[0], 4), "bitwise_equal": same}
+    except Exception as exc:          # reported, not fatal: the comparison is context
+        out["error"] = repr(exc)[:300]
+    mx.mx_device_error()
+    return out
+
+
 def unaligned_bench(mx, device, flush, peaks):
     """The unaligned geometry: the casts of a [16384, 576] gradient (576 = 18
     blocks of 32, scale columns padded to 20; L2 flushed between iterations; the
@@ -821,7 +881,7 @@ def main(argv=None):
     p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
     p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
     p.add_argument("--no-library", action="store_true",
-                   help="skip the interleaved comparison with cuBLASLt's MXFP8 GEMM")
+                   help="skip the interleaved comparisons with library GEMMs (cuBLASLt MXFP8, torch bf16 grouped)")
     p.add_argument("--no-unaligned", action="store_true",
                    help="skip the unaligned geometry ([16384, 576] casts, G=32 skewed grouped GEMMs)")
     p.add_argument("--e2e-steps", type=int, default=None, help="end-to-end steps (default: --steps)")
@@ -964,6 +1024,7 @@ def main(argv=None):
     gemm_alone = None if args.no_gemm_only else gemm_only(mx, step, peaks)
     # a library's kernel is context, measured on a single GPU only
     library = None if (args.no_library or world > 1) else library_mxfp8(mx, step, dev)
+    library_hp = None if (args.no_library or world > 1) else library_bf16(mx, step)
     unaligned = None
     if not args.no_unaligned:
         flush = L2Flush(dev)
@@ -1001,6 +1062,7 @@ def main(argv=None):
         "linear": linear,
         "gemm_only": gemm_alone,
         "library_mxfp8_cublaslt": library,
+        "library_bf16_grouped_mm": library_hp,
         "unaligned": unaligned,
     }
     print(json.dumps(line), flush=True)
