@@ -162,6 +162,26 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
                              const int32_t* offs, int32_t G, int64_t m_cap,
                              void* q, void* s, void* qt, void* st, void* stream);
 
+/* The MXFP8 dispatch of expert parallelism as one kernel ("Cache quantized
+ * weights for full AC", prime-rl PR #3388, Overview: enable_a2a): the dim0
+ * cast into padded groups above, with each group's padded rows written to
+ * their own destination instead of one buffer -- the receiving rank's
+ * buffer, which may be another GPU's memory mapped into this process (a peer
+ * or symmetric-memory mapping; written with plain stores, no TMA).
+ *   dst_q[g]  HOST array of G device pointers: group g's first padded row of
+ *             codes; its rows follow at K bytes each (ceil(size_g/128)*128 rows).
+ *   dst_s[g]  HOST array of G device pointers: group g's first 128-row band of
+ *             blocked scales (mx_scale_bytes(128, K/32) bytes per band).
+ * Every pointer must be non-NULL and 16-byte aligned (checked on the host;
+ * an empty group's destination is never written). Bytes written per group
+ * are exactly those its rows occupy in mx_cast_dim0_grouped's outputs; the
+ * pad capacity past the last group writes nothing. The kernel ends with a
+ * system-scope fence: once it is seen complete (e.g. through a collective
+ * issued after it on the same stream), other GPUs read the stores. */
+MX_API mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t K,
+                                              const int32_t* offs, int32_t G, int64_t m_cap,
+                                              void* const* dst_q, void* const* dst_s, void* stream);
+
 /* -------------------------------------------------- scaled grouped GEMM --
  * The MXFP8 scaled grouped GEMM over an offsets array (ao "[moe training]
  * Add backward_override to the MXFP8 grouped GEMM", Summary: forward, dgrad

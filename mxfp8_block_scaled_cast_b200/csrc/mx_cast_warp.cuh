@@ -77,9 +77,19 @@ __device__ __forceinline__ uint32_t warp_max_u16x2(uint32_t v) {
 // One 128x128 tile (column tile bx, row tile by, expert bz of a stack) of one
 // cast; every thread of the CTA calls it. `wsmem` holds the four warps'
 // slices, `s_row` / `s_col` the tile's two 512-byte scale tiles.
-template <int kMode, bool kGrouped>
+// Destinations of the scatter cast: group g's padded rows (codes) start at
+// q[g], its 128-row scale bands at s[g]. A destination may be another GPU's
+// memory (a peer mapping): the scatter cast writes it with plain stores.
+struct ScatterDests {
+  uint8_t* q[kMaxGroups];
+  uint8_t* s[kMaxGroups];
+};
+
+template <int kMode, bool kGrouped, bool kScatter = false>
 __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32_t by, uint32_t bz, uint8_t* wsmem,
-                                          GroupSlot* slots, uint8_t* s_row, uint8_t* s_col) {
+                                          GroupSlot* slots, uint8_t* s_row, uint8_t* s_col,
+                                          const ScatterDests* dests = nullptr) {
+  static_assert(!kScatter || (kGrouped && kMode == kModeRow), "the scatter cast is the grouped rowwise cast");
   constexpr bool kRow = (kMode & kModeRow) != 0;
   constexpr bool kCol = (kMode & kModeCol) != 0;
   constexpr bool kSq = (kMode & kModeSquare) != 0;
@@ -89,8 +99,8 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
   const int64_t r0 = int64_t(by) * kCastTile;
   const int64_t z = bz;                               // expert of a 32x32 stack
   const uint16_t* __restrict__ x = a.x + z * a.x_stride;
-  uint8_t* const q = a.q ? a.q + z * a.q_stride : nullptr;
-  uint8_t* const s = a.s ? a.s + z * a.s_stride : nullptr;
+  uint8_t* q = a.q ? a.q + z * a.q_stride : nullptr;
+  uint8_t* s = a.s ? a.s + z * a.s_stride : nullptr;
   uint8_t* const qt = a.qt ? a.qt + z * a.qt_stride : nullptr;
   uint8_t* const st = a.st ? a.st + z * a.st_stride : nullptr;
 
@@ -101,6 +111,17 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
     __syncwarp();
     src0 = slots[warp].src0;
     live = slots[warp].live;
+  }
+  if constexpr (kScatter) {
+    // the tile is rows r0 - pstart .. of its group's destination; a tile past
+    // every group has none and writes nothing (the same for the whole CTA,
+    // decided before any copy is issued)
+    const int g = slots[warp].group;
+    if (g < 0) return;
+    const long long pstart = slots[warp].pstart;
+    const int64_t bands = ceil_div(ceil_div(a.C, kBlock), 4) * 512;   // bytes of one 128-row scale band
+    q = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->q[g]) - uintptr_t(pstart * a.C));
+    s = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->s[g]) - uintptr_t((pstart / kCastTile) * bands));
   }
   const int rw = warp * 32;                           // first tile row of this warp
   uint8_t* slice = wsmem + warp * kWarpSliceBytes;
@@ -289,6 +310,22 @@ cast_warp_kernel(const CastArgs a) {
   __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
   __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
   cast_tile<kMode, kGrouped>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col);
+}
+
+// The grouped rowwise cast with each group's padded rows written to its own
+// destination (prime-rl PR #3388, Overview: enable_a2a, the MXFP8 dispatch of
+// expert parallelism): the cast and the token exchange in one kernel, each
+// tile stored straight into the receiving rank's buffer. Ends with a
+// system-scope fence so that the stores to peer memory are visible to the
+// other GPUs once this kernel is seen complete.
+__global__ void __launch_bounds__(kWarpCastThreads)
+cast_scatter_kernel(const __grid_constant__ CastArgs a, const __grid_constant__ ScatterDests d) {
+  extern __shared__ __align__(128) uint8_t wsmem[];
+  __shared__ GroupSlot slots[kWarpCastWarps];
+  __shared__ __align__(16) uint8_t s_row[512];
+  __shared__ __align__(16) uint8_t s_col[512];
+  cast_tile<kModeRow, true, true>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col, &d);
+  __threadfence_system();
 }
 
 // Up to three independent dense casts in one launch (the linear's weight and

@@ -100,6 +100,7 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
 struct GroupSlot {
   long long src0;   // first source row of this tile
   long long live;   // real rows from row0 (may exceed 128 or be <= 0)
+  long long pstart; // the group's first padded row
   int group;        // group index or -1
 };
 
@@ -116,7 +117,7 @@ __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ of
   unsigned carry = 0u;
   int prev_end = 0;
   bool bad = false;
-  unsigned f_src = 0u;
+  unsigned f_src = 0u, f_pbeg = 0u;
   long long f_live = 0;
   int f_group = -1;
   for (int base = 0; base < G; base += 32) {
@@ -139,6 +140,7 @@ __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ of
     if (in && pad > 0u && r0 >= pbeg && r0 < pend) {
       f_src = unsigned(s) + (r0 - pbeg);
       f_live = (long long)size - (long long)(r0 - pbeg);
+      f_pbeg = pbeg;
       f_group = g;
     }
     const int last = min(31, G - 1 - base);
@@ -152,13 +154,13 @@ __device__ __forceinline__ void find_group_of_row(const int32_t* __restrict__ of
   if (lane == 0) {
     if (bad) {
       flag_error(kErrOffsets);
-      out->src0 = 0; out->live = 0; out->group = -1;
+      out->src0 = 0; out->live = 0; out->pstart = 0; out->group = -1;
     } else if (hit == 0u) {
-      out->src0 = 0; out->live = 0; out->group = -1;
+      out->src0 = 0; out->live = 0; out->pstart = 0; out->group = -1;
     }
   }
   if (!bad && hit != 0u && lane == __ffs(hit) - 1) {
-    out->src0 = (long long)f_src; out->live = f_live; out->group = f_group;
+    out->src0 = (long long)f_src; out->live = f_live; out->pstart = (long long)f_pbeg; out->group = f_group;
   }
 }
 

@@ -498,6 +498,31 @@ mx_status mx_cast_dim0_grouped(const void* x, int64_t M, int64_t K, const int32_
                                      static_cast<cudaStream_t>(stream));
 }
 
+mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                                       int64_t m_cap, void* const* dst_q, void* const* dst_s, void* stream) {
+  MX_TRY(check_grouped(x, M, K, offs, G, m_cap));
+  MX_REQUIRE(dst_q != nullptr && dst_s != nullptr, MX_ERR_ARG, "null destination arrays");
+  ScatterDests d;
+  memset(&d, 0, sizeof(d));
+  for (int32_t g = 0; g < G; ++g) {
+    MX_REQUIRE(dst_q[g] != nullptr && dst_s[g] != nullptr, MX_ERR_ARG, "null destination of group %d", g);
+    MX_REQUIRE(aligned16(dst_q[g]) && aligned16(dst_s[g]), MX_ERR_ALIGN,
+               "destination of group %d not 16-byte aligned", g);
+    d.q[g] = static_cast<uint8_t*>(dst_q[g]);
+    d.s[g] = static_cast<uint8_t*>(dst_s[g]);
+  }
+  if (m_cap == 0) return MX_OK;
+  const int64_t row_tiles = m_cap / kCastTile, col_tiles = ceil_div(K, kCastTile);
+  MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535, MX_ERR_UNSUPPORTED,
+             "cast grid too large (%lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles);
+  CastArgs a = make_args(x, M, K, m_cap);
+  a.offs = offs;
+  a.G = G;
+  cast_scatter_kernel<<<dim3(unsigned(col_tiles), unsigned(row_tiles), 1u), kWarpCastThreads, kWarpCastSmem,
+                        static_cast<cudaStream_t>(stream)>>>(a, d);
+  return cuda_check("scatter cast launch");
+}
+
 mx_status mx_cast_dim1_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
                                int64_t m_cap, void* qt, void* st, void* stream) {
   MX_TRY(check_grouped(x, M, K, offs, G, m_cap));

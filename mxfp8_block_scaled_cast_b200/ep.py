@@ -31,7 +31,9 @@ Layout (this implementation's reading; the pages describe no layout):
     dW of expert e sums its groups from every source rank in one GEMM.
 
 Everything that moves data is torch.distributed.all_to_all_single (NCCL over
-NVLink on GPUs); every arithmetic step is a libmx kernel.
+NVLink on GPUs) -- or, for the dispatch with direct=True, the cast kernel
+itself storing into symmetric memory; every arithmetic step is a libmx
+kernel.
 """
 from __future__ import annotations
 
@@ -145,6 +147,85 @@ def dispatch_mxfp8(q, s, plan: ExchangePlan, a2a):
     return rq, rs
 
 
+# --------------------------------------- the dispatch as one kernel ---
+# The same exchange without a send buffer or an all-to-all: the rowwise cast
+# writes each of this rank's token groups straight into its destination's
+# receive buffer (mx_cast_dim0_grouped_scatter; the buffers are mapped into
+# every rank, e.g. symmetric memory over NVLink). The receive layout is the
+# one above, so everything downstream is unchanged. Every rank needs every
+# rank's counts to know where its groups land: one all-gather replaces the
+# all-to-all of the counts.
+def gather_counts(send_counts, W: int, all_gather, device) -> np.ndarray:
+    """counts [W, W*E]: tokens each rank sends to each global expert (one small
+    all-gather; all_gather(out [W, n], inp [n]) as torch.distributed's)."""
+    send = torch.as_tensor(np.asarray(send_counts, dtype=np.int64), device=device)
+    out = torch.empty(W, send.numel(), dtype=torch.int64, device=device)
+    all_gather(out, send)
+    return out.cpu().numpy()
+
+
+def dist_all_gather(group=None):
+    """all_gather over `group` into the rows of `out` (output [W, n], input [n])."""
+    import torch.distributed as dist
+
+    def ag(out, inp):
+        dist.all_gather(list(out.unbind(0)), inp, group=group)
+    return ag
+
+
+@dataclass
+class DirectPlan:
+    """Where rank `rank`'s token groups land in the receive buffers, from every
+    rank's counts ([W, W*E]): rank d's buffer holds groups (source s, local
+    expert e) source-major, each padded to whole 128-row tiles."""
+    W: int
+    E: int
+    rank: int
+    counts: np.ndarray
+
+    def __post_init__(self):
+        c = np.asarray(self.counts, dtype=np.int64)
+        if c.shape != (self.W, self.W * self.E):
+            raise ValueError(f"counts must be [W, W*E] = [{self.W}, {self.W * self.E}]")
+        if not 0 <= self.rank < self.W:
+            raise ValueError("rank outside [0, W)")
+        self.counts = c
+        self.exchange = ExchangePlan(self.W, self.E, c[self.rank], c[:, self.rank * self.E:(self.rank + 1) * self.E])
+        pad = np.vectorize(_pad, otypes=[np.int64])(c) if c.size else c      # [W, W*E]
+        rows = pad.reshape(self.W, self.W, self.E).sum(axis=2)               # rows[s, d]: s's rows to d
+        start = np.concatenate([np.zeros((1, self.W), np.int64), np.cumsum(rows, axis=0)[:-1]])  # [s, d]
+        self.recv_rows_of = rows.sum(axis=0)                                 # m_cap_recv of each rank
+        mine = pad[self.rank].reshape(self.W, self.E)
+        within = np.concatenate([np.zeros((self.W, 1), np.int64), np.cumsum(mine, axis=1)[:, :-1]], axis=1)
+        self.dst_row = (start[self.rank][:, None] + within).reshape(-1)     # per global expert g
+
+    def destinations(self, base_q, base_s, K: int):
+        """Device addresses of each group's first row of codes and first scale
+        band, given every rank's receive code and scale buffer addresses."""
+        band = scale_band_bytes(K)
+        dq, ds = [], []
+        for g, row in enumerate(self.dst_row):
+            d = g // self.E
+            dq.append(int(base_q[d]) + int(row) * K)
+            ds.append(int(base_s[d]) + int(row) // BLOCK_ROWS * band)
+        return dq, ds
+
+
+def dispatch_mxfp8_direct(x, plan: DirectPlan, base_q, base_s):
+    """The MXFP8 dispatch as one kernel: x [M, K] (tokens ordered by global
+    expert) cast rowwise straight into every rank's receive buffer (base_q[d],
+    base_s[d]: rank d's codes [rows, K] and scale bands as mapped on this
+    rank). The ranks must wait for one another (a collective issued after this
+    on the stream) before any of them reads its buffer."""
+    M, K = x.shape
+    ex = plan.exchange
+    if ex.m_cap_send == 0:
+        return
+    offs = torch.as_tensor(ex.offs_send(), device=x.device)
+    dq, ds = plan.destinations(base_q, base_s, K)
+    mx.mx_cast_dim0_grouped_scatter(x, offs, ex.m_cap_send, dq, ds)
+
+
 def expert_forward(rq, rs, wq, wsf, plan: ExchangePlan):
     """y_recv [M_recv, N] bf16 = each received group times its local expert (g % E)."""
     N, K = wq.shape[1], wq.shape[2]
@@ -207,14 +288,60 @@ class MXFP8ExpertParallelMM:
     forward(x [M, K] bf16 ordered by global expert, send_counts [W*E] tokens
     per global expert, w [E, N, K] bf16 local experts) -> y [M, N];
     backward(dy [M, N]) -> (dx [M, K], dw [E, N, K]). `a2a` defaults to
-    torch.distributed.all_to_all_single over `group`."""
+    torch.distributed.all_to_all_single over `group`.
 
-    def __init__(self, group=None, a2a=None):
+    direct=True dispatches with one kernel instead of a cast and an
+    all-to-all: the receive buffers are symmetric memory (every rank's buffer
+    mapped into every rank), each rank's cast writes its groups straight into
+    them with plain stores (no TMA, no multicast), and an all-reduce of one
+    element, ordered on the stream after the cast, is the barrier before the
+    expert GEMMs read. The buffer is kept and grown (collectively, on every
+    rank at once) when the largest receiver needs more rows; the backward
+    reads it, so a second forward of the same layer before its backward is
+    refused."""
+
+    def __init__(self, group=None, a2a=None, direct=False, all_gather=None):
         import torch.distributed as dist
         self.group = group
         self.W = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
         self.a2a = a2a if a2a is not None else dist_all_to_all(group)
+        self.direct = direct
+        self.all_gather = all_gather if all_gather is not None else (dist_all_gather(group) if direct else None)
+        self._recv = None            # direct mode: (buffer, handle, rows, K)
         self._saved = None
+
+    def _receive_buffers(self, rows: int, K: int, device):
+        """(codes base, scale base) of every rank's symmetric receive buffer,
+        holding at least `rows` padded rows; collective when it (re)allocates
+        (every rank computes the same `rows` from the gathered counts)."""
+        if self._recv is None or self._recv[2] < rows or self._recv[3] != K:
+            import torch.distributed as dist
+            import torch.distributed._symmetric_memory as symm_mem
+            cap = max(_pad(rows), BLOCK_ROWS)
+            band = scale_band_bytes(K)
+            buf = symm_mem.empty(cap * K + cap // BLOCK_ROWS * band, dtype=torch.uint8, device=device)
+            grp = self.group if self.group is not None else dist.group.WORLD
+            hdl = symm_mem.rendezvous(buf, grp.group_name)
+            self._recv = (buf, hdl, cap, K)
+        buf, hdl, cap, K = self._recv
+        base_q = [int(p) for p in hdl.buffer_ptrs]
+        return base_q, [b + cap * K for b in base_q]
+
+    def _dispatch_direct(self, x, send_counts, E):
+        import torch.distributed as dist
+        K = x.shape[1]
+        counts = gather_counts(send_counts, self.W, self.all_gather, x.device)
+        plan = DirectPlan(self.W, E, self.rank, counts)
+        base_q, base_s = self._receive_buffers(int(plan.recv_rows_of.max()) if self.W else 0, K, x.device)
+        dispatch_mxfp8_direct(x, plan, base_q, base_s)
+        flag = torch.zeros(1, dtype=torch.float32, device=x.device)
+        dist.all_reduce(flag, group=self.group)      # every rank's stores are in before anyone reads
+        ex = plan.exchange
+        buf, _, cap, _ = self._recv
+        rq = buf[:ex.m_cap_recv * K].view(ex.m_cap_recv, K)
+        rs = buf[cap * K:cap * K + ex.m_cap_recv // BLOCK_ROWS * scale_band_bytes(K)].view(-1, scale_band_bytes(K))
+        return ex, rq, rs
 
     def forward(self, x, send_counts, w):
         for name, t in (("x", x), ("w", w)):
@@ -224,10 +351,16 @@ class MXFP8ExpertParallelMM:
         E = w.shape[0]
         if int(np.sum(send_counts)) != x.shape[0]:
             raise ValueError("send_counts must sum to the number of tokens")
-        recv = exchange_counts(send_counts, self.W, E, self.a2a, x.device)
-        plan = ExchangePlan(self.W, E, send_counts, recv)
-        q, s = pack_mxfp8(x, plan)
-        rq, rs = dispatch_mxfp8(q, s, plan, self.a2a)
+        if self.direct:
+            if self._saved is not None:
+                raise RuntimeError("direct dispatch: the previous forward's backward has not run (its "
+                                   "receive buffer would be overwritten)")
+            plan, rq, rs = self._dispatch_direct(x, send_counts, E)
+        else:
+            recv = exchange_counts(send_counts, self.W, E, self.a2a, x.device)
+            plan = ExchangePlan(self.W, E, send_counts, recv)
+            q, s = pack_mxfp8(x, plan)
+            rq, rs = dispatch_mxfp8(q, s, plan, self.a2a)
         wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
         y = combine(expert_forward(rq, rs, wq, wsf, plan), plan, self.a2a)
         self._saved = (plan, rq, rs, wq, wsd)

@@ -34,6 +34,8 @@ _SIGNATURES = {
     "mx_cast_dim0_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_dim1_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp]),
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "mx_cast_dim0_grouped_scatter": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, ctypes.POINTER(_vp),
+                                                    ctypes.POINTER(_vp), _vp]),
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
     "mx_grouped_mm_experts": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                              _i64, _vp]),
@@ -177,6 +179,19 @@ def mx_cast_2d_grouped(x, offs, m_cap, q, s, qt, st, stream=None):
     M, K = x.shape
     _call("mx_cast_2d_grouped", _p(x), M, K, _p(offs), offs.numel(), m_cap, _p(q), _p(s), _p(qt),
           _p(st), _stream(stream))
+
+
+def mx_cast_dim0_grouped_scatter(x, offs, m_cap, dst_q, dst_s, stream=None):
+    """Grouped rowwise cast with group g's padded rows written at device address
+    dst_q[g] and its scale bands at dst_s[g] (lists of G integers, which may be
+    peer-mapped addresses)."""
+    M, K = x.shape
+    G = offs.numel()
+    if len(dst_q) != G or len(dst_s) != G:
+        raise ValueError("one code and one scale destination per group")
+    arr_q = (_vp * G)(*[int(v) for v in dst_q])
+    arr_s = (_vp * G)(*[int(v) for v in dst_s])
+    _call("mx_cast_dim0_grouped_scatter", _p(x), M, K, _p(offs), G, m_cap, arr_q, arr_s, _stream(stream))
 
 
 def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream=None):

@@ -92,5 +92,13 @@ def test_host_argument_checks_return_before_any_launch():
     assert L.mx_grouped_mm_experts(ok16, ok16, ok16, ok16, None, 1, 2, 0, ok16, 128, 256, 128, 0,
                                    None) == 1                           # dense needs E = 1
     assert L.mx_scales_unswizzle(odd, 4, 4, ok16, None) == 2
+    # the scatter cast checks every destination on the host
+    two = lambda *v: (ctypes.c_void_p * 2)(*v)
+    assert L.mx_cast_dim0_grouped_scatter(ok16, 64, 64, ok16, 2, 256, None, two(0x100000, 0x100000),
+                                          None) == 1                    # null destination array
+    assert L.mx_cast_dim0_grouped_scatter(ok16, 64, 64, ok16, 2, 256, two(0x100000, None),
+                                          two(0x100000, 0x100000), None) == 1   # null destination
+    assert L.mx_cast_dim0_grouped_scatter(ok16, 64, 64, ok16, 2, 256, two(0x100000, 0x100008),
+                                          two(0x100000, 0x100000), None) == 2   # misaligned destination
     msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
     assert b"not a multiple of 32" in msg

@@ -158,3 +158,68 @@ def test_module_over_a_one_rank_nccl_group(mx):
         _close(_f64(dw), dw_ref, dw_abs, "dw")
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("W,E,K", [(2, 3, 576), (4, 2, 256), (3, 1, 96)])
+def test_direct_dispatch_equals_the_all_to_all(mx, W, E, K):
+    """The dispatch as one kernel (every rank's cast storing straight into every
+    receive buffer), ranks emulated in one process with local buffers: each
+    receive buffer is bitwise what the cast + all-to-all path delivers."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    rng = np.random.default_rng(60 + W)
+    counts = rng.integers(0, 260, size=(W, W * E))
+    counts[0, -1] = 0
+    counts[W - 1, :E] = 128
+    xs = [S.normal_bf16((int(counts[r].sum()), K), seed=70 + r).cuda() for r in range(W)]
+    plans = [ep.ExchangePlan(W, E, counts[r], counts[:, r * E:(r + 1) * E]) for r in range(W)]
+    packed = [ep.pack_mxfp8(xs[r], plans[r]) for r in range(W)]
+    rq = _virtual_a2a([p[0] for p in packed], [pl.send_rows for pl in plans], [pl.recv_rows for pl in plans])
+    rs = _virtual_a2a([p[1] for p in packed], [pl.send_rows // 128 for pl in plans],
+                      [pl.recv_rows // 128 for pl in plans])
+    band = ep.scale_band_bytes(K)
+    bq = [torch.full((pl.m_cap_recv, K), 0xA5, dtype=torch.uint8, device="cuda") for pl in plans]
+    bs = [torch.full((pl.m_cap_recv // 128, band), 0xA5, dtype=torch.uint8, device="cuda") for pl in plans]
+    for r in range(W):
+        dplan = ep.DirectPlan(W, E, r, counts)
+        assert dplan.exchange.m_cap_send == plans[r].m_cap_send
+        ep.dispatch_mxfp8_direct(xs[r], dplan, [b.data_ptr() for b in bq], [b.data_ptr() for b in bs])
+    mx.mx_device_error()
+    for d in range(W):
+        assert torch.equal(bq[d], rq[d]), f"codes received by rank {d}"
+        assert torch.equal(bs[d], rs[d]), f"scales received by rank {d}"
+
+
+def test_module_direct_over_a_one_rank_nccl_group(mx):
+    """The layer with the one-kernel dispatch into symmetric memory: outputs and
+    gradients bitwise those of the all-to-all layer; a second forward before
+    the backward is refused."""
+    import torch.distributed as dist
+    from mxfp8_block_scaled_cast_b200 import ep
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        E, N, K = 4, 512, 256
+        counts = np.array([100, 0, 333, 129])
+        x = S.normal_bf16((int(counts.sum()), K), seed=50).cuda()
+        w = S.normal_bf16((E, N, K), 0.02, seed=51).cuda()
+        dy = S.normal_bf16((int(counts.sum()), N), 0.1, seed=52).cuda()
+        ref = ep.MXFP8ExpertParallelMM()
+        y0 = ref.forward(x, counts, w)
+        dx0, dw0 = ref.backward(dy)
+        layer = ep.MXFP8ExpertParallelMM(direct=True)
+        for _ in range(2):                              # the second step reuses the buffer
+            y = layer.forward(x, counts, w)
+            dx, dw = layer.backward(dy)
+            mx.mx_device_error()
+            assert torch.equal(y, y0) and torch.equal(dx, dx0) and torch.equal(dw, dw0)
+        layer.forward(x, counts, w)
+        with pytest.raises(RuntimeError):
+            layer.forward(x, counts, w)
+        layer.backward(dy)
+        del layer
+    finally:
+        dist.destroy_process_group()

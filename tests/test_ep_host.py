@@ -16,6 +16,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -193,3 +194,71 @@ def test_plan_rejects_inconsistent_counts():
         ep.ExchangePlan(2, 2, [1, 2, 3, -1], [[1, 1], [1, 1]])      # negative count
     with pytest.raises(ValueError):
         ep.ExchangePlan(64, 17, [0] * (64 * 17), [[0] * 17] * 64)   # more groups than the kernels take
+
+
+def test_direct_plan_places_groups_in_each_receive_layout():
+    """The one-kernel dispatch's placement: rank r's group for global expert
+    d*E + e starts at the padded start of group (r, e) in rank d's receive
+    layout -- ExchangePlan's, which the expert GEMMs read."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    rng = np.random.default_rng(11)
+    for W, E in ((3, 2), (4, 1), (2, 5)):
+        c = rng.integers(0, 300, size=(W, W * E))
+        c[0, :] = 0
+        c[-1, 0] = 128
+        for r in range(W):
+            p = ep.DirectPlan(W, E, r, c)
+            for d in range(W):
+                ex = ep.ExchangePlan(W, E, c[d], c[:, d * E:(d + 1) * E])
+                assert p.recv_rows_of[d] == ex.m_cap_recv
+                starts = np.concatenate([[0], np.cumsum([-(-v // 128) * 128 for v in ex.recv_counts.reshape(-1)])])
+                for e in range(E):
+                    assert p.dst_row[d * E + e] == starts[r * E + e]
+            K = 96
+            bq = [1 << 20 * (d + 1) for d in range(W)]
+            bs = [(1 << 20 * (d + 1)) + (1 << 19) for d in range(W)]
+            dq, ds = p.destinations(bq, bs, K)
+            for g in range(W * E):
+                d = g // E
+                assert dq[g] == bq[d] + int(p.dst_row[g]) * K
+                assert ds[g] == bs[d] + int(p.dst_row[g]) // 128 * ep.scale_band_bytes(K)
+    with pytest.raises(ValueError):
+        ep.DirectPlan(2, 2, 0, np.zeros((2, 3)))
+    with pytest.raises(ValueError):
+        ep.DirectPlan(2, 2, 2, np.zeros((2, 4)))
+
+
+def _gather_worker(rank, port, q):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        import torch.distributed as dist
+        from mxfp8_block_scaled_cast_b200 import ep
+        dist.init_process_group("gloo", rank=rank, world_size=W)
+        counts = [_counts(r) for r in range(W)]
+        full = ep.gather_counts(counts[rank], W, ep.dist_all_gather(), "cpu")
+        assert np.array_equal(full, np.stack(counts))
+        recv = ep.exchange_counts(counts[rank], W, E, ep.dist_all_to_all(), "cpu")
+        dp = ep.DirectPlan(W, E, rank, full)
+        xp = ep.ExchangePlan(W, E, counts[rank], recv)
+        assert dp.exchange.m_cap_recv == xp.m_cap_recv and dp.exchange.m_cap_send == xp.m_cap_send
+        assert np.array_equal(dp.exchange.offs_recv(), xp.offs_recv())
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except Exception as exc:  # reported to the parent
+        import traceback
+        q.put((rank, traceback.format_exc()))
+        raise SystemExit(1) from exc
+
+
+def test_gathered_counts_give_the_same_plan_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, port, q)) for r in range(W)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+    assert res == {0: "ok", 1: "ok"}, res

@@ -172,3 +172,22 @@ def test_linear_stays_in_bounds(mx, M, N, K):
     g = Guarded()
     mx.mx_linear_fwd_noalloc(x, w, g.bf16(M, N))
     g.check(mx, f"linear without allocation {M}x{N}x{K}")
+
+
+def test_scatter_cast_stays_in_bounds(mx):
+    """The one-kernel MXFP8 dispatch: every rank's groups into every receive
+    buffer (ranks emulated with local buffers), each buffer guarded."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    W, E, K = 3, 2, 576
+    rng = np.random.default_rng(5)
+    counts = rng.integers(0, 300, size=(W, W * E))
+    counts[1, :] = 0
+    plans = [ep.DirectPlan(W, E, r, counts) for r in range(W)]
+    band = ep.scale_band_bytes(K)
+    g = Guarded()
+    bq = [g.u8(int(plans[0].recv_rows_of[d]), K) for d in range(W)]
+    bs = [g.raw(int(plans[0].recv_rows_of[d]) // 128 * band) for d in range(W)]
+    for r in range(W):
+        x = _x(int(counts[r].sum()), K, 30 + r)
+        ep.dispatch_mxfp8_direct(x, plans[r], [b.data_ptr() for b in bq], [b.data_ptr() for b in bs])
+    g.check(mx, "scatter cast")
