@@ -240,6 +240,23 @@ MX_API mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const v
                                        const int32_t* offs, int32_t G, int32_t E, int32_t mode, void* out,
                                        int64_t M, int64_t N, int64_t K, int64_t m_cap, void* stream);
 
+/* The M-group modes above (MX_GROUPS_M, MX_GROUPS_M_KN; offsets required)
+ * with each group's output rows at their own destination: row i of group g
+ * (0 <= i < size_g) is written at out_rows[g] + i*N (bf16 elements) instead
+ * of at out + (start_g + i)*N. This is the combine of expert parallelism
+ * fused into the GEMM ("Cache quantized weights for full AC", prime-rl PR
+ * #3388, Overview: enable_a2a): each expert output row is stored straight
+ * into the rank that sent the token, tile by tile as the GEMM runs, instead
+ * of a bf16 all-to-all afterwards. out_rows is a HOST array of G device
+ * pointers, each non-NULL and 16-byte aligned (checked on the host; an empty
+ * group's destination is never written); a destination may be another GPU's
+ * memory mapped into this process (plain stores). The other arguments and
+ * the bytes per row are those of mx_grouped_mm_experts. */
+MX_API mx_status mx_grouped_mm_experts_to_rows(const void* a_q, const void* a_s, const void* b_q,
+                                               const void* b_s, const int32_t* offs, int32_t G, int32_t E,
+                                               int32_t mode, void* const* out_rows, int64_t M, int64_t N,
+                                               int64_t K, int64_t m_cap, void* stream);
+
 /* ------------------------------------------- backward-override arms -----
  * ao "[moe training] Add backward_override to the MXFP8 grouped GEMM", Design
  * notes: the "high_precision" arm computes dgrad and wgrad of the grouped GEMM

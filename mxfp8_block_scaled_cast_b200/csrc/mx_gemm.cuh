@@ -50,6 +50,8 @@
 // No TMA multicast is used.
 #pragma once
 
+#include <type_traits>
+
 #include "mx_sm100.cuh"
 
 namespace mx {
@@ -284,11 +286,24 @@ __device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int64_t cols_
   }
 }
 
-template <int kMode>
+// Per-group output rows (M-group modes): row i of group g is written at
+// base[g] + i * N instead of out + (start_g + i) * N. A base may be another
+// GPU's memory (the expert-parallel combine: each group's outputs stored
+// straight into the rank that sent its tokens, tile by tile as the GEMM
+// runs). The kernels without it take an empty parameter.
+struct RowDests {
+  __nv_bfloat16* base[kMaxGroups];
+};
+struct NoRowDests {};
+template <bool kRowDests>
+using RowDestsT = typename std::conditional<kRowDests, RowDests, NoRowDests>::type;
+
+template <int kMode, bool kRowDests = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-               const GemmArgs args) {
+               const GemmArgs args, const __grid_constant__ RowDestsT<kRowDests> rdests) {
+  static_assert(!kRowDests || kMode != kGroupsK, "per-group output rows are for the M-group modes");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -537,7 +552,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       if (kMode != kGroupsK) {
         const int64_t start = t.g ? ends[t.g - 1] : 0;
         const int64_t local = row - pstart[t.g];
-        if (local < ends[t.g] - start) dst = a.out + (start + local) * a.N + t.n0;
+        if (local < ends[t.g] - start) {
+          if constexpr (kRowDests) dst = rdests.base[t.g] + local * a.N + t.n0;
+          else dst = a.out + (start + local) * a.N + t.n0;
+        }
         cols_valid = a.N - t.n0;
       } else {
         if (row < a.N) dst = a.out + (int64_t(t.g) * a.N + row) * a.K + t.n0;
@@ -556,6 +574,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   }
 
   // ------------------------------------------------------------ teardown ---
+  if constexpr (kRowDests) __threadfence_system();   // rows stored to other GPUs: visible once this ends
   tc_fence_before();
   __syncthreads();
   cluster_sync();          // no CTA leaves while the pair's MMAs or copies may touch it

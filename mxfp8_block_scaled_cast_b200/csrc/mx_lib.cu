@@ -329,9 +329,10 @@ mx_status make_scale_map(CUtensorMap* m, const void* base, uint64_t chunks) {
   return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int kMode>
+template <int kMode, bool kRowDests = false>
 mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa, const CUtensorMap& msb,
-                      const GemmArgs& ga, int64_t pair_tiles_ub, cudaStream_t st) {
+                      const GemmArgs& ga, int64_t pair_tiles_ub, cudaStream_t st,
+                      const RowDestsT<kRowDests>& rd = RowDestsT<kRowDests>()) {
   static int max_pairs[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -349,17 +350,18 @@ mx_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs[dev] == 0) {       // once per device: shared-memory attribute and the resident pairs
-    e = cudaFuncSetAttribute(mx_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+    e = cudaFuncSetAttribute(mx_gemm_kernel<kMode, kRowDests>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kGemmSmem));
     MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm smem attribute: %s", cudaGetErrorString(e));
     cfg.gridDim = dim3(2, 1, 1);
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<kMode>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<kMode, kRowDests>, &cfg);
     MX_REQUIRE(e == cudaSuccess && n > 0, MX_ERR_CUDA, "no CTA pair fits on this device (%s)", cudaGetErrorString(e));
     max_pairs[dev] = n;
   }
   const int64_t pairs = pair_tiles_ub < max_pairs[dev] ? pair_tiles_ub : max_pairs[dev];
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
-  e = cudaLaunchKernelEx(&cfg, mx_gemm_kernel<kMode>, ma, mb, msa, msb, ga);
+  e = cudaLaunchKernelEx(&cfg, mx_gemm_kernel<kMode, kRowDests>, ma, mb, msa, msb, ga, rd);
   MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return cuda_check("gemm launch");
 }
@@ -555,9 +557,48 @@ mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K, const int32_t*
                                         static_cast<cudaStream_t>(stream));
 }
 
-mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
-                                const int32_t* offs, int32_t G, int32_t E, int32_t mode, void* out, int64_t M,
-                                int64_t N, int64_t K, int64_t m_cap, void* stream) {
+}  // extern "C"
+
+namespace mx {
+namespace {
+// The M-group modes of the grouped GEMM (forward, and dgrad with B read
+// MN-major), arguments checked by the caller: tensor maps and the launch,
+// with per-group output rows when kRowDests.
+template <bool kRowDests>
+mx_status grouped_mm_m_modes(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                             const int32_t* offs, int32_t G, int32_t E, int32_t mode, GemmArgs& ga, int64_t M,
+                             int64_t N, int64_t K, int64_t m_cap, cudaStream_t st, const RowDestsT<kRowDests>& rd) {
+  CUtensorMap map_a, map_b, map_sa, map_sb;
+  const int64_t rows_a = offs ? m_cap : M;
+  ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
+  if (rows_a == 0 || M == 0) return MX_OK;
+  MX_REQUIRE(a_q && a_s && b_q && b_s, MX_ERR_ARG, "null operand");
+  ga.a_sc_tiles = ceil_div(K, kBK);
+  ga.b_sc_tiles = ceil_div(K, kBK);
+  ga.b_sc_group_chunks = scale_bytes(N, K / kBlock) / 512;
+  MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kCtaM));
+  if (mode == MX_GROUPS_M_KN)
+    MX_TRY(make_map(&map_b, b_q, uint64_t(N), uint64_t(E) * uint64_t(K), kBK));
+  else
+    MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(E) * uint64_t(N), kBN / 2));
+  MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(rows_a, K / kBlock) / 512)));
+  MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(E) * uint64_t(ga.b_sc_group_chunks)));
+  const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * ceil_div(N, kBN);
+  if (mode == MX_GROUPS_M_KN)
+    return launch_gemm<kGroupsMKn, kRowDests>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st, rd);
+  return launch_gemm<kGroupsM, kRowDests>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st, rd);
+}
+}  // namespace
+}  // namespace mx
+
+extern "C" {
+
+}  // extern "C"
+
+namespace mx {
+namespace {
+mx_status check_grouped_gemm(int32_t mode, const int32_t* offs, int32_t G, int32_t E, int64_t M, int64_t N, int64_t K,
+                             int64_t m_cap) {
   MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_K || mode == MX_GROUPS_M_KN, MX_ERR_ARG, "unknown mode %d",
              mode);
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
@@ -571,6 +612,50 @@ mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_
     MX_REQUIRE(G == 1 && E == 1, MX_ERR_ARG, "without offsets G and E must be 1 (dense)");
     MX_REQUIRE(M < (1ll << 31), MX_ERR_ARG, "M too large");
   }
+  return MX_OK;
+}
+}  // namespace
+}  // namespace mx
+
+extern "C" {
+
+mx_status mx_grouped_mm_experts_to_rows(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                                        const int32_t* offs, int32_t G, int32_t E, int32_t mode,
+                                        void* const* out_rows, int64_t M, int64_t N, int64_t K, int64_t m_cap,
+                                        void* stream) {
+  MX_REQUIRE(mode == MX_GROUPS_M || mode == MX_GROUPS_M_KN, MX_ERR_ARG,
+             "per-group output rows take the M-group modes (got %d)", mode);
+  MX_REQUIRE(offs != nullptr, MX_ERR_ARG, "per-group output rows need offsets");
+  MX_TRY(check_grouped_gemm(mode, offs, G, E, M, N, K, m_cap));
+  MX_REQUIRE(out_rows != nullptr, MX_ERR_ARG, "null output row array");
+  RowDests rd;
+  memset(&rd, 0, sizeof(rd));
+  for (int32_t g = 0; g < G; ++g) {
+    MX_REQUIRE(out_rows[g] != nullptr, MX_ERR_ARG, "null output rows of group %d", g);
+    MX_REQUIRE(aligned16(out_rows[g]), MX_ERR_ALIGN, "output rows of group %d not 16-byte aligned", g);
+    rd.base[g] = static_cast<__nv_bfloat16*>(out_rows[g]);
+  }
+  const void* ptrs[4] = {a_q, a_s, b_q, b_s};
+  for (const void* p : ptrs) MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "operand not 16-byte aligned");
+  MX_REQUIRE(N % kBlock == 0 && K % kBlock == 0, MX_ERR_UNSUPPORTED,
+             "N = %lld and K = %lld must be multiples of 32", (long long)N, (long long)K);
+  MX_REQUIRE(N < (1ll << 31) && K < (1ll << 31), MX_ERR_ARG, "N or K is 2^31 or more");
+  GemmArgs ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.offs = offs;
+  ga.G = G;
+  ga.E = E;
+  ga.M = M;
+  ga.N = N;
+  ga.K = K;
+  return grouped_mm_m_modes<true>(a_q, a_s, b_q, b_s, offs, G, E, mode, ga, M, N, K, m_cap,
+                                  static_cast<cudaStream_t>(stream), rd);
+}
+
+mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_q, const void* b_s,
+                                const int32_t* offs, int32_t G, int32_t E, int32_t mode, void* out, int64_t M,
+                                int64_t N, int64_t K, int64_t m_cap, void* stream) {
+  MX_TRY(check_grouped_gemm(mode, offs, G, E, M, N, K, m_cap));
   const void* ptrs[5] = {a_q, a_s, b_q, b_s, out};
   for (const void* p : ptrs) MX_REQUIRE(aligned16(p), MX_ERR_ALIGN, "operand not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -593,23 +678,8 @@ mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const void* b_
              "N = %lld and K = %lld must be multiples of 32", (long long)N, (long long)K);
   MX_REQUIRE(N < (1ll << 31) && K < (1ll << 31), MX_ERR_ARG, "N or K is 2^31 or more");
   if (mode != MX_GROUPS_K) {
-    const int64_t rows_a = offs ? m_cap : M;
-    ga.m_cap = offs ? m_cap : ceil_to(M, kBM);
-    if (rows_a == 0 || M == 0) return MX_OK;
-    MX_REQUIRE(a_q && a_s && b_q && b_s && out, MX_ERR_ARG, "null operand");
-    ga.a_sc_tiles = ceil_div(K, kBK);
-    ga.b_sc_tiles = ceil_div(K, kBK);
-    ga.b_sc_group_chunks = scale_bytes(N, K / kBlock) / 512;
-    MX_TRY(make_map(&map_a, a_q, uint64_t(K), uint64_t(rows_a), kCtaM));
-    if (mode == MX_GROUPS_M_KN)
-      MX_TRY(make_map(&map_b, b_q, uint64_t(N), uint64_t(E) * uint64_t(K), kBK));
-    else
-      MX_TRY(make_map(&map_b, b_q, uint64_t(K), uint64_t(E) * uint64_t(N), kBN / 2));
-    MX_TRY(make_scale_map(&map_sa, a_s, uint64_t(scale_bytes(rows_a, K / kBlock) / 512)));
-    MX_TRY(make_scale_map(&map_sb, b_s, uint64_t(E) * uint64_t(ga.b_sc_group_chunks)));
-    const int64_t pair_tiles_ub = (ceil_div(rows_a, kPairM) + (offs ? G : 0)) * ceil_div(N, kBN);
-    if (mode == MX_GROUPS_M_KN) return launch_gemm<kGroupsMKn>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
-    return launch_gemm<kGroupsM>(map_a, map_b, map_sa, map_sb, ga, pair_tiles_ub, st);
+    MX_REQUIRE(out != nullptr || M == 0, MX_ERR_ARG, "null output");
+    return grouped_mm_m_modes<false>(a_q, a_s, b_q, b_s, offs, G, E, mode, ga, M, N, K, m_cap, st, NoRowDests());
   }
   MX_REQUIRE(out != nullptr, MX_ERR_ARG, "null output");
   const int64_t len = offs ? m_cap : M;

@@ -211,6 +211,16 @@ class DirectPlan:
         return dq, ds
 
 
+    def combine_destinations(self, out_base, width: int, itemsize: int = 2):
+        """Device addresses where each group this rank receives sends its output
+        rows: group (source s, local expert e) -> rank s's output buffer
+        (out_base[s], [M_s, width] rows of `itemsize` bytes, in s's token
+        order) at s's first token of global expert rank*E + e."""
+        starts = np.concatenate([np.zeros((self.W, 1), np.int64), np.cumsum(self.counts, axis=1)[:, :-1]], axis=1)
+        return [int(out_base[s]) + int(starts[s, self.rank * self.E + e]) * width * itemsize
+                for s in range(self.W) for e in range(self.E)]
+
+
 def dispatch_mxfp8_direct(x, plan: DirectPlan, base_q, base_s):
     """The MXFP8 dispatch as one kernel: x [M, K] (tokens ordered by global
     expert) cast rowwise straight into every rank's receive buffer (base_q[d],
@@ -224,6 +234,20 @@ def dispatch_mxfp8_direct(x, plan: DirectPlan, base_q, base_s):
     offs = torch.as_tensor(ex.offs_send(), device=x.device)
     dq, ds = plan.destinations(base_q, base_s, K)
     mx.mx_cast_dim0_grouped_scatter(x, offs, ex.m_cap_send, dq, ds)
+
+
+def expert_forward_to_senders(rq, rs, wq, wsf, plan: DirectPlan, y_base):
+    """The expert GEMMs with the combine fused: each received group's outputs
+    stored straight into the rank that sent its tokens (y_base[s]: rank s's
+    output buffer [M_s, N] bf16 as mapped here), tile by tile as the GEMM runs.
+    The ranks must wait for one another before reading their outputs."""
+    ex = plan.exchange
+    N, K = wq.shape[1], wq.shape[2]
+    if ex.M_recv == 0:
+        return
+    offs = torch.as_tensor(ex.offs_recv(), device=rq.device)
+    mx.mx_grouped_mm_experts_to_rows(rq, rs, wq, wsf, offs, ex.G_recv, ex.E, mx.MX_GROUPS_M,
+                                     plan.combine_destinations(y_base, N), ex.M_recv, N, K, ex.m_cap_recv)
 
 
 def expert_forward(rq, rs, wq, wsf, plan: ExchangePlan):
@@ -251,23 +275,29 @@ def dispatch_bf16(t, plan: ExchangePlan, a2a):
     return out
 
 
-def expert_backward(dy_recv, rq, rs, wq, wsd, plan: ExchangePlan):
+def expert_backward(dy_recv, rq, rs, wq, wsd, plan: ExchangePlan, dx_rows=None):
     """(dx_recv [M_recv, K], dw [E, N, K]) of the received groups.
 
     dX = dY W_e (dY cast rowwise along N, W's forward codes read MN-major);
     dW_e = sum over the groups of expert e of dY_g^T X_g, both cast columnwise
-    per group, X from the received codes dequantized to bf16."""
+    per group, X from the received codes dequantized to bf16. With dx_rows
+    (one device address per received group: where its dX rows go, e.g. into
+    the senders' buffers) dX is stored there and dx_recv is None."""
     E, N, K = wq.shape
     dev = dy_recv.device
     dw = torch.empty(E, N, K, dtype=torch.bfloat16, device=dev)
-    dx = torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
+    dx = None if dx_rows is not None else torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
     if plan.M_recv == 0:
         dw.zero_()
         return dx, dw
     offs = torch.as_tensor(plan.offs_recv(), device=dev)
     G, cap = plan.G_recv, plan.m_cap_recv
     dq, ds, dqt, dst = mx.cast_2d_grouped(dy_recv, offs, cap)
-    mx.mx_grouped_mm_experts(dq, ds, wq, wsd, offs, G, E, mx.MX_GROUPS_M_KN, dx, plan.M_recv, K, N, cap)
+    if dx_rows is not None:
+        mx.mx_grouped_mm_experts_to_rows(dq, ds, wq, wsd, offs, G, E, mx.MX_GROUPS_M_KN, dx_rows, plan.M_recv, K, N,
+                                         cap)
+    else:
+        mx.mx_grouped_mm_experts(dq, ds, wq, wsd, offs, G, E, mx.MX_GROUPS_M_KN, dx, plan.M_recv, K, N, cap)
     x_deq = torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
     mx.mx_dequant_dim0_grouped(rq, rs.reshape(-1), offs, plan.M_recv, K, cap, x_deq)
     xqt, xst = mx.cast_dim1_grouped(x_deq, offs, cap)
@@ -290,15 +320,18 @@ class MXFP8ExpertParallelMM:
     backward(dy [M, N]) -> (dx [M, K], dw [E, N, K]). `a2a` defaults to
     torch.distributed.all_to_all_single over `group`.
 
-    direct=True dispatches with one kernel instead of a cast and an
-    all-to-all: the receive buffers are symmetric memory (every rank's buffer
-    mapped into every rank), each rank's cast writes its groups straight into
-    them with plain stores (no TMA, no multicast), and an all-reduce of one
-    element, ordered on the stream after the cast, is the barrier before the
-    expert GEMMs read. The buffer is kept and grown (collectively, on every
-    rank at once) when the largest receiver needs more rows; the backward
-    reads it, so a second forward of the same layer before its backward is
-    refused."""
+    direct=True fuses the exchanges into the kernels: the dispatch is the
+    rowwise cast storing each tile straight into the receiving rank's buffer,
+    and the combine (and, in backward, the return of dX) is the expert GEMM's
+    epilogue storing each output row straight into the rank that sent the
+    token. The buffers are symmetric memory (every rank's mapped into every
+    rank) written with plain stores (no TMA, no multicast); a one-element
+    all-reduce, ordered on the stream after each such kernel, is the barrier
+    before anyone reads. The buffers are kept and grown collectively (every
+    rank computes the same sizes from the gathered counts); outputs are
+    copied out of them, and the received codes the backward reads stay in
+    them, so a second forward of the same layer before its backward is
+    refused. dY still goes to the experts by a bf16 all-to-all."""
 
     def __init__(self, group=None, a2a=None, direct=False, all_gather=None):
         import torch.distributed as dist
@@ -308,40 +341,62 @@ class MXFP8ExpertParallelMM:
         self.a2a = a2a if a2a is not None else dist_all_to_all(group)
         self.direct = direct
         self.all_gather = all_gather if all_gather is not None else (dist_all_gather(group) if direct else None)
-        self._recv = None            # direct mode: (buffer, handle, rows, K)
+        self._symm_bufs = {}          # direct mode: name -> (buffer, handle, bytes)
         self._saved = None
 
-    def _receive_buffers(self, rows: int, K: int, device):
-        """(codes base, scale base) of every rank's symmetric receive buffer,
-        holding at least `rows` padded rows; collective when it (re)allocates
-        (every rank computes the same `rows` from the gathered counts)."""
-        if self._recv is None or self._recv[2] < rows or self._recv[3] != K:
+    def _symm(self, name: str, nbytes: int, device):
+        """A symmetric-memory byte buffer of at least nbytes and every rank's
+        address of it; (re)allocated collectively when it must grow."""
+        cur = self._symm_bufs.get(name)
+        if cur is None or cur[2] < nbytes:
             import torch.distributed as dist
             import torch.distributed._symmetric_memory as symm_mem
-            cap = max(_pad(rows), BLOCK_ROWS)
-            band = scale_band_bytes(K)
-            buf = symm_mem.empty(cap * K + cap // BLOCK_ROWS * band, dtype=torch.uint8, device=device)
+            size = max(int(nbytes), 512)
+            buf = symm_mem.empty(size, dtype=torch.uint8, device=device)
             grp = self.group if self.group is not None else dist.group.WORLD
-            hdl = symm_mem.rendezvous(buf, grp.group_name)
-            self._recv = (buf, hdl, cap, K)
-        buf, hdl, cap, K = self._recv
-        base_q = [int(p) for p in hdl.buffer_ptrs]
-        return base_q, [b + cap * K for b in base_q]
+            cur = (buf, symm_mem.rendezvous(buf, grp.group_name), size)
+            self._symm_bufs[name] = cur
+        return cur[0], [int(p) for p in cur[1].buffer_ptrs]
 
-    def _dispatch_direct(self, x, send_counts, E):
+    def _barrier(self, device):
         import torch.distributed as dist
-        K = x.shape[1]
-        counts = gather_counts(send_counts, self.W, self.all_gather, x.device)
-        plan = DirectPlan(self.W, E, self.rank, counts)
-        base_q, base_s = self._receive_buffers(int(plan.recv_rows_of.max()) if self.W else 0, K, x.device)
-        dispatch_mxfp8_direct(x, plan, base_q, base_s)
-        flag = torch.zeros(1, dtype=torch.float32, device=x.device)
+        flag = torch.zeros(1, dtype=torch.float32, device=device)
         dist.all_reduce(flag, group=self.group)      # every rank's stores are in before anyone reads
+
+    def _forward_direct(self, x, send_counts, w):
+        E, N, K = w.shape
+        dev = x.device
+        counts = gather_counts(send_counts, self.W, self.all_gather, dev)
+        plan = DirectPlan(self.W, E, self.rank, counts)
         ex = plan.exchange
-        buf, _, cap, _ = self._recv
-        rq = buf[:ex.m_cap_recv * K].view(ex.m_cap_recv, K)
-        rs = buf[cap * K:cap * K + ex.m_cap_recv // BLOCK_ROWS * scale_band_bytes(K)].view(-1, scale_band_bytes(K))
-        return ex, rq, rs
+        rows = int(plan.recv_rows_of.max())
+        band = scale_band_bytes(K)
+        rbuf, rbase = self._symm("recv", rows * K + rows // BLOCK_ROWS * band, dev)
+        dispatch_mxfp8_direct(x, plan, rbase, [b + rows * K for b in rbase])
+        self._barrier(dev)
+        rq = rbuf[:ex.m_cap_recv * K].view(ex.m_cap_recv, K)
+        rs = rbuf[rows * K:rows * K + ex.m_cap_recv // BLOCK_ROWS * band].view(-1, band)
+        wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
+        m_max = int(counts.sum(axis=1).max())
+        ybuf, ybase = self._symm("y", m_max * N * 2, dev)
+        expert_forward_to_senders(rq, rs, wq, wsf, plan, ybase)
+        self._barrier(dev)
+        y = ybuf[:ex.M * N * 2].view(torch.bfloat16).view(ex.M, N).clone()
+        self._saved = (plan, rq, rs, wq, wsd)
+        return y
+
+    def _backward_direct(self, dy):
+        plan, rq, rs, wq, wsd = self._saved
+        self._saved = None
+        ex = plan.exchange
+        E, N, K = wq.shape
+        dev = dy.device
+        dy_recv = dispatch_bf16(dy.contiguous(), ex, self.a2a)
+        m_max = int(plan.counts.sum(axis=1).max())
+        dxbuf, dxbase = self._symm("dx", m_max * K * 2, dev)
+        _, dw = expert_backward(dy_recv, rq, rs, wq, wsd, ex, dx_rows=plan.combine_destinations(dxbase, K))
+        self._barrier(dev)
+        return dxbuf[:ex.M * K * 2].view(torch.bfloat16).view(ex.M, K).clone(), dw
 
     def forward(self, x, send_counts, w):
         for name, t in (("x", x), ("w", w)):
@@ -353,14 +408,13 @@ class MXFP8ExpertParallelMM:
             raise ValueError("send_counts must sum to the number of tokens")
         if self.direct:
             if self._saved is not None:
-                raise RuntimeError("direct dispatch: the previous forward's backward has not run (its "
+                raise RuntimeError("direct mode: the previous forward's backward has not run (its "
                                    "receive buffer would be overwritten)")
-            plan, rq, rs = self._dispatch_direct(x, send_counts, E)
-        else:
-            recv = exchange_counts(send_counts, self.W, E, self.a2a, x.device)
-            plan = ExchangePlan(self.W, E, send_counts, recv)
-            q, s = pack_mxfp8(x, plan)
-            rq, rs = dispatch_mxfp8(q, s, plan, self.a2a)
+            return self._forward_direct(x, send_counts, w)
+        recv = exchange_counts(send_counts, self.W, E, self.a2a, x.device)
+        plan = ExchangePlan(self.W, E, send_counts, recv)
+        q, s = pack_mxfp8(x, plan)
+        rq, rs = dispatch_mxfp8(q, s, plan, self.a2a)
         wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
         y = combine(expert_forward(rq, rs, wq, wsf, plan), plan, self.a2a)
         self._saved = (plan, rq, rs, wq, wsd)
@@ -371,6 +425,8 @@ class MXFP8ExpertParallelMM:
             raise RuntimeError("backward before forward")
         if dy.dtype != torch.bfloat16:
             raise TypeError("MXFP8ExpertParallelMM takes a bf16 gradient")
+        if self.direct:
+            return self._backward_direct(dy)
         plan, rq, rs, wq, wsd = self._saved
         self._saved = None
         dy_recv = dispatch_bf16(dy.contiguous(), plan, self.a2a)

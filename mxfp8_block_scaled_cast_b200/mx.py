@@ -39,6 +39,8 @@ _SIGNATURES = {
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
     "mx_grouped_mm_experts": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                              _i64, _vp]),
+    "mx_grouped_mm_experts_to_rows": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                                     ctypes.POINTER(_vp), _i64, _i64, _i64, _i64, _vp]),
     "mx_wcache_create": (_vp, []),
     "mx_wcache_evict": (None, [_vp, _vp]),
     "mx_wcache_clear": (None, [_vp]),
@@ -201,6 +203,16 @@ def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream
 
 def mx_grouped_mm_experts(a_q, a_s, b_q, b_s, offs, G, E, mode, out, M, N, K, m_cap, stream=None):
     _call("mx_grouped_mm_experts", _p(a_q), _p(a_s), _p(b_q), _p(b_s), _p(offs), G, E, mode, _p(out), M, N, K,
+          m_cap, _stream(stream))
+
+
+def mx_grouped_mm_experts_to_rows(a_q, a_s, b_q, b_s, offs, G, E, mode, out_rows, M, N, K, m_cap, stream=None):
+    """M-group GEMM with group g's output rows at device address out_rows[g] (a
+    list of G integers, which may be peer-mapped addresses)."""
+    if len(out_rows) != G:
+        raise ValueError("one output destination per group")
+    arr = (_vp * G)(*[int(v) for v in out_rows])
+    _call("mx_grouped_mm_experts_to_rows", _p(a_q), _p(a_s), _p(b_q), _p(b_s), _p(offs), G, E, mode, arr, M, N, K,
           m_cap, _stream(stream))
 
 

@@ -100,5 +100,12 @@ def test_host_argument_checks_return_before_any_launch():
                                           two(0x100000, 0x100000), None) == 1   # null destination
     assert L.mx_cast_dim0_grouped_scatter(ok16, 64, 64, ok16, 2, 256, two(0x100000, 0x100008),
                                           two(0x100000, 0x100000), None) == 2   # misaligned destination
+    # the GEMM with per-group output rows: M-group modes only, every destination checked
+    assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, ok16, 2, 2, 1, two(0x100000, 0x100000),
+                                           128, 256, 128, 256, None) == 1    # K-groups mode
+    assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, None, 1, 1, 0, two(0x100000, 0x100000),
+                                           128, 256, 128, 256, None) == 1    # no offsets
+    assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, ok16, 2, 2, 0, two(0x100000, 0x100004),
+                                           128, 256, 128, 256, None) == 2    # misaligned destination
     msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
     assert b"not a multiple of 32" in msg

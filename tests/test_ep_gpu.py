@@ -223,3 +223,43 @@ def test_module_direct_over_a_one_rank_nccl_group(mx):
         del layer
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("W,E,N,K", [(2, 3, 256, 576), (4, 2, 576, 256)])
+def test_fused_combine_equals_the_all_to_all(mx, W, E, N, K):
+    """The combine fused into the expert GEMMs (each output row, and in backward
+    each dX row, stored straight into the sender's buffer), ranks emulated with
+    local buffers: bitwise the outputs of the all-to-all path."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    rng = np.random.default_rng(80 + W)
+    counts = rng.integers(0, 260, size=(W, W * E))
+    counts[1, 0] = 0
+    xs = [S.normal_bf16((int(counts[r].sum()), K), seed=90 + r).cuda() for r in range(W)]
+    ws = [S.normal_bf16((E, N, K), 0.02, seed=100 + r).cuda() for r in range(W)]
+    dys = [S.normal_bf16((int(counts[r].sum()), N), 0.1, seed=110 + r).cuda() for r in range(W)]
+    plans = [ep.ExchangePlan(W, E, counts[r], counts[:, r * E:(r + 1) * E]) for r in range(W)]
+    dplans = [ep.DirectPlan(W, E, r, counts) for r in range(W)]
+    packed = [ep.pack_mxfp8(xs[r], plans[r]) for r in range(W)]
+    rq = _virtual_a2a([p[0] for p in packed], [pl.send_rows for pl in plans], [pl.recv_rows for pl in plans])
+    rs = _virtual_a2a([p[1] for p in packed], [pl.send_rows // 128 for pl in plans],
+                      [pl.recv_rows // 128 for pl in plans])
+    wc = [mx.cast_w32x32(w, transposed=False, dgrad_scales=True) for w in ws]
+    # the all-to-all path
+    y_recv = [ep.expert_forward(rq[r], rs[r], wc[r][0], wc[r][1], plans[r]) for r in range(W)]
+    ys = _virtual_a2a(y_recv, [pl.recv_tokens for pl in plans], [pl.send_tokens for pl in plans])
+    dy_recv = _virtual_a2a(dys, [pl.send_tokens for pl in plans], [pl.recv_tokens for pl in plans])
+    back = [ep.expert_backward(dy_recv[r], rq[r], rs[r], wc[r][0], wc[r][3], plans[r]) for r in range(W)]
+    dxs = _virtual_a2a([b[0] for b in back], [pl.recv_tokens for pl in plans], [pl.send_tokens for pl in plans])
+    # fused: every expert rank stores into every sender's buffers (NaN-filled first)
+    nan = lambda *sh: torch.full(sh, float("nan"), dtype=torch.bfloat16, device="cuda")
+    ybuf = [nan(int(counts[s].sum()), N) for s in range(W)]
+    dxbuf = [nan(int(counts[s].sum()), K) for s in range(W)]
+    for r in range(W):
+        ep.expert_forward_to_senders(rq[r], rs[r], wc[r][0], wc[r][1], dplans[r], [b.data_ptr() for b in ybuf])
+        none, dw = ep.expert_backward(dy_recv[r], rq[r], rs[r], wc[r][0], wc[r][3], plans[r],
+                                      dx_rows=dplans[r].combine_destinations([b.data_ptr() for b in dxbuf], K))
+        assert none is None and torch.equal(dw, back[r][1]), f"dW of rank {r}"
+    mx.mx_device_error()
+    for s in range(W):
+        assert torch.equal(ybuf[s], ys[s]), f"outputs of rank {s}"
+        assert torch.equal(dxbuf[s], dxs[s]), f"dX of rank {s}"

@@ -191,3 +191,29 @@ def test_scatter_cast_stays_in_bounds(mx):
         x = _x(int(counts[r].sum()), K, 30 + r)
         ep.dispatch_mxfp8_direct(x, plans[r], [b.data_ptr() for b in bq], [b.data_ptr() for b in bs])
     g.check(mx, "scatter cast")
+
+
+def test_gemm_to_sender_rows_stays_in_bounds(mx):
+    """The expert GEMMs with the combine fused: outputs and dX rows stored into
+    every sender's (guarded) buffer, ranks emulated."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    W, E, N, K = 2, 2, 96, 160
+    rng = np.random.default_rng(6)
+    counts = rng.integers(0, 300, size=(W, W * E))
+    counts[0, 1] = 0
+    g = Guarded()
+    ybuf = [g.bf16(int(counts[s].sum()), N) for s in range(W)]
+    dxbuf = [g.bf16(int(counts[s].sum()), K) for s in range(W)]
+    for r in range(W):
+        dp = ep.DirectPlan(W, E, r, counts)
+        ex = dp.exchange
+        x = S.normal_bf16((ex.M_recv, K), seed=r).cuda()
+        dy = S.normal_bf16((ex.M_recv, N), 0.1, seed=10 + r).cuda()
+        w = S.normal_bf16((E, N, K), 0.02, seed=20 + r).cuda()
+        offs = torch.as_tensor(ex.offs_recv()).cuda()
+        rq, rs = mx.cast_dim0_grouped(x, offs, ex.m_cap_recv)
+        rs = rs.view(ex.m_cap_recv // 128, ep.scale_band_bytes(K))
+        wq, wsf, _, wsd = mx.cast_w32x32(w, transposed=False, dgrad_scales=True)
+        ep.expert_forward_to_senders(rq, rs, wq, wsf, dp, [b.data_ptr() for b in ybuf])
+        ep.expert_backward(dy, rq, rs, wq, wsd, ex, dx_rows=dp.combine_destinations([b.data_ptr() for b in dxbuf], K))
+    g.check(mx, "GEMM rows to senders")
