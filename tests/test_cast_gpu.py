@@ -276,6 +276,39 @@ def test_square_sweep_full_size_sampled(mx, n):
     assert np.array_equal(_np(q1[:, band * 32:(band + 1) * 32]), eqt)
 
 
+@pytest.mark.parametrize("n", [1024, 4096, 8192, 16384])
+def test_sweep_every_mode_in_the_benchmark_launch(mx, n):
+    """Every mode of the bandwidth sweep at every square size, in the launch the
+    benchmark times: dim0 rows and dim1 32-row bands against the oracle (all of
+    them at 1024^2, sampled above), the fused cast bitwise equal to the two, and
+    sampled 32x32 tiles of the weight cast with both of its scale views."""
+    xb = S.sweep_tensor((n, n), seed=11, device="cuda")
+    rng = np.random.default_rng(n + 1)
+    full = n <= 1024
+    q0, s0 = mx.cast_dim0(xb)
+    rows = np.arange(n) if full else np.sort(rng.choice(n, 16, replace=False))
+    _sample_rows_check_dim0(q0, s0, xb, n, rows)
+    q1, s1 = mx.cast_dim1(xb)
+    s1b, cc = _np(s1), np.arange(n)
+    for band in (range(n // 32) if full else rng.choice(n // 32, 2, replace=False)):
+        eqt, est = O.cast_dim1(S.bf16_bits(xb[band * 32:(band + 1) * 32]))
+        assert np.array_equal(_np(q1[:, band * 32:(band + 1) * 32]), eqt), f"dim1 band {band}"
+        assert np.array_equal(s1b[O.blocked_offset(cc, np.full(n, band), n // 32)], est[:, 0])
+    q, s, qt, st = mx.cast_2d(xb)
+    assert torch.equal(q, q0) and torch.equal(s, s0) and torch.equal(qt, q1) and torch.equal(st, s1)
+    del q, s, qt, st, q0, s0, q1, s1
+    wq, wsf, wqt, wsd = mx.cast_w32x32(xb)
+    sfb, sdb = _np(wsf), _np(wsd)
+    for _ in range(16):
+        i, j = int(rng.integers(n // 32)), int(rng.integers(n // 32))
+        eq, st32 = O.cast_32x32(S.bf16_bits(xb[32 * i:32 * i + 32, 32 * j:32 * j + 32]))
+        assert np.array_equal(_np(wq[32 * i:32 * i + 32, 32 * j:32 * j + 32]), eq), f"32x32 tile {i},{j}"
+        assert np.array_equal(_np(wqt[32 * j:32 * j + 32, 32 * i:32 * i + 32]), eq.T)
+        idx = np.arange(32)
+        assert np.all(sfb[O.blocked_offset(32 * i + idx, j, n // 32)] == st32[0, 0])
+        assert np.all(sdb[O.blocked_offset(32 * j + idx, i, n // 32)] == st32[0, 0])
+
+
 def test_expert_stack_full_size_sampled(mx):
     """[64, 2048, 7168] expert weight stack, 32x32 cast, sampled tiles."""
     G, N, K = 64, 2048, 7168
