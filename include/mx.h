@@ -250,8 +250,11 @@ MX_API mx_status mx_grouped_mm_experts(const void* a_q, const void* a_s, const v
  * of a bf16 all-to-all afterwards. out_rows is a HOST array of G device
  * pointers, each non-NULL and 16-byte aligned (checked on the host; an empty
  * group's destination is never written); a destination may be another GPU's
- * memory mapped into this process (plain stores). The other arguments and
- * the bytes per row are those of mx_grouped_mm_experts. */
+ * memory mapped into this process (plain stores, no TMA). Bytes written per
+ * group: size_g rows of N bf16; nothing else is written. The kernel ends with
+ * a system-scope fence: once it is seen complete (e.g. through a collective
+ * issued after it on the same stream), other GPUs read the rows. The other
+ * arguments are those of mx_grouped_mm_experts. */
 MX_API mx_status mx_grouped_mm_experts_to_rows(const void* a_q, const void* a_s, const void* b_q,
                                                const void* b_s, const int32_t* offs, int32_t G, int32_t E,
                                                int32_t mode, void* const* out_rows, int64_t M, int64_t N,
