@@ -618,6 +618,95 @@ def unaligned_bench(mx, device, flush, peaks):
     return out
 
 
+def ep_fused_kernels(mx, device, flush, peaks, W=8, tokens=16384, K=4096, N=4096, seed=0, rounds=4):
+    """What fusing the expert-parallel exchange into the kernels costs the kernels,
+    on one GPU (prime-rl PR #3388, Overview: enable_a2a; ao PR #4705, the
+    expert-parallel pipeline benchmark). W ranks of one expert each, `tokens` per
+    rank spread evenly over the W experts; rank 0's view:
+      dispatch  its tokens cast rowwise into the W receiving ranks' buffers (the
+                scatter cast) against the same grouped cast into one send buffer;
+      combine   its expert GEMM over the groups received from the W senders,
+                storing each output row into its sender's buffer, against the
+                same GEMM into one output.
+    Local buffers stand in for the peers' mapped buffers, so the NVLink transfer
+    is not in these numbers (every run here has one GPU). Casts are timed
+    in-stream after an L2 flush, GEMMs as CUDA-graph replays; each pair
+    alternates over `rounds` rounds, median per variant. Both forms of each
+    write the same bytes (checked)."""
+    import numpy as np
+    import torch
+    from mxfp8_block_scaled_cast_b200 import ep, synthetic as S
+    E = 1
+    rng = np.random.default_rng(seed)
+    counts = np.stack([rng.multinomial(tokens, np.full(W * E, 1.0 / (W * E))) for _ in range(W)])
+    plan = ep.DirectPlan(W, E, 0, counts)
+    ex = plan.exchange
+    band = ep.scale_band_bytes(K)
+    u8 = lambda n: torch.empty(int(n), dtype=torch.uint8, device=device)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    med = lambda v: sorted(v)[len(v) // 2]
+
+    # ---- dispatch ----
+    x = S.normal_bf16((ex.M, K), seed=seed, device=device)
+    offs_s = torch.as_tensor(ex.offs_send(), device=device)
+    recv_q = [u8(plan.recv_rows_of[d] * K) for d in range(W)]
+    recv_s = [u8(plan.recv_rows_of[d] // 128 * band) for d in range(W)]
+    dst_q, dst_s = plan.destinations([b.data_ptr() for b in recv_q], [b.data_ptr() for b in recv_s], K)
+    one_q, one_s = u8(ex.m_cap_send * K), u8(ex.m_cap_send // 128 * band)
+    cast_one = lambda: mx.mx_cast_dim0_grouped(x, offs_s, ex.m_cap_send, one_q, one_s)
+    cast_scatter = lambda: mx.mx_cast_dim0_grouped_scatter(x, offs_s, ex.m_cap_send, dst_q, dst_s)
+    t = {"one": [], "scatter": []}
+    for r in range(rounds):
+        for k in (("one", "scatter") if r % 2 == 0 else ("scatter", "one")):
+            t[k].append(flushed_time(cast_one if k == "one" else cast_scatter, flush, reps=5, pairs=20, runs=7)[1])
+    nbytes = ex.M * K * 2 + ex.m_cap_send * K + ex.m_cap_send // 128 * band
+    pads = [ep._pad(c) for c in counts[0]]
+    starts = np.concatenate([[0], np.cumsum(pads)[:-1]])
+    same_cast = all(
+        torch.equal(one_q[int(starts[d]) * K:int(starts[d] + pads[d]) * K],
+                    recv_q[d][int(plan.dst_row[d]) * K:int(plan.dst_row[d] + pads[d]) * K]) and
+        torch.equal(one_s[int(starts[d]) // 128 * band:int(starts[d] + pads[d]) // 128 * band],
+                    recv_s[d][int(plan.dst_row[d]) // 128 * band:int(plan.dst_row[d] + pads[d]) // 128 * band])
+        for d in range(W))
+    rate = lambda sec: {"gbs": round(nbytes / sec / 1e9, 1), "frac_of_measured_hbm": round(nbytes / sec / 1e9 / hbm, 3)}
+    dispatch = {"bytes_per_launch": nbytes, "one_buffer": rate(med(t["one"])),
+                "scattered_to_ranks": rate(med(t["scatter"])),
+                "scattered_over_one": round(med(t["one"]) / med(t["scatter"]), 4), "same_bytes": same_cast}
+    del x, recv_q, recv_s, one_q, one_s
+
+    # ---- combine ----
+    M_recv, cap, G = ex.M_recv, ex.m_cap_recv, ex.G_recv
+    offs_r = torch.as_tensor(ex.offs_recv(), device=device)
+    rq, rs = mx.cast_dim0_grouped(S.normal_bf16((M_recv, K), seed=seed + 1, device=device), offs_r, cap)
+    wq, wsf, _, _ = mx.cast_w32x32(S.normal_bf16((E, N, K), 0.02, seed=seed + 2, device=device), transposed=False)
+    y_one = torch.empty(M_recv, N, dtype=torch.bfloat16, device=device)
+    y_send = [torch.empty(int(counts[s_].sum()), N, dtype=torch.bfloat16, device=device) for s_ in range(W)]
+    rows = plan.combine_destinations([b.data_ptr() for b in y_send], N)
+    gemm_one = lambda: mx.mx_grouped_mm_experts(rq, rs, wq, wsf, offs_r, G, E, mx.MX_GROUPS_M, y_one, M_recv, N, K,
+                                                cap)
+    gemm_rows = lambda: mx.mx_grouped_mm_experts_to_rows(rq, rs, wq, wsf, offs_r, G, E, mx.MX_GROUPS_M, rows,
+                                                         M_recv, N, K, cap)
+    t = {"one": [], "rows": []}
+    for r in range(rounds):
+        for k in (("one", "rows") if r % 2 == 0 else ("rows", "one")):
+            t[k].append(graph_time(gemm_one if k == "one" else gemm_rows, iters=20, runs=5))
+    mx.mx_device_error()
+    ends = np.cumsum(counts[:, 0])
+    same_gemm = all(torch.equal(y_one[int(ends[s_] - counts[s_, 0]):int(ends[s_])], y_send[s_][:int(counts[s_, 0])])
+                    for s_ in range(W))
+    flops = 2 * M_recv * N * K
+    combine = {"flops_per_launch": flops,
+               "one_output_tflops": round(flops / med(t["one"]) / 1e12, 1),
+               "rows_to_senders_tflops": round(flops / med(t["rows"]) / 1e12, 1),
+               "rows_over_one": round(med(t["one"]) / med(t["rows"]), 4), "same_bytes": same_gemm}
+    del rq, rs, wq, wsf, y_one, y_send
+    torch.cuda.empty_cache()
+    return {"ranks_emulated": W, "experts_per_rank": E, "tokens_per_rank": tokens, "K": K, "N": N,
+            "method": "local buffers stand in for the peers' mapped buffers (NVLink not measured: one GPU); casts "
+                      "in-stream after an L2 flush, GEMMs as CUDA-graph replays, the two forms alternating",
+            "dispatch": dispatch, "combine": combine}
+
+
 def kva_gemms(mx, device, peaks, Mk=16384, Nk=576, Kk=7168):
     """The GEMMs around the 576-wide output gradient (torchtitan PR #5334, review
     thread: the KV-A projection, y [16384, 576] = x [16384, 7168] w [576, 7168]^T):
@@ -892,6 +981,8 @@ def main(argv=None):
     p.add_argument("--no-arms", action="store_true", help="skip timing the backward-override arms")
     p.add_argument("--no-linear", action="store_true", help="skip timing the MXFP8 linear")
     p.add_argument("--no-gemm-only", action="store_true", help="skip the graph-replayed GEMM-only timing")
+    p.add_argument("--no-ep", action="store_true",
+                   help="skip timing the expert-parallel exchange fused into the kernels (ranks emulated)")
     p.add_argument("--no-library", action="store_true",
                    help="skip the interleaved comparisons with library GEMMs (cuBLASLt MXFP8, torch bf16 grouped)")
     p.add_argument("--no-unaligned", action="store_true",
@@ -1052,6 +1143,11 @@ def main(argv=None):
     if not args.no_arms:
         flush = L2Flush(dev)
         arms = override_arms(mx, step, flush, peaks)
+    ep_fused = None
+    if not args.no_ep and world == 1:      # ranks emulated on one GPU: context, single-GPU runs only
+        flush = L2Flush(dev)
+        ep_fused = ep_fused_kernels(mx, dev, flush, peaks)
+        del flush
 
     if rank != 0:
         if world > 1:
@@ -1082,6 +1178,7 @@ def main(argv=None):
         "library_mxfp8_cublaslt": library,
         "library_bf16_grouped_mm": library_hp,
         "unaligned": unaligned,
+        "ep_fused_kernels": ep_fused,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

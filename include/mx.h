@@ -175,9 +175,10 @@ MX_API mx_status mx_cast_2d_grouped(const void* x, int64_t M, int64_t K,
  * Every pointer must be non-NULL and 16-byte aligned (checked on the host;
  * an empty group's destination is never written). Bytes written per group
  * are exactly those its rows occupy in mx_cast_dim0_grouped's outputs; the
- * pad capacity past the last group writes nothing. The kernel ends with a
- * system-scope fence: once it is seen complete (e.g. through a collective
- * issued after it on the same stream), other GPUs read the stores. */
+ * pad capacity past the last group writes nothing. The call ends with a
+ * system-scope fence (a one-thread kernel after the cast, on the same
+ * stream): once that is seen complete (e.g. through a collective issued
+ * after the call on the same stream), other GPUs read the stores. */
 MX_API mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t K,
                                               const int32_t* offs, int32_t G, int64_t m_cap,
                                               void* const* dst_q, void* const* dst_s, void* stream);

@@ -325,8 +325,15 @@ cast_scatter_kernel(const __grid_constant__ CastArgs a, const __grid_constant__ 
   __shared__ __align__(16) uint8_t s_row[512];
   __shared__ __align__(16) uint8_t s_col[512];
   cast_tile<kModeRow, true, true>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col, &d);
-  __threadfence_system();
 }
+
+// One system-scope fence issued after a kernel that stored to other GPUs'
+// memory, on the same stream: every store of that kernel precedes it in stream
+// order, so one fence for the whole launch replaces a fence in every CTA (which
+// holds each CTA until its own stores are visible system-wide: measured 0.49x
+// the throughput of the same cast into one local buffer, against 0.86x with
+// this launch after it).
+__global__ void system_fence_kernel() { __threadfence_system(); }
 
 // Up to three independent dense casts in one launch (the linear's weight and
 // activation casts): CTAs [0, n0) take cast 0's tiles, the next n1 cast 1's,

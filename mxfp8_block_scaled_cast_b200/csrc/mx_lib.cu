@@ -522,7 +522,9 @@ mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t K, cons
   a.G = G;
   cast_scatter_kernel<<<dim3(unsigned(col_tiles), unsigned(row_tiles), 1u), kWarpCastThreads, kWarpCastSmem,
                         static_cast<cudaStream_t>(stream)>>>(a, d);
-  return cuda_check("scatter cast launch");
+  MX_TRY(cuda_check("scatter cast launch"));
+  system_fence_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_check("fence launch");
 }
 
 mx_status mx_cast_dim1_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
