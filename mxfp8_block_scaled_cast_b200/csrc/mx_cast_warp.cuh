@@ -315,9 +315,9 @@ cast_warp_kernel(const CastArgs a) {
 // The grouped rowwise cast with each group's padded rows written to its own
 // destination (prime-rl PR #3388, Overview: enable_a2a, the MXFP8 dispatch of
 // expert parallelism): the cast and the token exchange in one kernel, each
-// tile stored straight into the receiving rank's buffer. Ends with a
-// system-scope fence so that the stores to peer memory are visible to the
-// other GPUs once this kernel is seen complete.
+// tile stored straight into the receiving rank's buffer. The host follows it
+// with system_fence_kernel on the same stream, so that the stores to peer
+// memory are visible to the other GPUs once that launch is seen complete.
 __global__ void __launch_bounds__(kWarpCastThreads)
 cast_scatter_kernel(const __grid_constant__ CastArgs a, const __grid_constant__ ScatterDests d) {
   extern __shared__ __align__(128) uint8_t wsmem[];
