@@ -216,6 +216,17 @@ def test_module_direct_over_a_one_rank_nccl_group(mx):
             dx, dw = layer.backward(dy)
             mx.mx_device_error()
             assert torch.equal(y, y0) and torch.equal(dx, dx0) and torch.equal(dw, dw0)
+        # a larger step (the symmetric buffers are regrown collectively), then a
+        # smaller one (buffers larger than needed): still bitwise the all-to-all layer
+        for step_counts, seed in ((np.array([300, 129, 513, 7]), 60), (np.array([0, 40, 0, 33]), 70)):
+            xs = S.normal_bf16((int(step_counts.sum()), K), seed=seed).cuda()
+            dys = S.normal_bf16((int(step_counts.sum()), N), 0.1, seed=seed + 1).cuda()
+            y_ref = ref.forward(xs, step_counts, w)
+            dx_ref, dw_ref = ref.backward(dys)
+            y = layer.forward(xs, step_counts, w)
+            dx, dw = layer.backward(dys)
+            mx.mx_device_error()
+            assert torch.equal(y, y_ref) and torch.equal(dx, dx_ref) and torch.equal(dw, dw_ref), step_counts
         layer.forward(x, counts, w)
         with pytest.raises(RuntimeError):
             layer.forward(x, counts, w)
