@@ -160,11 +160,12 @@ def test_module_over_a_one_rank_nccl_group(mx):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("W,E,K", [(2, 3, 576), (4, 2, 256), (3, 1, 96)])
+@pytest.mark.parametrize("W,E,K", [(2, 3, 576), (4, 2, 256), (3, 1, 96), (9, 8, 64)])
 def test_direct_dispatch_equals_the_all_to_all(mx, W, E, K):
     """The dispatch as one kernel (every rank's cast storing straight into every
     receive buffer), ranks emulated in one process with local buffers: each
-    receive buffer is bitwise what the cast + all-to-all path delivers."""
+    receive buffer is bitwise what the cast + all-to-all path delivers (up to
+    W*E = 72 groups, destinations in nine buffers)."""
     from mxfp8_block_scaled_cast_b200 import ep
     rng = np.random.default_rng(60 + W)
     counts = rng.integers(0, 260, size=(W, W * E))
