@@ -66,3 +66,48 @@ def test_step_captured_once_replays_under_new_routing(mx, arm):
         for g in np.flatnonzero(np.asarray(ROUTINGS[i]) == 0):
             assert not outs[2][g].any(), f"dW of empty group {g} must be exact zeros"
     del graph
+
+
+def test_linear_captured_once_replays_new_inputs(mx):
+    """The linear forward and backward without the weight cache (the cache decides
+    hit or miss on the host, once, at capture), with its workspace: one capture,
+    replays on new x, w and dy bitwise equal to eager calls. Sizes off the GEMM
+    tile (N = 96, K = 576) take the pad path."""
+    Ml, Nl, Kl = 256, 96, 576
+    x = torch.empty(Ml, Kl, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(Nl, Kl, dtype=torch.bfloat16, device="cuda")
+    dy = torch.empty(Ml, Nl, dtype=torch.bfloat16, device="cuda")
+    ws = mx.linear_workspace(Ml, Nl, Kl)
+    outs = [torch.empty(Ml, Nl, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(Ml, Kl, dtype=torch.bfloat16, device="cuda"),
+            torch.empty(Nl, Kl, dtype=torch.bfloat16, device="cuda")]
+
+    def load(i):
+        x.copy_(S.normal_bf16((Ml, Kl), seed=30 + i, device="cuda"))
+        w.copy_(S.normal_bf16((Nl, Kl), 0.02, seed=40 + i, device="cuda"))
+        dy.copy_(S.normal_bf16((Ml, Nl), 0.1, seed=50 + i, device="cuda"))
+
+    def step(y, dx, dw):
+        mx.mx_linear_fwd(x, w, None, 0, y, ws)
+        mx.mx_linear_bwd(dy, x, w, None, 0, dx, dw, ws)
+
+    load(0)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(*outs)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(*outs)
+    refs = [torch.empty_like(o) for o in outs]
+    for i in range(3):
+        load(i)
+        graph.replay()
+        torch.cuda.synchronize()
+        step(*refs)
+        torch.cuda.synchronize()
+        mx.mx_device_error()
+        for name, got, want in zip(("y", "dx", "dw"), outs, refs):
+            assert torch.equal(got, want), f"linear {name}, inputs {i}"
+    del graph
