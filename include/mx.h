@@ -183,6 +183,33 @@ MX_API mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t 
                                               const int32_t* offs, int32_t G, int64_t m_cap,
                                               void* const* dst_q, void* const* dst_s, void* stream);
 
+/* The fused grouped cast (rowwise and columnwise from one read, as
+ * mx_cast_2d_grouped) with each group's outputs written to its own
+ * destination: the backward dispatch of expert parallelism (prime-rl PR
+ * #3388, Overview: enable_a2a), each token group's gradient cast both ways
+ * straight into the buffers of the rank that holds its expert, exactly as
+ * that rank's own mx_cast_2d_grouped of the received rows would write them
+ * (the 32-token column blocks start at each group start on both sides).
+ *   dst_q[g], dst_s[g]  as mx_cast_dim0_grouped_scatter.
+ *   dst_qt[g]  HOST array of G device pointers: group g's first padded token
+ *              column in the destination's columnwise codes [K, dst_cap[g]]
+ *              (row stride dst_cap[g] bytes).
+ *   dst_st[g]  HOST array of G device pointers: group g's first 512-byte tile
+ *              in the destination's blocked(K, dst_cap[g]/32) scales.
+ *   dst_cap[g] HOST array of G padded capacities of the destinations (each a
+ *              positive multiple of 128 below 2^31).
+ * G at most 512. Every pointer non-NULL and 16-byte aligned (checked on the
+ * host; an empty group's destinations are never written). Bytes written per
+ * group: its rows' codes and scale bands as in the rowwise scatter, and its
+ * columns' codes and scale tiles as in mx_cast_2d_grouped's columnwise
+ * outputs. The call ends with a system-scope fence (a one-thread kernel after
+ * the cast, on the same stream). */
+MX_API mx_status mx_cast_2d_grouped_scatter(const void* x, int64_t M, int64_t K,
+                                            const int32_t* offs, int32_t G, int64_t m_cap,
+                                            void* const* dst_q, void* const* dst_s,
+                                            void* const* dst_qt, void* const* dst_st,
+                                            const int64_t* dst_cap, void* stream);
+
 /* -------------------------------------------------- scaled grouped GEMM --
  * The MXFP8 scaled grouped GEMM over an offsets array (ao "[moe training]
  * Add backward_override to the MXFP8 grouped GEMM", Summary: forward, dgrad

@@ -84,12 +84,26 @@ struct ScatterDests {
   uint8_t* q[kMaxGroups];
   uint8_t* s[kMaxGroups];
 };
+// Destinations of the fused rowwise + columnwise scatter cast: q and s as
+// above, and the group's columnwise outputs in the destination's transposed
+// buffers: qt[g] its first padded token column of codes [C, cap[g]] (row
+// stride cap[g], the destination's padded capacity), st[g] its first 512-byte
+// tile of blocked(C, cap[g]/32) scales (cap[g]/128 tiles per 128-row band).
+constexpr int kScatter2dMaxGroups = 512;     // the table is a kernel parameter (18 KB)
+struct ScatterDests2d {
+  uint8_t* q[kScatter2dMaxGroups];
+  uint8_t* s[kScatter2dMaxGroups];
+  uint8_t* qt[kScatter2dMaxGroups];
+  uint8_t* st[kScatter2dMaxGroups];
+  int32_t cap[kScatter2dMaxGroups];
+};
 
-template <int kMode, bool kGrouped, bool kScatter = false>
+template <int kMode, bool kGrouped, bool kScatter = false, class Dests = ScatterDests>
 __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32_t by, uint32_t bz, uint8_t* wsmem,
                                           GroupSlot* slots, uint8_t* s_row, uint8_t* s_col,
-                                          const ScatterDests* dests = nullptr) {
-  static_assert(!kScatter || (kGrouped && kMode == kModeRow), "the scatter cast is the grouped rowwise cast");
+                                          const Dests* dests = nullptr) {
+  static_assert(!kScatter || (kGrouped && (kMode == kModeRow || kMode == kModeRowCol)),
+                "the scatter casts are the grouped rowwise and fused casts");
   constexpr bool kRow = (kMode & kModeRow) != 0;
   constexpr bool kCol = (kMode & kModeCol) != 0;
   constexpr bool kSq = (kMode & kModeSquare) != 0;
@@ -101,8 +115,10 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
   const uint16_t* __restrict__ x = a.x + z * a.x_stride;
   uint8_t* q = a.q ? a.q + z * a.q_stride : nullptr;
   uint8_t* s = a.s ? a.s + z * a.s_stride : nullptr;
-  uint8_t* const qt = a.qt ? a.qt + z * a.qt_stride : nullptr;
-  uint8_t* const st = a.st ? a.st + z * a.st_stride : nullptr;
+  uint8_t* qt = a.qt ? a.qt + z * a.qt_stride : nullptr;
+  uint8_t* st = a.st ? a.st + z * a.st_stride : nullptr;
+  int64_t qt_rows = a.rows_out;                                               // row stride of qt
+  int64_t col_tiles_col = ceil_div(ceil_div(a.rows_out, kBlock), 4);         // of blocked(C, rows_out/32)
 
   // rows of this tile that hold data, and their first source row
   long long src0 = r0, live = a.rows_src - r0;
@@ -122,6 +138,15 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
     const int64_t bands = ceil_div(ceil_div(a.C, kBlock), 4) * 512;   // bytes of one 128-row scale band
     q = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->q[g]) - uintptr_t(pstart * a.C));
     s = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->s[g]) - uintptr_t((pstart / kCastTile) * bands));
+    if constexpr (kCol) {
+      // token column r of the source's padded layout is column r - pstart of
+      // the group in the destination, whose row stride is its own capacity
+      const int64_t cap = dests->cap[g];
+      qt = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->qt[g]) - uintptr_t(pstart));
+      st = reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(dests->st[g]) - uintptr_t((pstart / kCastTile) * 512));
+      qt_rows = cap;
+      col_tiles_col = cap / kCastTile;
+    }
   }
   const int rw = warp * 32;                           // first tile row of this warp
   uint8_t* slice = wsmem + warp * kWarpSliceBytes;
@@ -162,7 +187,6 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
   }
 
   const int64_t col_tiles_row = ceil_div(ceil_div(a.C, kBlock), 4);          // of blocked(rows_out, C/32)
-  const int64_t col_tiles_col = ceil_div(ceil_div(a.rows_out, kBlock), 4);   // of blocked(C, rows_out/32)
   const int64_t chunk_row = int64_t(by) * col_tiles_row + bx;
   const int64_t chunk_col = int64_t(bx) * col_tiles_col + by;
   const bool rows_out_ok = r0 + rw < a.rows_out;       // the warp's 32 output rows exist
@@ -274,8 +298,8 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
         }
         const int64_t c = c0 + 2 * cp;
         if (rows_out_ok && c < a.C) {
-          st_sector(qt + c * a.rows_out + r0 + rw, qt_al, lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
-          st_sector(qt + (c + 1) * a.rows_out + r0 + rw, qt_al, hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6],
+          st_sector(qt + c * qt_rows + r0 + rw, qt_al, lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
+          st_sector(qt + (c + 1) * qt_rows + r0 + rw, qt_al, hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6],
                     hi[7]);
         }
       }
@@ -325,6 +349,20 @@ cast_scatter_kernel(const __grid_constant__ CastArgs a, const __grid_constant__ 
   __shared__ __align__(16) uint8_t s_row[512];
   __shared__ __align__(16) uint8_t s_col[512];
   cast_tile<kModeRow, true, true>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col, &d);
+}
+
+// The fused rowwise + columnwise cast into per-group destinations: the
+// backward dispatch of expert parallelism (dY of each token group cast both
+// ways, straight into the expert's buffers, in the layout the expert's own
+// fused grouped cast would write). Followed by system_fence_kernel, as above.
+__global__ void __launch_bounds__(kWarpCastThreads)
+cast_scatter2d_kernel(const __grid_constant__ CastArgs a, const __grid_constant__ ScatterDests2d d) {
+  extern __shared__ __align__(128) uint8_t wsmem[];
+  __shared__ GroupSlot slots[kWarpCastWarps];
+  __shared__ __align__(16) uint8_t s_row[512];
+  __shared__ __align__(16) uint8_t s_col[512];
+  cast_tile<kModeRowCol, true, true, ScatterDests2d>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row,
+                                                     s_col, &d);
 }
 
 // One system-scope fence issued after a kernel that stored to other GPUs'

@@ -527,6 +527,42 @@ mx_status mx_cast_dim0_grouped_scatter(const void* x, int64_t M, int64_t K, cons
   return cuda_check("fence launch");
 }
 
+mx_status mx_cast_2d_grouped_scatter(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                                     int64_t m_cap, void* const* dst_q, void* const* dst_s, void* const* dst_qt,
+                                     void* const* dst_st, const int64_t* dst_cap, void* stream) {
+  MX_TRY(check_grouped(x, M, K, offs, G, m_cap));
+  MX_REQUIRE(G <= kScatter2dMaxGroups, MX_ERR_UNSUPPORTED, "G = %d above the fused scatter's %d groups", G,
+             kScatter2dMaxGroups);
+  MX_REQUIRE(dst_q && dst_s && dst_qt && dst_st && dst_cap, MX_ERR_ARG, "null destination arrays");
+  ScatterDests2d d;
+  memset(&d, 0, sizeof(d));
+  for (int32_t g = 0; g < G; ++g) {
+    MX_REQUIRE(dst_q[g] && dst_s[g] && dst_qt[g] && dst_st[g], MX_ERR_ARG, "null destination of group %d", g);
+    MX_REQUIRE(aligned16(dst_q[g]) && aligned16(dst_s[g]) && aligned16(dst_qt[g]) && aligned16(dst_st[g]),
+               MX_ERR_ALIGN, "destination of group %d not 16-byte aligned", g);
+    MX_REQUIRE(dst_cap[g] > 0 && dst_cap[g] % kCastTile == 0 && dst_cap[g] < (1ll << 31), MX_ERR_ARG,
+               "destination capacity of group %d (%lld) must be a positive multiple of 128 below 2^31", g,
+               (long long)dst_cap[g]);
+    d.q[g] = static_cast<uint8_t*>(dst_q[g]);
+    d.s[g] = static_cast<uint8_t*>(dst_s[g]);
+    d.qt[g] = static_cast<uint8_t*>(dst_qt[g]);
+    d.st[g] = static_cast<uint8_t*>(dst_st[g]);
+    d.cap[g] = int32_t(dst_cap[g]);
+  }
+  if (m_cap == 0) return MX_OK;
+  const int64_t row_tiles = m_cap / kCastTile, col_tiles = ceil_div(K, kCastTile);
+  MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535, MX_ERR_UNSUPPORTED,
+             "cast grid too large (%lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles);
+  CastArgs a = make_args(x, M, K, m_cap);
+  a.offs = offs;
+  a.G = G;
+  cast_scatter2d_kernel<<<dim3(unsigned(col_tiles), unsigned(row_tiles), 1u), kWarpCastThreads, kWarpCastSmem,
+                          static_cast<cudaStream_t>(stream)>>>(a, d);
+  MX_TRY(cuda_check("fused scatter cast launch"));
+  system_fence_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_check("fence launch");
+}
+
 mx_status mx_cast_dim1_grouped(const void* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
                                int64_t m_cap, void* qt, void* st, void* stream) {
   MX_TRY(check_grouped(x, M, K, offs, G, m_cap));

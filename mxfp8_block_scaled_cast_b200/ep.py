@@ -211,6 +211,21 @@ class DirectPlan:
         return dq, ds
 
 
+    def destinations_2d(self, base_q, base_s, base_qt, base_st, K: int):
+        """Destinations of the fused (rowwise + columnwise) dispatch, e.g. of dY in
+        backward: each group's rowwise codes and scale bands as destinations(),
+        its first padded token column in the receiving rank's columnwise codes
+        [K, cap_d] and its first tile of their blocked(K, cap_d/32) scales, and
+        cap_d (the receiving rank's padded capacity, the row stride there)."""
+        dq, ds = self.destinations(base_q, base_s, K)
+        dqt, dst, cap = [], [], []
+        for g, row in enumerate(self.dst_row):
+            d = g // self.E
+            dqt.append(int(base_qt[d]) + int(row))
+            dst.append(int(base_st[d]) + int(row) // BLOCK_ROWS * 512)
+            cap.append(int(self.recv_rows_of[d]))
+        return dq, ds, dqt, dst, cap
+
     def combine_destinations(self, out_base, width: int, itemsize: int = 2):
         """Device addresses where each group this rank receives sends its output
         rows: group (source s, local expert e) -> rank s's output buffer
@@ -234,6 +249,22 @@ def dispatch_mxfp8_direct(x, plan: DirectPlan, base_q, base_s):
     offs = torch.as_tensor(ex.offs_send(), device=x.device)
     dq, ds = plan.destinations(base_q, base_s, K)
     mx.mx_cast_dim0_grouped_scatter(x, offs, ex.m_cap_send, dq, ds)
+
+
+def dispatch_2d_direct(t, plan: DirectPlan, base_q, base_s, base_qt, base_st):
+    """The backward dispatch as one kernel: t [M, C] (tokens ordered by global
+    expert; dY in backward) cast rowwise and columnwise straight into every
+    rank's buffers (rank d's rowwise codes [rows, C] and scale bands, its
+    columnwise codes [C, cap_d] and their scale tiles, as mapped on this rank),
+    exactly as rank d's own fused grouped cast of the rows it receives would
+    write them. The ranks must wait for one another before reading."""
+    M, C = t.shape
+    ex = plan.exchange
+    if ex.m_cap_send == 0:
+        return
+    offs = torch.as_tensor(ex.offs_send(), device=t.device)
+    dq, ds, dqt, dst, cap = plan.destinations_2d(base_q, base_s, base_qt, base_st, C)
+    mx.mx_cast_2d_grouped_scatter(t, offs, ex.m_cap_send, dq, ds, dqt, dst, cap)
 
 
 def expert_forward_to_senders(rq, rs, wq, wsf, plan: DirectPlan, y_base):
@@ -283,8 +314,20 @@ def expert_backward(dy_recv, rq, rs, wq, wsd, plan: ExchangePlan, dx_rows=None):
     per group, X from the received codes dequantized to bf16. With dx_rows
     (one device address per received group: where its dX rows go, e.g. into
     the senders' buffers) dX is stored there and dx_recv is None."""
+    if plan.M_recv == 0:
+        return expert_backward_from_codes(None, None, None, None, rq, rs, wq, wsd, plan, dx_rows)
+    offs = torch.as_tensor(plan.offs_recv(), device=dy_recv.device)
+    dq, ds, dqt, dst = mx.cast_2d_grouped(dy_recv, offs, plan.m_cap_recv)
+    return expert_backward_from_codes(dq, ds, dqt, dst, rq, rs, wq, wsd, plan, dx_rows)
+
+
+def expert_backward_from_codes(dq, ds, dqt, dst, rq, rs, wq, wsd, plan: ExchangePlan, dx_rows=None):
+    """expert_backward from dY already cast both ways in the receive layout (dq
+    [m_cap_recv, N] and its scales, dqt [N, m_cap_recv] and its scales: what
+    the fused grouped cast of the received dY writes, or what the senders'
+    dispatch_2d_direct stored there)."""
     E, N, K = wq.shape
-    dev = dy_recv.device
+    dev = rq.device
     dw = torch.empty(E, N, K, dtype=torch.bfloat16, device=dev)
     dx = None if dx_rows is not None else torch.empty(plan.M_recv, K, dtype=torch.bfloat16, device=dev)
     if plan.M_recv == 0:
@@ -292,7 +335,6 @@ def expert_backward(dy_recv, rq, rs, wq, wsd, plan: ExchangePlan, dx_rows=None):
         return dx, dw
     offs = torch.as_tensor(plan.offs_recv(), device=dev)
     G, cap = plan.G_recv, plan.m_cap_recv
-    dq, ds, dqt, dst = mx.cast_2d_grouped(dy_recv, offs, cap)
     if dx_rows is not None:
         mx.mx_grouped_mm_experts_to_rows(dq, ds, wq, wsd, offs, G, E, mx.MX_GROUPS_M_KN, dx_rows, plan.M_recv, K, N,
                                          cap)
@@ -324,14 +366,16 @@ class MXFP8ExpertParallelMM:
     rowwise cast storing each tile straight into the receiving rank's buffer,
     and the combine (and, in backward, the return of dX) is the expert GEMM's
     epilogue storing each output row straight into the rank that sent the
-    token. The buffers are symmetric memory (every rank's mapped into every
-    rank) written with plain stores (no TMA, no multicast); a one-element
-    all-reduce, ordered on the stream after each such kernel, is the barrier
-    before anyone reads. The buffers are kept and grown collectively (every
-    rank computes the same sizes from the gathered counts); outputs are
-    copied out of them, and the received codes the backward reads stay in
-    them, so a second forward of the same layer before its backward is
-    refused. dY still goes to the experts by a bf16 all-to-all."""
+    token; in backward each sender casts dY rowwise and columnwise straight
+    into the experts' buffers. The buffers are
+    symmetric memory (every rank's mapped into every rank) written with plain
+    stores (no TMA, no multicast); a one-element all-reduce, ordered on the
+    stream after each such call, is the barrier before anyone reads. The
+    buffers are kept and grown collectively (every rank computes the same
+    sizes from the gathered counts); outputs are copied out of them, and the
+    received codes the backward reads stay in them, so a second forward of
+    the same layer before its backward is refused. No all-to-all is left on
+    this path."""
 
     def __init__(self, group=None, a2a=None, direct=False, all_gather=None):
         import torch.distributed as dist
@@ -391,10 +435,28 @@ class MXFP8ExpertParallelMM:
         ex = plan.exchange
         E, N, K = wq.shape
         dev = dy.device
-        dy_recv = dispatch_bf16(dy.contiguous(), ex, self.a2a)
+        # dY cast both ways by its senders straight into one symmetric buffer per
+        # rank: rowwise codes [rows, N], their scale bands, columnwise codes
+        # [N, cap] (this rank reads them with its own cap as the row stride)
+        # and their scale tiles; every region starts on a 512-byte boundary
+        rows = int(plan.recv_rows_of.max())
+        band = scale_band_bytes(N)
+        o_s = rows * N
+        o_qt = o_s + rows // BLOCK_ROWS * band
+        o_st = o_qt + N * rows
+        dbuf, dbase = self._symm("dy", o_st + mx.mx_scale_bytes(N, rows // 32), dev)
+        dispatch_2d_direct(dy.contiguous(), plan, dbase, [b + o_s for b in dbase], [b + o_qt for b in dbase],
+                           [b + o_st for b in dbase])
+        self._barrier(dev)
+        cap = ex.m_cap_recv
+        dq = dbuf[:cap * N].view(cap, N)
+        ds = dbuf[o_s:o_s + cap // BLOCK_ROWS * band]
+        dqt = dbuf[o_qt:o_qt + N * cap].view(N, cap)
+        dst = dbuf[o_st:o_st + mx.mx_scale_bytes(N, cap // 32)]
         m_max = int(plan.counts.sum(axis=1).max())
         dxbuf, dxbase = self._symm("dx", m_max * K * 2, dev)
-        _, dw = expert_backward(dy_recv, rq, rs, wq, wsd, ex, dx_rows=plan.combine_destinations(dxbase, K))
+        _, dw = expert_backward_from_codes(dq, ds, dqt, dst, rq, rs, wq, wsd, ex,
+                                           dx_rows=plan.combine_destinations(dxbase, K))
         self._barrier(dev)
         return dxbuf[:ex.M * K * 2].view(torch.bfloat16).view(ex.M, K).clone(), dw
 

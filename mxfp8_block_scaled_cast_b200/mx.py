@@ -36,6 +36,9 @@ _SIGNATURES = {
     "mx_cast_2d_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _vp]),
     "mx_cast_dim0_grouped_scatter": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, ctypes.POINTER(_vp),
                                                     ctypes.POINTER(_vp), _vp]),
+    "mx_cast_2d_grouped_scatter": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _i64, ctypes.POINTER(_vp),
+                                                  ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                                  ctypes.POINTER(_i64), _vp]),
     "mx_grouped_mm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _i64, _vp]),
     "mx_grouped_mm_experts": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                              _i64, _vp]),
@@ -194,6 +197,20 @@ def mx_cast_dim0_grouped_scatter(x, offs, m_cap, dst_q, dst_s, stream=None):
     arr_q = (_vp * G)(*[int(v) for v in dst_q])
     arr_s = (_vp * G)(*[int(v) for v in dst_s])
     _call("mx_cast_dim0_grouped_scatter", _p(x), M, K, _p(offs), G, m_cap, arr_q, arr_s, _stream(stream))
+
+
+def mx_cast_2d_grouped_scatter(x, offs, m_cap, dst_q, dst_s, dst_qt, dst_st, dst_cap, stream=None):
+    """Fused grouped cast with group g's rowwise outputs at dst_q[g] / dst_s[g]
+    and its columnwise outputs at dst_qt[g] / dst_st[g] in a destination of
+    padded capacity dst_cap[g] (lists of G integers; addresses may be
+    peer-mapped)."""
+    M, K = x.shape
+    G = offs.numel()
+    if not (len(dst_q) == len(dst_s) == len(dst_qt) == len(dst_st) == len(dst_cap) == G):
+        raise ValueError("one destination of each kind per group")
+    arrs = [(_vp * G)(*[int(v) for v in lst]) for lst in (dst_q, dst_s, dst_qt, dst_st)]
+    caps = (_i64 * G)(*[int(v) for v in dst_cap])
+    _call("mx_cast_2d_grouped_scatter", _p(x), M, K, _p(offs), G, m_cap, *arrs, caps, _stream(stream))
 
 
 def mx_grouped_mm(a_q, a_s, b_q, b_s, offs, G, mode, out, M, N, K, m_cap, stream=None):

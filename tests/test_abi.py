@@ -100,6 +100,15 @@ def test_host_argument_checks_return_before_any_launch():
                                           two(0x100000, 0x100000), None) == 1   # null destination
     assert L.mx_cast_dim0_grouped_scatter(ok16, 64, 64, ok16, 2, 256, two(0x100000, 0x100008),
                                           two(0x100000, 0x100000), None) == 2   # misaligned destination
+    # the fused scatter cast: four destinations and a capacity per group
+    ok2 = two(0x100000, 0x100000)
+    caps = (ctypes.c_int64 * 2)(256, 256)
+    assert L.mx_cast_2d_grouped_scatter(ok16, 64, 64, ok16, 2, 256, ok2, ok2, ok2, None, caps,
+                                        None) == 1                      # null destination array
+    assert L.mx_cast_2d_grouped_scatter(ok16, 64, 64, ok16, 2, 256, ok2, ok2, two(0x100000, 0x100008), ok2,
+                                        caps, None) == 2                # misaligned destination
+    assert L.mx_cast_2d_grouped_scatter(ok16, 64, 64, ok16, 2, 256, ok2, ok2, ok2, ok2,
+                                        (ctypes.c_int64 * 2)(256, 200), None) == 1   # capacity not 128-aligned
     # the GEMM with per-group output rows: M-group modes only, every destination checked
     assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, ok16, 2, 2, 1, two(0x100000, 0x100000),
                                            128, 256, 128, 256, None) == 1    # K-groups mode

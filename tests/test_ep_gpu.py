@@ -275,3 +275,38 @@ def test_fused_combine_equals_the_all_to_all(mx, W, E, N, K):
     for s in range(W):
         assert torch.equal(ybuf[s], ys[s]), f"outputs of rank {s}"
         assert torch.equal(dxbuf[s], dxs[s]), f"dX of rank {s}"
+
+
+@pytest.mark.parametrize("W,E,N", [(2, 3, 576), (4, 2, 256), (3, 1, 96)])
+def test_direct_dy_dispatch_equals_the_experts_own_cast(mx, W, E, N):
+    """The backward dispatch as one kernel (every rank's dY cast rowwise and
+    columnwise straight into every expert's buffers), ranks emulated with local
+    buffers: each rank's four outputs are bitwise what its own fused grouped
+    cast of the dY the all-to-all delivers would write."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    rng = np.random.default_rng(90 + W)
+    counts = rng.integers(0, 260, size=(W, W * E))
+    counts[0, -1] = 0
+    counts[W - 1, :E] = 128
+    dys = [S.normal_bf16((int(counts[r].sum()), N), 0.1, seed=95 + r).cuda() for r in range(W)]
+    plans = [ep.ExchangePlan(W, E, counts[r], counts[:, r * E:(r + 1) * E]) for r in range(W)]
+    dy_recv = _virtual_a2a(dys, [pl.send_tokens for pl in plans], [pl.recv_tokens for pl in plans])
+    band = ep.scale_band_bytes(N)
+    fill = lambda n: torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
+    bq = [fill(pl.m_cap_recv * N) for pl in plans]
+    bs = [fill(pl.m_cap_recv // 128 * band) for pl in plans]
+    bqt = [fill(N * pl.m_cap_recv) for pl in plans]
+    bst = [fill(mx.mx_scale_bytes(N, pl.m_cap_recv // 32)) for pl in plans]
+    ptrs = lambda bufs: [b.data_ptr() for b in bufs]
+    for r in range(W):
+        ep.dispatch_2d_direct(dys[r], ep.DirectPlan(W, E, r, counts), ptrs(bq), ptrs(bs), ptrs(bqt), ptrs(bst))
+    mx.mx_device_error()
+    for d, pl in enumerate(plans):
+        if pl.M_recv == 0:
+            continue
+        offs = torch.as_tensor(pl.offs_recv()).cuda()
+        q, s, qt, st = mx.cast_2d_grouped(dy_recv[d], offs, pl.m_cap_recv)
+        assert torch.equal(bq[d], q.reshape(-1)), f"rowwise codes of rank {d}"
+        assert torch.equal(bs[d], s.reshape(-1)), f"rowwise scales of rank {d}"
+        assert torch.equal(bqt[d], qt.reshape(-1)), f"columnwise codes of rank {d}"
+        assert torch.equal(bst[d], st.reshape(-1)), f"columnwise scales of rank {d}"

@@ -193,6 +193,28 @@ def test_scatter_cast_stays_in_bounds(mx):
     g.check(mx, "scatter cast")
 
 
+def test_fused_scatter_cast_stays_in_bounds(mx):
+    """The fused (rowwise + columnwise) scatter cast of three emulated ranks'
+    dY into every rank's four guarded receive buffers (N = 96, ragged groups)."""
+    from mxfp8_block_scaled_cast_b200 import ep
+    W, E, N = 3, 2, 96
+    rng = np.random.default_rng(7)
+    counts = rng.integers(0, 300, size=(W, W * E))
+    counts[1, 2] = 0
+    plans = [ep.ExchangePlan(W, E, counts[r], counts[:, r * E:(r + 1) * E]) for r in range(W)]
+    band = ep.scale_band_bytes(N)
+    g = Guarded()
+    bq = [g.raw(pl.m_cap_recv * N) for pl in plans]
+    bs = [g.raw(pl.m_cap_recv // 128 * band) for pl in plans]
+    bqt = [g.raw(N * pl.m_cap_recv) for pl in plans]
+    bst = [g.raw(mx.mx_scale_bytes(N, pl.m_cap_recv // 32)) for pl in plans]
+    ptrs = lambda bufs: [b.data_ptr() for b in bufs]
+    for r in range(W):
+        dy = S.normal_bf16((int(counts[r].sum()), N), 0.1, seed=r).cuda()
+        ep.dispatch_2d_direct(dy, ep.DirectPlan(W, E, r, counts), ptrs(bq), ptrs(bs), ptrs(bqt), ptrs(bst))
+    g.check(mx, "fused scatter cast")
+
+
 def test_gemm_to_sender_rows_stays_in_bounds(mx):
     """The expert GEMMs with the combine fused: outputs and dX rows stored into
     every sender's (guarded) buffer, ranks emulated."""
