@@ -625,6 +625,9 @@ def ep_fused_kernels(mx, device, flush, peaks, W=8, tokens=16384, K=4096, N=4096
     rank spread evenly over the W experts; rank 0's view:
       dispatch  its tokens cast rowwise into the W receiving ranks' buffers (the
                 scatter cast) against the same grouped cast into one send buffer;
+      dispatch_dy  in backward, its dY [tokens, N] cast rowwise and columnwise
+                into the W ranks' buffers against the same fused grouped cast
+                into one buffer;
       combine   its expert GEMM over the groups received from the W senders,
                 storing each output row into its sender's buffer, against the
                 same GEMM into one output.
@@ -674,6 +677,37 @@ def ep_fused_kernels(mx, device, flush, peaks, W=8, tokens=16384, K=4096, N=4096
                 "scattered_over_one": round(med(t["one"]) / med(t["scatter"]), 4), "same_bytes": same_cast}
     del x, recv_q, recv_s, one_q, one_s
 
+    # ---- backward dispatch: dY cast rowwise and columnwise into the W ranks' buffers ----
+    dy = S.normal_bf16((ex.M, N), 0.1, seed=seed + 3, device=device)
+    band_n = ep.scale_band_bytes(N)
+    caps = [int(plan.recv_rows_of[d]) for d in range(W)]
+    rq_ = [u8(c * N) for c in caps]
+    rs_ = [u8(c // 128 * band_n) for c in caps]
+    rqt = [u8(N * c) for c in caps]
+    rst = [u8(mx.mx_scale_bytes(N, c // 32)) for c in caps]
+    d4 = plan.destinations_2d(*[[b.data_ptr() for b in bufs] for bufs in (rq_, rs_, rqt, rst)], N)
+    cm = ex.m_cap_send
+    o_q, o_s, o_qt, o_st = u8(cm * N), u8(cm // 128 * band_n), u8(N * cm), u8(mx.mx_scale_bytes(N, cm // 32))
+    cast2_one = lambda: mx.mx_cast_2d_grouped(dy, offs_s, cm, o_q, o_s, o_qt, o_st)
+    cast2_scatter = lambda: mx.mx_cast_2d_grouped_scatter(dy, offs_s, cm, *d4)
+    t = {"one": [], "scatter": []}
+    for r in range(rounds):
+        for k in (("one", "scatter") if r % 2 == 0 else ("scatter", "one")):
+            t[k].append(flushed_time(cast2_one if k == "one" else cast2_scatter, flush, reps=5, pairs=20, runs=7)[1])
+    nbytes = ex.M * N * 2 + 2 * cm * N + cm // 128 * band_n + o_st.numel()
+    pads_n = [ep._pad(c) for c in counts[0]]
+    starts_n = np.concatenate([[0], np.cumsum(pads_n)[:-1]])
+    same_2d = all(
+        torch.equal(o_q[int(starts_n[d]) * N:int(starts_n[d] + pads_n[d]) * N],
+                    rq_[d][int(plan.dst_row[d]) * N:int(plan.dst_row[d] + pads_n[d]) * N]) and
+        torch.equal(o_qt.view(N, cm)[:, int(starts_n[d]):int(starts_n[d] + pads_n[d])],
+                    rqt[d].view(N, caps[d])[:, int(plan.dst_row[d]):int(plan.dst_row[d] + pads_n[d])])
+        for d in range(W))
+    dispatch_dy = {"bytes_per_launch": nbytes, "one_buffer": rate(med(t["one"])),
+                   "scattered_to_ranks": rate(med(t["scatter"])),
+                   "scattered_over_one": round(med(t["one"]) / med(t["scatter"]), 4), "same_bytes": same_2d}
+    del dy, rq_, rs_, rqt, rst, o_q, o_s, o_qt, o_st
+
     # ---- combine ----
     M_recv, cap, G = ex.M_recv, ex.m_cap_recv, ex.G_recv
     offs_r = torch.as_tensor(ex.offs_recv(), device=device)
@@ -704,7 +738,7 @@ def ep_fused_kernels(mx, device, flush, peaks, W=8, tokens=16384, K=4096, N=4096
     return {"ranks_emulated": W, "experts_per_rank": E, "tokens_per_rank": tokens, "K": K, "N": N,
             "method": "local buffers stand in for the peers' mapped buffers (NVLink not measured: one GPU); casts "
                       "in-stream after an L2 flush, GEMMs as CUDA-graph replays, the two forms alternating",
-            "dispatch": dispatch, "combine": combine}
+            "dispatch": dispatch, "dispatch_dy": dispatch_dy, "combine": combine}
 
 
 def kva_gemms(mx, device, peaks, Mk=16384, Nk=576, Kk=7168):
