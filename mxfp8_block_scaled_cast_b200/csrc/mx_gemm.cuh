@@ -483,6 +483,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                                                    : smem_desc(sbase + kOffB, 16, 1024, 2);
       constexpr uint64_t kBStep = kMode == kGroupsMKn ? (4096 >> 4) : (32 >> 4);
       constexpr uint32_t kIdesc = kIdescBase | (kMode == kGroupsMKn ? (1u << 16) : 0u);
+      // N = 128: the pair MMA's columns [0, 64) are the first CTA's B rows [0, 64)
+      // with their scales in the same TMEM columns as at N = 256
+      constexpr uint32_t kIdescNarrow = (kIdesc & ~(0x3Fu << 17)) | (uint32_t(128 >> 3) << 17);
       const uint64_t sfa_desc0 = smem_desc(sbase + kOffSfa, 0, 128, 0);
       const uint64_t sfb_desc0 = smem_desc(sbase + kOffSfb, 0, 128, 0);
       for (int64_t tile = pair; tile < total_tiles; tile += npairs) {
@@ -495,6 +498,12 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         if (!mbar_wait_warp(ovl_free, (tiles_done & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (slot ? kAccSlot1 : 0u);
+        // a tile at a ragged edge with at most 64 output columns (all from the first
+        // CTA's B rows) runs its MMAs at N = 128, half the tensor work; the columns
+        // this leaves stale are past the output and never stored. B read MN-major
+        // (the dgrad) keeps N = 256: its shared-memory layout is fixed per 128 columns.
+        const int64_t cols_valid = (kMode == kGroupsK ? a.K : a.N) - t.n0;
+        const uint32_t idesc = (kMode != kGroupsMKn && cols_valid <= 64) ? kIdescNarrow : kIdesc;
         bool ok = true;
         for (int kt = 0; kt < t.nk; ++kt) {
           // The TMA bytes of this stage are visible to the tensor core once
@@ -513,10 +522,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             tmem_cp_32x128b_x4_pair(sfb_t, sfb_desc0 + uint64_t((stage * kSfbBytes) >> 4));
             tmem_cp_32x128b_x4_pair(sfb_t + 4, sfb_desc0 + uint64_t((stage * kSfbBytes + 512) >> 4));
             // K block k of the 128-deep stage: +32 bytes (2 in the >>4 field)
-            mma_mxf8_pair(d_tmem, ad, bd, kIdesc, sfa_t, sfb_t, acc0);
-            mma_mxf8_pair(d_tmem, ad + 2, bd + kBStep, kIdesc | (1u << 4) | (1u << 29), sfa_t, sfb_t, 1u);
-            mma_mxf8_pair(d_tmem, ad + 4, bd + 2 * kBStep, kIdesc | (2u << 4) | (2u << 29), sfa_t, sfb_t, 1u);
-            mma_mxf8_pair(d_tmem, ad + 6, bd + 3 * kBStep, kIdesc | (3u << 4) | (3u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad, bd, idesc, sfa_t, sfb_t, acc0);
+            mma_mxf8_pair(d_tmem, ad + 2, bd + kBStep, idesc | (1u << 4) | (1u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 4, bd + 2 * kBStep, idesc | (2u << 4) | (2u << 29), sfa_t, sfb_t, 1u);
+            mma_mxf8_pair(d_tmem, ad + 6, bd + 3 * kBStep, idesc | (3u << 4) | (3u << 29), sfa_t, sfb_t, 1u);
             tc_commit_pair(empty_bar(stage));
           }
           __syncwarp();

@@ -47,6 +47,9 @@ def _nan(*shape):
     ([300, 45], 96, 96),              # smaller than one tile in N and one K step
     ([257], 576, 128),                # ragged N only
     ([128, 1, 200], 512, 160),        # ragged K only
+    ([300, 45], 64, 160),             # every tile 64 columns wide (run at MMA N = 128)
+    ([200, 0, 77], 320, 96),          # 256 + 64 columns
+    ([130], 32, 64),                  # one 32-column tile
 ])
 def test_forward_m_groups_ragged(mx, sizes, N, K):
     M, G = sum(sizes), len(sizes)
@@ -96,6 +99,8 @@ def test_dgrad_from_forward_codes_ragged(mx, sizes, Nw, Kw):
     ([100, 0, 333], 576, 96),         # the 576-wide gradient's wgrad rows, a narrow K
     ([257, 31], 96, 576),
     ([0, 400], 544, 288),
+    ([100, 200], 96, 64),             # output tiles 64 columns wide (run at MMA N = 128)
+    ([257], 64, 32),
 ])
 def test_wgrad_k_groups_ragged(mx, sizes, N, K):
     M, G = sum(sizes), len(sizes)
