@@ -109,6 +109,9 @@ def test_host_argument_checks_return_before_any_launch():
                                         caps, None) == 2                # misaligned destination
     assert L.mx_cast_2d_grouped_scatter(ok16, 64, 64, ok16, 2, 256, ok2, ok2, ok2, ok2,
                                         (ctypes.c_int64 * 2)(256, 200), None) == 1   # capacity not 128-aligned
+    many = (ctypes.c_void_p * 513)(*([0x100000] * 513))
+    assert L.mx_cast_2d_grouped_scatter(ok16, 64, 64, ok16, 513, 128 * 513, many, many, many, many,
+                                        (ctypes.c_int64 * 513)(*([256] * 513)), None) == 3   # above 512 groups
     # the GEMM with per-group output rows: M-group modes only, every destination checked
     assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, ok16, 2, 2, 1, two(0x100000, 0x100000),
                                            128, 256, 128, 256, None) == 1    # K-groups mode
