@@ -46,6 +46,7 @@ from . import mx
 
 BLOCK_ROWS = 128          # rows of a blocked scale tile: the pad path's group alignment
 MAX_GROUPS = 1024         # groups the grouped casts and GEMMs take (include/mx.h)
+DIRECT_MAX_GROUPS = 512   # groups the fused scatter cast takes (the direct mode's dY dispatch)
 
 
 def _pad(n):
@@ -409,6 +410,9 @@ class MXFP8ExpertParallelMM:
 
     def _forward_direct(self, x, send_counts, w):
         E, N, K = w.shape
+        if self.W * E > DIRECT_MAX_GROUPS:
+            raise ValueError(f"direct mode takes at most {DIRECT_MAX_GROUPS} groups (ranks x local experts), "
+                             f"got {self.W} x {E}")
         dev = x.device
         counts = gather_counts(send_counts, self.W, self.all_gather, dev)
         plan = DirectPlan(self.W, E, self.rank, counts)

@@ -262,3 +262,16 @@ def test_gathered_counts_give_the_same_plan_two_gloo_ranks():
     for p in procs:
         p.join(timeout=120)
     assert res == {0: "ok", 1: "ok"}, res
+
+
+def test_direct_mode_refuses_more_groups_than_the_fused_scatter_takes():
+    """Direct mode dispatches dY through the fused scatter cast, which takes at
+    most 512 groups (ranks x local experts): refused before any work."""
+    import torch
+    from mxfp8_block_scaled_cast_b200 import ep
+    layer = ep.MXFP8ExpertParallelMM(direct=True, a2a=lambda *a: None, all_gather=lambda *a: None)
+    E = ep.DIRECT_MAX_GROUPS + 1
+    x = torch.zeros(E, 32, dtype=torch.bfloat16)
+    w = torch.zeros(E, 32, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="at most 512 groups"):
+        layer.forward(x, np.ones(E, dtype=np.int64), w)
