@@ -31,9 +31,12 @@ Layout (this implementation's reading; the pages describe no layout):
     dW of expert e sums its groups from every source rank in one GEMM.
 
 Everything that moves data is torch.distributed.all_to_all_single (NCCL over
-NVLink on GPUs) -- or, for the dispatch with direct=True, the cast kernel
-itself storing into symmetric memory; every arithmetic step is a libmx
-kernel.
+NVLink on GPUs) -- or, with direct=True, the kernels themselves storing into
+symmetric memory: the rowwise cast of the tokens into the receivers' buffers,
+the expert GEMMs' epilogue storing outputs and dX rows into the senders'
+buffers, and in backward the fused cast of dY (rowwise and columnwise, per
+group, bitwise what the receiver's own cast would write) into the experts'
+buffers, so no all-to-all is left. Every arithmetic step is a libmx kernel.
 """
 from __future__ import annotations
 
