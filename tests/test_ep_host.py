@@ -222,6 +222,17 @@ def test_direct_plan_places_groups_in_each_receive_layout():
                 d = g // E
                 assert dq[g] == bq[d] + int(p.dst_row[g]) * K
                 assert ds[g] == bs[d] + int(p.dst_row[g]) // 128 * ep.scale_band_bytes(K)
+            # the fused (backward) dispatch: the columnwise outputs at the group's padded
+            # token column of rank d's [K, cap_d] codes and its 512-byte scale tile there
+            bqt = [(3 << 40) + (1 << 20 * (d + 1)) for d in range(W)]
+            bst = [(5 << 40) + (1 << 20 * (d + 1)) for d in range(W)]
+            dq2, ds2, dqt, dst, cap = p.destinations_2d(bq, bs, bqt, bst, K)
+            assert dq2 == dq and ds2 == ds
+            for g in range(W * E):
+                d = g // E
+                assert cap[g] == p.recv_rows_of[d]
+                assert dqt[g] == bqt[d] + int(p.dst_row[g])
+                assert dst[g] == bst[d] + int(p.dst_row[g]) // 128 * 512
     with pytest.raises(ValueError):
         ep.DirectPlan(2, 2, 0, np.zeros((2, 3)))
     with pytest.raises(ValueError):
