@@ -375,3 +375,21 @@ def test_bf16_token_groups_tiny_shapes(mx):
     offs = offs_t.numpy()
     _assert_close(_f64(out), O.hp_grouped_mm_k(af, bf, offs), O.hp_grouped_mm_k(np.abs(af), np.abs(bf), offs),
                   "tiny token groups")
+
+
+@pytest.mark.parametrize("arm,hp", [(None, False), (None, True), ("high_precision", False), ("dequantized", False)])
+def test_layer_with_no_tokens(mx, arm, hp):
+    """Every group empty (M = 0): the forward returns [0, N], dX [0, K], and dW
+    exact zeros for every expert, under each backward arm."""
+    Gz, Nz, Kz = 4, 256, 384
+    x = torch.empty(0, Kz, dtype=torch.bfloat16, device="cuda")
+    dy = torch.empty(0, Nz, dtype=torch.bfloat16, device="cuda")
+    w = S.normal_bf16((Gz, Nz, Kz), 0.02, seed=9, device="cuda")
+    offs = torch.zeros(Gz, dtype=torch.int32, device="cuda")
+    op = mx.MXFP8GroupedMM(backward_override=arm, wgrad_with_hp=hp)
+    y = op.forward(x, w, offs)
+    dx, dw = op.backward(dy)
+    torch.cuda.synchronize()
+    mx.mx_device_error()
+    assert tuple(y.shape) == (0, Nz) and tuple(dx.shape) == (0, Kz) and tuple(dw.shape) == (Gz, Nz, Kz)
+    assert not dw.any()

@@ -111,3 +111,4 @@ def test_linear_captured_once_replays_new_inputs(mx):
         for name, got, want in zip(("y", "dx", "dw"), outs, refs):
             assert torch.equal(got, want), f"linear {name}, inputs {i}"
     del graph
+
