@@ -98,7 +98,8 @@ struct ScatterDests2d {
   int32_t cap[kScatter2dMaxGroups];
 };
 
-template <int kMode, bool kGrouped, bool kScatter = false, class Dests = ScatterDests>
+template <int kMode, bool kGrouped, bool kScatter = false, class Dests = ScatterDests,
+          bool kSplitLoad = (kMode & kModeCol) != 0>
 __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32_t by, uint32_t bz, uint8_t* wsmem,
                                           GroupSlot* slots, uint8_t* s_row, uint8_t* s_col,
                                           const Dests* dests = nullptr) {
@@ -153,12 +154,15 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
   const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(slice));
 
   // ---- load the 32 x 128 slice ----
-  // With a column pass (dim1, fused) in two halves of 64 columns (two copy
-  // groups, per instruction four rows of eight 16-byte chunks), so that the
-  // first half's columns are converted while the second half is still
-  // arriving (measured: +4-6% at 8192^2); rowwise and 32x32 in one group of
-  // two rows of sixteen chunks per instruction (the split cost them 1-2%).
-  constexpr bool kTwoPhase = kCol;
+  // In two halves of 64 columns (two copy groups, per instruction four rows
+  // of eight 16-byte chunks), so that the first half is converted while the
+  // second is still arriving, or in one group of two rows of sixteen chunks
+  // per instruction. A column pass (dim1, fused) always splits (measured:
+  // +4-6% at 8192^2); rowwise and 32x32 split when the launch is at most a
+  // few waves of tiles, where loads and stores otherwise run in lockstep
+  // (+5% in-stream for 32x32 at 4096^2 and 8192^2 and rowwise at 16384x576),
+  // and load whole slices on larger ones (the split cost them ~1% there).
+  constexpr bool kTwoPhase = kSplitLoad;
   if constexpr (kTwoPhase) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -326,14 +330,15 @@ __device__ __forceinline__ void cast_tile(const CastArgs& a, uint32_t bx, uint32
   }
 }
 
-template <int kMode, bool kGrouped>
+template <int kMode, bool kGrouped, bool kSplitLoad = (kMode & kModeCol) != 0>
 __global__ void __launch_bounds__(kWarpCastThreads)
 cast_warp_kernel(const CastArgs a) {
   extern __shared__ __align__(128) uint8_t wsmem[];
   __shared__ GroupSlot slots[kWarpCastWarps];
   __shared__ __align__(16) uint8_t s_row[512];    // the tile's rowwise (square: forward) scale tile
   __shared__ __align__(16) uint8_t s_col[512];    // the tile's columnwise (square: dgrad) scale tile
-  cast_tile<kMode, kGrouped>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots, s_row, s_col);
+  cast_tile<kMode, kGrouped, false, ScatterDests, kSplitLoad>(a, blockIdx.x, blockIdx.y, blockIdx.z, wsmem, slots,
+                                                             s_row, s_col);
 }
 
 // The grouped rowwise cast with each group's padded rows written to its own

@@ -47,6 +47,10 @@ mx_status cuda_check(const char* what) {
     if (!(cond)) return fail(st, __VA_ARGS__); \
   } while (0)
 
+// Rowwise and 32x32 casts of at most this many 128x128 tiles load each slice in
+// two halves (about nine waves of six CTAs per SM); larger ones load it whole.
+constexpr int64_t kSplitLoadMaxTiles = 8192;
+
 template <int kMode, bool kGrouped>
 mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, int64_t depth,
                       cudaStream_t stream) {
@@ -56,8 +60,15 @@ mx_status launch_cast(const CastArgs& a, int64_t col_tiles, int64_t row_tiles, i
   MX_REQUIRE(col_tiles < (1ll << 31) && row_tiles <= 65535 && depth <= 65535, MX_ERR_UNSUPPORTED,
              "cast grid too large (%lld x %lld x %lld tiles)", (long long)col_tiles, (long long)row_tiles,
              (long long)depth);
-  cast_warp_kernel<kMode, kGrouped><<<dim3(unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)),
-                                      kWarpCastThreads, kWarpCastSmem, stream>>>(a);
+  const dim3 grid{unsigned(col_tiles), unsigned(row_tiles), unsigned(depth)};
+  if constexpr ((kMode & kModeCol) == 0) {
+    // rowwise and 32x32: split loads on launches of a few waves of tiles
+    if (col_tiles * row_tiles * depth > kSplitLoadMaxTiles) {
+      cast_warp_kernel<kMode, kGrouped, false><<<grid, kWarpCastThreads, kWarpCastSmem, stream>>>(a);
+      return cuda_check("cast launch");
+    }
+  }
+  cast_warp_kernel<kMode, kGrouped, true><<<grid, kWarpCastThreads, kWarpCastSmem, stream>>>(a);
   return cuda_check("cast launch");
 }
 
