@@ -98,7 +98,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period_s=0.002):
+    def __init__(self, index, period_s=0.0005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.index = period_s, index
         self._stop = threading.Event()
