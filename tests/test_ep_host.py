@@ -145,7 +145,7 @@ def test_module_rejects_bad_arguments_before_any_exchange():
         layer.backward(torch.zeros(10, 64, dtype=torch.bfloat16))
 
 
-def _dead_peer_worker(rank, port, q):
+def _dead_peer_worker(rank, port, q, direct=False):
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     from datetime import timedelta
@@ -160,20 +160,24 @@ def _dead_peer_worker(rank, port, q):
     import time
     t0 = time.monotonic()
     try:
-        ep.exchange_counts(np.array([1, 2, 3, 4]), 2, 2, ep.dist_all_to_all(), "cpu")
+        if direct:                               # direct mode's first exchange: the count all-gather
+            ep.gather_counts(np.array([1, 2, 3, 4]), 2, ep.dist_all_gather(), "cpu")
+        else:
+            ep.exchange_counts(np.array([1, 2, 3, 4]), 2, 2, ep.dist_all_to_all(), "cpu")
         q.put((0, "no error"))
     except Exception as exc:                     # the collective must end with an error
         q.put((0, f"error after {time.monotonic() - t0:.0f} s: {type(exc).__name__}"))
 
 
-def test_exchange_with_a_dead_peer_ends_with_an_error():
-    """A rank that leaves between steps: the other rank's all-to-all of the token counts
-    (the first exchange of a step) ends with an error within the group's timeout instead
-    of waiting for good."""
+@pytest.mark.parametrize("direct", [False, True])
+def test_exchange_with_a_dead_peer_ends_with_an_error(direct):
+    """A rank that leaves between steps: the other rank's first exchange of a step (the
+    all-to-all of the token counts, or in direct mode their all-gather) ends with an error
+    within the group's timeout instead of waiting for good."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_dead_peer_worker, args=(r, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_dead_peer_worker, args=(r, port, q, direct)) for r in range(2)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=120) for _ in procs)
