@@ -89,3 +89,13 @@ def test_profile_traffic_is_null_once_the_kernel_changes(tmp_path, monkeypatch):
         f.write("// edited\n")
     assert bench.profile_traffic("k.txt", srcs) is None
     assert bench.profile_traffic("missing.txt", srcs) is None
+
+
+def test_committed_gemm_profile_matches_the_kernel_source():
+    """The committed GEMM summary was taken on the kernel as it stands (else the
+    bench would report no traffic)."""
+    import bench
+    t = bench.profile_traffic("mx_gemm_kernel_moe_G8_K4096_N4096.txt",
+                              ["mxfp8_block_scaled_cast_b200/csrc/mx_gemm.cuh",
+                               "mxfp8_block_scaled_cast_b200/csrc/mx_sm100.cuh"])
+    assert t is not None and 2e8 < t < 4e8
