@@ -121,3 +121,31 @@ def test_host_argument_checks_return_before_any_launch():
                                            128, 256, 128, 256, None) == 2    # misaligned destination
     msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
     assert b"not a multiple of 32" in msg
+
+
+def test_oracle_and_product_share_no_code():
+    """The oracle is independent of the CUDA path: the product package (its Python
+    and its CUDA sources) never imports, includes or reads anything under oracle/,
+    and the oracle imports nothing but numpy. Only tests, smoke() and bench.py's
+    CPU legs may use the oracle."""
+    import ast
+    pkg = os.path.join(ROOT, "mxfp8_block_scaled_cast_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                text = open(path).read()
+                for tok in ("mx_oracle", "import oracle", "from oracle", "oracle/"):
+                    assert tok not in text, f"{path} refers to the oracle ({tok!r})"
+            if f.endswith(".py"):
+                tree = ast.parse(open(path).read())
+                for node in ast.walk(tree):
+                    mods = [a.name for a in node.names] if isinstance(node, ast.Import) else (
+                        [node.module or ""] if isinstance(node, ast.ImportFrom) else [])
+                    assert not any(m.split(".")[0] == "oracle" for m in mods), f"{path} imports the oracle"
+    tree = ast.parse(open(os.path.join(ROOT, "oracle", "mx_oracle.py")).read())
+    for node in ast.walk(tree):
+        if isinstance(node, ast.Import):
+            assert all(a.name.split(".")[0] in ("numpy",) for a in node.names), ast.dump(node)
+        elif isinstance(node, ast.ImportFrom) and node.module not in ("__future__",):
+            assert (node.module or "").split(".")[0] == "numpy", ast.dump(node)
