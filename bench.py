@@ -240,6 +240,21 @@ class MoEStep:
                 calls[name]()
 
 
+def select_peak(region_ms, reasons, peaks):
+    """The measured bf16 peak the in-step GEMM rate is held against.
+
+    A timed region of tens of milliseconds is a burst: the burst figure. A long
+    one (beyond 100 ms, or one that saw the power cap engage) takes the
+    sustained figure, as do the seconds-long back-to-back replays of
+    `gemm_only`. Returns (kind, bf16 TFLOP/s, why); a peak missing from the
+    measured file falls back to FALLBACK_PEAKS."""
+    capped = "sw_power_cap" in reasons
+    sustained = region_ms > 100.0 or capped
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    why = f"the timed region lasts {region_ms:.1f} ms" + (" with the power cap engaged" if capped else "")
+    return ("sustained" if sustained else "burst"), float(peaks.get(key, FALLBACK_PEAKS[key])), why
+
+
 def flushed_time(fn, flush, reps=20, pairs=40, runs=15):
     """Seconds per launch of `fn` with the L2 flushed before it, measured two ways.
 
@@ -1066,17 +1081,8 @@ def main(argv=None):
     gemm_ms = [a.elapsed_time(b) for a, b in step.gemm_events]
     gemm_avg_s = sum(gemm_ms) / len(gemm_ms) * 1e-3
     gemm_tflops = GEMM_FLOPS / gemm_avg_s / 1e12
-    # A timed region of tens of milliseconds is a burst: the in-step GEMM rate
-    # is held against the burst figure. A long one (the power cap engaged, or
-    # beyond 100 ms) is held against the sustained figure, as are the
-    # seconds-long back-to-back replays of `gemm_only`.
-    sustained = total_ms > 100.0 or "sw_power_cap" in clocks.summary()["reasons"]
-    peak_kind = "sustained" if sustained else "burst"
-    peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
-    bf16_peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    peak_kind, bf16_peak, peak_why = select_peak(total_ms, clocks.summary()["reasons"], peaks)
     fp8_peak = bf16_peak * FP8_OVER_BF16
-    peak_why = (f"the timed region lasts {total_ms:.1f} ms" +
-                (" with the power cap engaged" if "sw_power_cap" in clocks.summary()["reasons"] else ""))
     traffic = profile_traffic("mx_gemm_kernel_moe_G8_K4096_N4096.txt",
                               ["mxfp8_block_scaled_cast_b200/csrc/mx_gemm.cuh",
                                "mxfp8_block_scaled_cast_b200/csrc/mx_sm100.cuh"])

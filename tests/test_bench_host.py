@@ -99,3 +99,18 @@ def test_committed_gemm_profile_matches_the_kernel_source():
                               ["mxfp8_block_scaled_cast_b200/csrc/mx_gemm.cuh",
                                "mxfp8_block_scaled_cast_b200/csrc/mx_sm100.cuh"])
     assert t is not None and 2e8 < t < 4e8
+
+
+def test_peak_follows_the_length_of_the_timed_region_and_the_power_cap():
+    """The in-step GEMM rate is held against the burst peak for a short region
+    and against the sustained one for a long or power-capped region."""
+    import bench
+    peaks = {"bf16_tflops": 1665.9, "bf16_tflops_sustained": 1414.4}
+    kind, peak, why = bench.select_peak(16.3, [], peaks)
+    assert (kind, peak) == ("burst", 1665.9) and "16.3 ms" in why
+    kind, peak, why = bench.select_peak(16.3, ["sw_power_cap"], peaks)
+    assert (kind, peak) == ("sustained", 1414.4) and "power cap" in why
+    assert bench.select_peak(250.0, [], peaks)[:2] == ("sustained", 1414.4)
+    # a measured file without a figure falls back to the recorded ones
+    assert bench.select_peak(16.3, [], {})[1] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert bench.select_peak(250.0, [], {})[1] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
