@@ -798,7 +798,9 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
     """MXFP8 linear forward + backward at M=4096, N=4096, K=2048 (the MXFP8Linear
     benchmark shape of ao PR #4705): y = x w^T, dx = dy w, dw = dy^T x, each step
     re-quantizing w (no cache) or reusing its cached quantization (cache hit, as in
-    activation-checkpoint recompute). A step is ~0.15 ms of GPU work in seven
+    activation-checkpoint recompute); as separate forward and backward calls (each
+    casting what it reads, w included) and as the training pair (the backward
+    reusing the forward's casts of x and w, as the autograd linear does). A step is ~0.15 ms of GPU work in seven
     launches, so it is timed both as issued from Python (eager, median of
     L2-flushed repetitions, includes host submission) and as CUDA-graph replays of
     `graph_steps` steps (median of 5 replays, per step)."""
@@ -807,6 +809,7 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
     Ml, Nl, Kl = 4096, 4096, 2048
     x, w, dy = S.linear_problem(Ml, Nl, Kl, seed=0, device=device)
     ws = mx.linear_workspace(Ml, Nl, Kl, device)
+    ws_train = mx.linear_workspace(Ml, Nl, Kl, device, train=True)
     y = torch.empty(Ml, Nl, dtype=torch.bfloat16, device=device)
     dx = torch.empty(Ml, Kl, dtype=torch.bfloat16, device=device)
     dw = torch.empty(Nl, Kl, dtype=torch.bfloat16, device=device)
@@ -815,6 +818,10 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
     def step(c):
         mx.mx_linear_fwd(x, w, c, 0, y, ws)
         mx.mx_linear_bwd(dy, x, w, c, 0, dx, dw, ws)
+
+    def train_step(c):              # the forward's casts of x and w serve the backward
+        mx.mx_linear_fwd_train(x, w, c, 0, y, ws_train)
+        mx.mx_linear_bwd_after_fwd(dy, w, c, 0, dx, dw, ws_train)
 
     def timed(fn):
         for _ in range(3):
@@ -857,6 +864,8 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
 
     t_nc, g_nc = timed(lambda: step(None)), graphed(lambda: step(None))
     t_hit, g_hit = timed(lambda: step(cache)), graphed(lambda: step(cache))
+    tp_nc, gp_nc = timed(lambda: train_step(None)), graphed(lambda: train_step(None))
+    tp_hit, gp_hit = timed(lambda: train_step(cache)), graphed(lambda: train_step(cache))
     mx.mx_device_error()
     hits = cache.stats()["hits"]
     cache.close()
@@ -864,7 +873,11 @@ def linear_bench(mx, device, flush, peaks, reps=20, graph_steps=10):
     entry = lambda te, tg: {"ms_per_step_graph": round(tg * 1e3, 4), "tflops_graph": round(flops / tg / 1e12, 1),
                             "ms_per_step_eager": round(te * 1e3, 4), "tflops_eager": round(flops / te / 1e12, 1)}
     return {"shape": {"M": Ml, "N": Nl, "K": Kl}, "flops_per_step": flops,
-            "no_cache": entry(t_nc, g_nc), "cache_hit": dict(entry(t_hit, g_hit), hits=hits)}
+            "no_cache": entry(t_nc, g_nc), "cache_hit": dict(entry(t_hit, g_hit), hits=hits),
+            "training_pair": {"no_cache": entry(tp_nc, gp_nc), "cache_hit": entry(tp_hit, gp_hit),
+                              "what": "mx_linear_fwd_train + mx_linear_bwd_after_fwd: the backward "
+                                      "casts dY only (x's columnwise cast and w's quantization are the "
+                                      "forward's)"}}
 
 
 def override_arms(mx, step, flush, peaks):

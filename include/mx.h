@@ -387,6 +387,42 @@ MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
                                mx_wcache* cache, uint64_t w_version, void* dx, void* dw,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------ linear training pair -----
+ * The same linear for a training step whose backward follows its forward:
+ * the forward keeps, in the workspace, what the backward would otherwise
+ * re-compute from x and w. The 32x32 weight cast writes both scale views at
+ * once (ao PR #4705, "MXFP8Linear training paths"), so the forward's
+ * quantization of w serves the dgrad; and x's columnwise cast comes out of
+ * the forward's single read of x (the fused rowwise + columnwise cast).
+ *   mx_linear_fwd_train     y as mx_linear_fwd; x cast rowwise and
+ *                           columnwise in one launch with the weight's cast;
+ *                           x's columnwise codes and scales, and (without a
+ *                           cache) w's quantization, stay in ws.
+ *   mx_linear_bwd_after_fwd dx, dw as mx_linear_bwd, casting only dy: x's
+ *                           columnwise cast and w's quantization are the
+ *                           forward's (with a cache: the cache entry, re-cast
+ *                           from w only on a miss). x is not read.
+ * Results are bitwise those of mx_linear_fwd + mx_linear_bwd on the same
+ * x, w and dy. Contract: the backward runs on the workspace of the forward
+ * whose step it completes, with nothing else using that workspace in
+ * between, the same cache argument (NULL or not), and -- when a cache is
+ * given -- w's bytes unchanged since that forward. Without a cache, w's bytes
+ * may change in between: the backward uses the forward's quantization, as
+ * the gradient of that forward's product. x may be freed or overwritten
+ * once the forward's work on `stream` is done.
+ * ws: caller-owned, at least mx_linear_train_ws_bytes(M, N, K) bytes -- x's
+ * columnwise cast, then the larger of x's rowwise and dy's casts, then w's
+ * quantization; more than mx_linear_ws_bytes when K > 2N, because the forward
+ * holds both casts of x at once. Size rules and errors as mx_linear_fwd and
+ * mx_linear_bwd (a workspace below mx_linear_train_ws_bytes: MX_ERR_ARG). */
+MX_API size_t mx_linear_train_ws_bytes(int64_t M, int64_t N, int64_t K);
+MX_API mx_status mx_linear_fwd_train(const void* x, const void* w, int64_t M, int64_t N, int64_t K,
+                                     mx_wcache* cache, uint64_t w_version, void* y,
+                                     void* ws, size_t ws_bytes, void* stream);
+MX_API mx_status mx_linear_bwd_after_fwd(const void* dy, const void* w, int64_t M, int64_t N, int64_t K,
+                                         mx_wcache* cache, uint64_t w_version, void* dx, void* dw,
+                                         void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------- linear forward, no allocation --
  * No counterpart on the source pages: an addition for callers that cannot
  * allocate device memory and so cannot pass a workspace -- a plain C host

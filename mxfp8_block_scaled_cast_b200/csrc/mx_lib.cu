@@ -803,17 +803,22 @@ size_t mx_linear_ws_bytes(int64_t M, int64_t N, int64_t K) {
   return size_t((fwd > bwd ? fwd : bwd) + wq_bytes(N, K));
 }
 
+size_t mx_linear_train_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N <= 0 || K <= 0) return 0;
+  return size_t(linear_train_ws_bytes(M, N, K));
+}
+
 }  // extern "C"
 
 namespace mx {
 namespace {
 
-mx_status check_linear(int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes) {
+mx_status check_linear(int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, bool train = false) {
   MX_REQUIRE(M >= 0 && N > 0 && K > 0, MX_ERR_ARG, "sizes must be M >= 0, N > 0, K > 0");
   MX_REQUIRE(M % kBlock == 0, MX_ERR_UNSUPPORTED, "M = %lld is not a multiple of 32", (long long)M);
   MX_REQUIRE(N % kBlock == 0 && K % kBlock == 0, MX_ERR_UNSUPPORTED, "N and K must be multiples of 32");
-  MX_REQUIRE(ws_bytes >= mx_linear_ws_bytes(M, N, K), MX_ERR_ARG, "workspace too small (%zu < %zu bytes)",
-             ws_bytes, mx_linear_ws_bytes(M, N, K));
+  const size_t need = train ? mx_linear_train_ws_bytes(M, N, K) : mx_linear_ws_bytes(M, N, K);
+  MX_REQUIRE(ws_bytes >= need, MX_ERR_ARG, "workspace too small (%zu < %zu bytes)", ws_bytes, need);
   MX_REQUIRE(ws != nullptr && aligned16(ws), MX_ERR_ALIGN, "workspace null or not 16-byte aligned");
   return MX_OK;
 }
@@ -947,6 +952,56 @@ mx_status mx_linear_bwd(const void* dy, const void* x, const void* w, int64_t M,
   const WeightView& wv = wp.view;
   MX_TRY(mx_grouped_mm(dyq, dys, wv.q, wv.s_dgrad, nullptr, 1, MX_GROUPS_M_KN, dx, M, K, N, 0, stream));
   return mx_grouped_mm(dyqt, dyst, xqt, xst, nullptr, 1, MX_GROUPS_K, dw, M, N, K, 0, stream);
+}
+
+mx_status mx_linear_fwd_train(const void* x, const void* w, int64_t M, int64_t N, int64_t K, mx_wcache* cache,
+                              uint64_t w_version, void* y, void* ws, size_t ws_bytes, void* stream) {
+  MX_TRY(check_linear(M, N, K, ws, ws_bytes, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const LinearTrainWs L = carve_train_ws(ws, M, N, K);
+  // the weight's cast (on a miss) and X's fused rowwise + columnwise cast go
+  // out as one launch; the columnwise codes stay in the workspace for the backward
+  std::unique_lock<std::mutex> lk = lock_cache(cache);
+  WeightPlan wp;
+  MX_TRY(plan_weight(w, N, K, cache, w_version, L.wq, &wp));
+  PreparedCast casts[2];
+  casts[0] = wp.cast;
+  if (M > 0) MX_TRY(prepare_2d(x, M, K, L.xq, L.xs, L.xqt, L.xst, &casts[1]));
+  MX_TRY(launch_casts(casts, 2, st));
+  commit_weight(wp);
+  if (lk.owns_lock()) lk.unlock();
+  if (M == 0) return MX_OK;
+  const WeightView& wv = wp.view;
+  return mx_grouped_mm(L.xq, L.xs, wv.q, wv.s_fwd, nullptr, 1, MX_GROUPS_M, y, M, N, K, 0, stream);
+}
+
+mx_status mx_linear_bwd_after_fwd(const void* dy, const void* w, int64_t M, int64_t N, int64_t K,
+                                  mx_wcache* cache, uint64_t w_version, void* dx, void* dw, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  MX_TRY(check_linear(M, N, K, ws, ws_bytes, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const LinearTrainWs L = carve_train_ws(ws, M, N, K);
+  // X's columnwise cast is the forward's; the weight's quantization is the
+  // forward's (workspace) or the cache's (re-cast only on a miss); dY's fused
+  // cast is the one cast of this call
+  std::unique_lock<std::mutex> lk = lock_cache(cache);
+  WeightPlan wp;
+  if (cache != nullptr) MX_TRY(plan_weight(w, N, K, cache, w_version, L.wq, &wp));
+  else wp.view = carve_weight(L.wq, N, K);
+  PreparedCast casts[2];
+  casts[0] = wp.cast;
+  if (M > 0) MX_TRY(prepare_2d(dy, M, N, L.dyq, L.dys, L.dyqt, L.dyst, &casts[1]));
+  MX_TRY(launch_casts(casts, 2, st));
+  commit_weight(wp);
+  if (lk.owns_lock()) lk.unlock();
+  if (M == 0) {
+    cudaError_t e = cudaMemsetAsync(dw, 0, size_t(N) * K * 2, st);
+    MX_REQUIRE(e == cudaSuccess, MX_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MX_OK;
+  }
+  const WeightView& wv = wp.view;
+  MX_TRY(mx_grouped_mm(L.dyq, L.dys, wv.q, wv.s_dgrad, nullptr, 1, MX_GROUPS_M_KN, dx, M, K, N, 0, stream));
+  return mx_grouped_mm(L.dyqt, L.dyst, L.xqt, L.xst, nullptr, 1, MX_GROUPS_K, dw, M, N, K, 0, stream);
 }
 
 }  // extern "C"

@@ -61,3 +61,53 @@ inline WeightView carve_weight(uint8_t* base, int64_t N, int64_t K) {
 }
 
 }  // namespace mx
+
+namespace mx {
+
+// Workspace pieces of the linear, each rounded up to 256 bytes: X cast
+// rowwise ([M, K] codes + blocked(M, K/32)), X cast columnwise ([K, M] +
+// blocked(K, M/32)), dY cast both ways ([M, N] + blocked(M, N/32), [N, M] +
+// blocked(N, M/32)).
+inline int64_t linear_x_bytes(int64_t M, int64_t K) {
+  return ceil_to(M * K, 256) + ceil_to(scale_bytes(M, K / kBlock), 256);
+}
+inline int64_t linear_xt_bytes(int64_t M, int64_t K) {
+  return ceil_to(K * M, 256) + ceil_to(scale_bytes(K, M / kBlock), 256);
+}
+inline int64_t linear_dy_bytes(int64_t M, int64_t N) {
+  return 2 * ceil_to(M * N, 256) + ceil_to(scale_bytes(M, N / kBlock), 256) + ceil_to(scale_bytes(N, M / kBlock), 256);
+}
+
+// The training pair's workspace (forward that keeps X's columnwise cast for
+// its backward): X's columnwise codes and scales first -- written by the
+// forward, read by the backward -- then the forward's rowwise X or the
+// backward's dY casts (the larger of the two), then W's quantization.
+struct LinearTrainWs {
+  uint8_t *xqt, *xst;                 // [K, M], blocked(K, M/32)
+  uint8_t *xq, *xs;                   // [M, K], blocked(M, K/32)      (forward)
+  uint8_t *dyq, *dys, *dyqt, *dyst;   // [M, N], blocked(M, N/32), [N, M], blocked(N, M/32)  (backward)
+  uint8_t* wq;                        // carve_weight(wq, N, K) when there is no cache
+};
+
+inline int64_t linear_train_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  const int64_t x = linear_x_bytes(M, K), dy = linear_dy_bytes(M, N);
+  return linear_xt_bytes(M, K) + (x > dy ? x : dy) + wq_bytes(N, K);
+}
+
+inline LinearTrainWs carve_train_ws(void* ws, int64_t M, int64_t N, int64_t K) {
+  LinearTrainWs L;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  L.xqt = p;
+  L.xst = L.xqt + ceil_to(K * M, 256);
+  uint8_t* mid = p + linear_xt_bytes(M, K);
+  L.xq = mid;
+  L.xs = L.xq + ceil_to(M * K, 256);
+  L.dyq = mid;
+  L.dys = L.dyq + ceil_to(M * N, 256);
+  L.dyqt = L.dys + ceil_to(scale_bytes(M, N / kBlock), 256);
+  L.dyst = L.dyqt + ceil_to(M * N, 256);
+  L.wq = p + (linear_train_ws_bytes(M, N, K) - wq_bytes(N, K));
+  return L;
+}
+
+}  // namespace mx

@@ -54,6 +54,10 @@ _SIGNATURES = {
     "mx_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _vp, _sz,
                                      _vp]),
     "mx_linear_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "mx_linear_train_ws_bytes": (_sz, [_i64, _i64, _i64]),
+    "mx_linear_fwd_train": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _sz, _vp]),
+    "mx_linear_bwd_after_fwd": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_uint64, _vp, _vp, _vp,
+                                               _sz, _vp]),
     "mx_cast_ex": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "mx_grouped_mm_bf16": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _vp, _i64, _i64, _i64, _vp]),
     "mx_dequant_dim0": (ctypes.c_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp]),
@@ -248,6 +252,27 @@ def mx_linear_bwd(dy, x, w, cache, w_version, dx, dw, ws, stream=None):
     M, K = x.shape
     N = w.shape[0]
     _call("mx_linear_bwd", _p(dy), _p(x), _p(w), M, N, K, cache.handle if cache is not None else None,
+          int(w_version), _p(dx), _p(dw), _p(ws), ws.numel(), _stream(stream))
+
+
+def mx_linear_train_ws_bytes(M, N, K) -> int:
+    return int(lib().mx_linear_train_ws_bytes(M, N, K))
+
+
+def mx_linear_fwd_train(x, w, cache, w_version, y, ws, stream=None):
+    """Forward of a training step: as mx_linear_fwd, and keeps x's columnwise
+    cast (and, without a cache, w's quantization) in `ws` for mx_linear_bwd_after_fwd."""
+    M, K = x.shape
+    N = w.shape[0]
+    _call("mx_linear_fwd_train", _p(x), _p(w), M, N, K, cache.handle if cache is not None else None,
+          int(w_version), _p(y), _p(ws), ws.numel(), _stream(stream))
+
+
+def mx_linear_bwd_after_fwd(dy, w, cache, w_version, dx, dw, ws, stream=None):
+    """Backward of the step whose forward was mx_linear_fwd_train on `ws`: casts dY only."""
+    M, N = dy.shape
+    K = w.shape[1]
+    _call("mx_linear_bwd_after_fwd", _p(dy), _p(w), M, N, K, cache.handle if cache is not None else None,
           int(w_version), _p(dx), _p(dw), _p(ws), ws.numel(), _stream(stream))
 
 
@@ -460,8 +485,11 @@ def grouped_mm_wgrad(a_q, a_s, b_q, b_s, offs, M, G=None):
     return out
 
 
-def linear_workspace(M, N, K, device="cuda"):
-    return torch.empty(mx_linear_ws_bytes(M, N, K), dtype=torch.uint8, device=device)
+def linear_workspace(M, N, K, device="cuda", train=False):
+    """Workspace of mx_linear_fwd / mx_linear_bwd, or (train=True) of the
+    training pair mx_linear_fwd_train / mx_linear_bwd_after_fwd."""
+    n = mx_linear_train_ws_bytes(M, N, K) if train else mx_linear_ws_bytes(M, N, K)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def _version_of(w, cache):
@@ -666,7 +694,11 @@ def mxfp8_grouped_mm(x, w, offs, backward_override=None, wgrad_with_hp=False):
 
 
 class _LinearFn(torch.autograd.Function):
-    """Autograd wrapper of the MXFP8 linear (mx_linear_fwd / mx_linear_bwd)."""
+    """Autograd wrapper of the MXFP8 linear. When a gradient is wanted the
+    forward is mx_linear_fwd_train and the backward mx_linear_bwd_after_fwd:
+    the forward's casts of x and w serve the backward, so x itself is not
+    saved (its columnwise codes are, in the workspace, one byte per element)
+    and the backward casts dY only. Otherwise the forward is mx_linear_fwd."""
 
     @staticmethod
     def forward(ctx, x, w, cache):
@@ -674,22 +706,24 @@ class _LinearFn(torch.autograd.Function):
         version = _version_of(w, cache)
         M, K = x.shape
         N = w.shape[0]
-        ws = linear_workspace(M, N, K, x.device)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
-        mx_linear_fwd(x, w, cache, version, y, ws)
-        ctx.save_for_backward(x, w)
-        ctx.cache, ctx.version, ctx.ws = cache, version, ws
+        if not any(ctx.needs_input_grad[:2]):
+            mx_linear_fwd(x, w, cache, version, y, linear_workspace(M, N, K, x.device))
+            return y
+        ws = linear_workspace(M, N, K, x.device, train=True)
+        mx_linear_fwd_train(x, w, cache, version, y, ws)
+        ctx.save_for_backward(w)        # autograd refuses the backward if w is updated in place meanwhile
+        ctx.cache, ctx.version, ctx.ws, ctx.M = cache, version, ws, M
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        x, w = ctx.saved_tensors
+        w, = ctx.saved_tensors
         dy = _check_bf16(dy)
-        M, K = x.shape
-        N = w.shape[0]
-        dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
-        dw = torch.empty(N, K, dtype=torch.bfloat16, device=x.device)
-        mx_linear_bwd(dy, x, w, ctx.cache, ctx.version, dx, dw, ctx.ws)
+        N, K = w.shape
+        dx = torch.empty(ctx.M, K, dtype=torch.bfloat16, device=w.device)
+        dw = torch.empty(N, K, dtype=torch.bfloat16, device=w.device)
+        mx_linear_bwd_after_fwd(dy, w, ctx.cache, ctx.version, dx, dw, ctx.ws)
         if ctx.cache is not None and ctx.cache.clear_after_backward:
             ctx.cache.evict(w)
         ctx.ws = None

@@ -119,6 +119,16 @@ def test_host_argument_checks_return_before_any_launch():
                                            128, 256, 128, 256, None) == 1    # no offsets
     assert L.mx_grouped_mm_experts_to_rows(ok16, ok16, ok16, ok16, ok16, 2, 2, 0, two(0x100000, 0x100004),
                                            128, 256, 128, 256, None) == 2    # misaligned destination
+    # the linear training pair: its own workspace, larger than the plain pair's when K > 2N
+    # (the forward holds both casts of x at once), the same where dY's casts are the larger
+    Ml, Nl, Kl = 256, 96, 576
+    plain, train = L.mx_linear_ws_bytes(Ml, Nl, Kl), L.mx_linear_train_ws_bytes(Ml, Nl, Kl)
+    assert train > plain
+    assert L.mx_linear_train_ws_bytes(4096, 4096, 2048) == L.mx_linear_ws_bytes(4096, 4096, 2048)
+    assert L.mx_linear_fwd_train(ok16, ok16, Ml, Nl, Kl, None, 0, ok16, ok16, plain, None) == 1  # ws too small
+    assert L.mx_linear_bwd_after_fwd(ok16, ok16, Ml, Nl, Kl, None, 0, ok16, ok16, ok16, plain, None) == 1
+    assert L.mx_linear_fwd_train(ok16, ok16, 48, Nl, Kl, None, 0, ok16, ok16, train, None) == 3  # M % 32
+    assert L.mx_linear_bwd_after_fwd(ok16, ok16, Ml, Nl, Kl, None, 0, ok16, ok16, odd, train, None) == 2
     msg = (L.mx_cast_dim0(ok16, 64, 48, ok16, ok16, None), L.mx_last_error())[1]
     assert b"not a multiple of 32" in msg
 

@@ -68,16 +68,18 @@ def test_step_captured_once_replays_under_new_routing(mx, arm):
     del graph
 
 
-def test_linear_captured_once_replays_new_inputs(mx):
+@pytest.mark.parametrize("train", [False, True])
+def test_linear_captured_once_replays_new_inputs(mx, train):
     """The linear forward and backward without the weight cache (the cache decides
     hit or miss on the host, once, at capture), with its workspace: one capture,
     replays on new x, w and dy bitwise equal to eager calls. Sizes off the GEMM
-    tile (N = 96, K = 576) take the pad path."""
+    tile (N = 96, K = 576) take the pad path. Both the separate calls and the
+    training pair (whose backward reads the forward's casts from the workspace)."""
     Ml, Nl, Kl = 256, 96, 576
     x = torch.empty(Ml, Kl, dtype=torch.bfloat16, device="cuda")
     w = torch.empty(Nl, Kl, dtype=torch.bfloat16, device="cuda")
     dy = torch.empty(Ml, Nl, dtype=torch.bfloat16, device="cuda")
-    ws = mx.linear_workspace(Ml, Nl, Kl)
+    ws = mx.linear_workspace(Ml, Nl, Kl, train=train)
     outs = [torch.empty(Ml, Nl, dtype=torch.bfloat16, device="cuda"),
             torch.empty(Ml, Kl, dtype=torch.bfloat16, device="cuda"),
             torch.empty(Nl, Kl, dtype=torch.bfloat16, device="cuda")]
@@ -88,8 +90,12 @@ def test_linear_captured_once_replays_new_inputs(mx):
         dy.copy_(S.normal_bf16((Ml, Nl), 0.1, seed=50 + i, device="cuda"))
 
     def step(y, dx, dw):
-        mx.mx_linear_fwd(x, w, None, 0, y, ws)
-        mx.mx_linear_bwd(dy, x, w, None, 0, dx, dw, ws)
+        if train:
+            mx.mx_linear_fwd_train(x, w, None, 0, y, ws)
+            mx.mx_linear_bwd_after_fwd(dy, w, None, 0, dx, dw, ws)
+        else:
+            mx.mx_linear_fwd(x, w, None, 0, y, ws)
+            mx.mx_linear_bwd(dy, x, w, None, 0, dx, dw, ws)
 
     load(0)
     side = torch.cuda.Stream()

@@ -220,3 +220,71 @@ def test_linear_autograd_clears_the_entry_after_backward(mx):
     assert keep.stats()["entries"] == 1
     cache.close()
     keep.close()
+
+
+def _linear_inputs(M, N, K, seed):
+    if M:
+        return S.linear_problem(M=M, N=N, K=K, seed=seed, device="cuda")
+    return (torch.empty(0, K, dtype=torch.bfloat16, device="cuda"),
+            S.normal_bf16((N, K), 0.02, seed=seed, device="cuda"),
+            torch.empty(0, N, dtype=torch.bfloat16, device="cuda"))
+
+
+def _separate_calls(mx, x, w, dy):
+    M, K = x.shape
+    N = w.shape[0]
+    out = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda"),
+           torch.empty(M, K, dtype=torch.bfloat16, device="cuda"),
+           torch.empty(N, K, dtype=torch.bfloat16, device="cuda")]
+    ws = mx.linear_workspace(M, N, K)
+    mx.mx_linear_fwd(x, w, None, 0, out[0], ws)
+    mx.mx_linear_bwd(dy, x, w, None, 0, out[1], out[2], ws)
+    return out
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 512, 256), (256, 96, 576), (96, 256, 128), (0, 256, 256)])
+@pytest.mark.parametrize("cached", [False, True])
+def test_training_pair_is_bitwise_the_separate_calls(mx, M, N, K, cached):
+    """mx_linear_fwd_train + mx_linear_bwd_after_fwd give y, dX and dW bitwise
+    equal to mx_linear_fwd + mx_linear_bwd on the same x, w and dY. The backward
+    reads neither x (zeroed after the forward here) nor, without a cache, w
+    (doubled in between: the gradient stays that of the forward's product).
+    Shapes: aligned, the GEMM pad path with K > 2N (the pair's larger
+    workspace), M off the 128-row tile, and no tokens."""
+    x, w, dy = _linear_inputs(M, N, K, seed=7)
+    ref = _separate_calls(mx, x, w, dy)
+    cache = mx.WeightCache() if cached else None
+    ver = cache.key_version(w) if cached else 0
+    got = [torch.full_like(t, float("nan")) for t in ref]
+    ws = mx.linear_workspace(M, N, K, train=True)
+    mx.mx_linear_fwd_train(x, w, cache, ver, got[0], ws)
+    x.zero_()
+    if not cached:
+        w.mul_(2)
+    mx.mx_linear_bwd_after_fwd(dy, w, cache, ver, got[1], got[2], ws)
+    torch.cuda.synchronize()
+    mx.mx_device_error()
+    for name, a, b in zip(("y", "dx", "dw"), got, ref):
+        assert torch.equal(a, b), f"{name} of the training pair at M={M}, N={N}, K={K}"
+    if cached:
+        st = cache.stats()
+        assert (st["misses"], st["hits"]) == (1, 1), st     # the backward reuses the forward's entry
+        cache.close()
+
+
+def test_autograd_linear_runs_the_training_pair(mx):
+    """mxfp8_linear under autograd: y, dX and dW bitwise those of the separate
+    calls, x not saved for the backward (only w is), and a forward without
+    gradients (mx_linear_fwd) gives the same y."""
+    M, N, K = 256, 96, 576
+    x, w, dy = _linear_inputs(M, N, K, seed=11)
+    ref = _separate_calls(mx, x, w, dy)
+    xg, wg = x.clone().requires_grad_(), w.clone().requires_grad_()
+    y = mx.mxfp8_linear(xg, wg)
+    assert len(y.grad_fn.saved_tensors) == 1
+    y.backward(dy)
+    assert torch.equal(y.detach(), ref[0])
+    assert torch.equal(xg.grad, ref[1]) and torch.equal(wg.grad, ref[2])
+    with torch.no_grad():
+        assert torch.equal(mx.mxfp8_linear(x, w), ref[0])
+    mx.mx_device_error()
