@@ -583,9 +583,12 @@ BACKWARD_OVERRIDES = (None, "quantized", "high_precision", "dequantized")
 class MXFP8GroupedMM:
     """MXFP8 grouped GEMM of an MoE layer, y[rows of g] = x[rows of g] @ w[g]^T.
 
-    forward(x [M, K], w [G, N, K], offs) casts x rowwise into the padded group
-    layout and w in 32x32 tiles, and runs the scaled grouped GEMM; backward(dy)
-    returns (dx, dw). ``backward_override`` selects where the gradients come
+    forward(x [M, K], w [G, N, K], offs) casts x into the padded group layout
+    and w in 32x32 tiles, and runs the scaled grouped GEMM; backward(dy)
+    returns (dx, dw). In the MXFP8 backward x is cast rowwise and columnwise
+    from one read in the forward (the fused grouped cast), and its columnwise
+    codes -- one byte per element -- are kept for the wgrad instead of x
+    itself, so the backward casts dy alone. ``backward_override`` selects where the gradients come
     from (ao "[moe training] Add backward_override to the MXFP8 grouped GEMM",
     Design notes): None or "quantized" (alias) is the MXFP8 backward;
     "high_precision" uses bf16 grouped GEMMs on the saved bf16 x and w;
@@ -620,7 +623,11 @@ class MXFP8GroupedMM:
         if offs.numel() != G:
             raise ValueError("offs must hold one end offset per expert")
         m_cap = mx_padded_rows_capacity(M, G)
-        xq, xs = cast_dim0_grouped(x, offs, m_cap)
+        keep_codes = self.backward_override is None and not self.wgrad_with_hp
+        if keep_codes:          # the wgrad's columnwise codes of x, from the forward's one read of x
+            xq, xs, xqt, xst = cast_2d_grouped(x, offs, m_cap)
+        else:
+            xq, xs = cast_dim0_grouped(x, offs, m_cap)
         wq, wsf, _, wsd = cast_w32x32(w, transposed=False, dgrad_scales=self.backward_override is None)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
         mx_grouped_mm(xq, xs, wq, wsf, offs, G, MX_GROUPS_M, y, M, N, K, m_cap)
@@ -628,6 +635,8 @@ class MXFP8GroupedMM:
             self._saved = (x, w, offs)
         elif self.backward_override == "dequantized":
             self._saved = (xq, xs, wq, wsf, offs, M, m_cap)
+        elif keep_codes:
+            self._saved = ((xqt, xst, M, K), wq, wsd, offs, m_cap)
         else:
             self._saved = (x, wq, wsd, offs, m_cap)
         return y
@@ -648,18 +657,18 @@ class MXFP8GroupedMM:
             wd = dequant_dim0(wq, wsf)
             return grouped_mm_bf16(dy, wd, offs), grouped_mm_bf16_wgrad(dy, xd, offs)
         x, wq, wsd, offs, m_cap = saved
-        M, K = x.shape
         G, N, _ = wq.shape
         if self.wgrad_with_hp:
+            M, K = x.shape
             dq, ds = cast_dim0_grouped(dy, offs, m_cap)
             dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
             mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
             return dx, grouped_mm_bf16_wgrad(dy, x, offs)
+        xqt, xst, M, K = x
         dq, ds, dqt, dst = cast_2d_grouped(dy, offs, m_cap)
-        xqt, xst = cast_dim1_grouped(x, offs, m_cap)
-        dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
         mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
-        dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=x.device)
+        dw = torch.empty(G, N, K, dtype=torch.bfloat16, device=dy.device)
         mx_grouped_mm(dqt, dst, xqt, xst, offs, G, MX_GROUPS_K, dw, M, N, K, m_cap)
         return dx, dw
 

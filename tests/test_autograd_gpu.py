@@ -68,3 +68,27 @@ def test_linear_autograd_with_cache(mx):
     err = np.abs(y1.detach().float().cpu().numpy() - ref)
     assert np.all(err <= O.gemm_bound(ref, absref))
     cache.close()
+
+
+def test_grouped_layer_backward_reads_the_forwards_codes_not_x(mx):
+    """The MXFP8 backward of the grouped layer takes the wgrad's columnwise codes
+    of x from the forward's fused cast: x overwritten between forward and backward
+    leaves y, dX and dW bitwise those of an untouched run (ragged and empty groups)."""
+    G, N, K = 4, 256, 384
+    sizes = [300, 0, 129, 595]
+    M = sum(sizes)
+    x = S.normal_bf16((M, K), seed=5, device="cuda")
+    w = S.normal_bf16((G, N, K), 0.02, seed=6, device="cuda")
+    dy = S.normal_bf16((M, N), 0.1, seed=7, device="cuda")
+    offs = S.offsets_from_sizes(sizes).cuda()
+    op = mx.MXFP8GroupedMM()
+    y_ref = op.forward(x, w, offs)
+    ref = op.backward(dy)
+    op = mx.MXFP8GroupedMM()
+    y = op.forward(x, w, offs)
+    x.zero_()
+    got = op.backward(dy)
+    mx.mx_device_error()
+    assert torch.equal(y, y_ref)
+    for name, a, b in zip(("dx", "dw"), got, ref):
+        assert torch.equal(a, b), name
