@@ -6,7 +6,11 @@
  *   2. runs the linear forward twice -- with a caller workspace
  *      (mx_linear_fwd) and without any allocation (mx_linear_fwd_noalloc) --
  *      and requires the two outputs to be bitwise equal;
- *   3. requires an invalid call (a width that is not a multiple of 32) to
+ *   3. runs the linear backward after the forward both as separate calls
+ *      (mx_linear_fwd + mx_linear_bwd) and as the training pair
+ *      (mx_linear_fwd_train + mx_linear_bwd_after_fwd, whose backward reuses
+ *      the forward's casts) and requires y, dx and dw to be bitwise equal;
+ *   4. requires an invalid call (a width that is not a multiple of 32) to
  *      return MX_ERR_UNSUPPORTED with a reason, before touching any buffer.
  * Usage: mx_c_host OUT ; exit status 0 when every check holds. */
 #include <stdint.h>
@@ -81,12 +85,17 @@ int main(int argc, char** argv) {
   uint8_t* hs = (uint8_t*)malloc(sbytes);
   uint16_t* hy1 = (uint16_t*)malloc(sizeof(uint16_t) * M * N);
   uint16_t* hy2 = (uint16_t*)malloc(sizeof(uint16_t) * M * N);
-  if (!hx || !hw || !hq || !hs || !hy1 || !hy2) return 4;
+  uint16_t* hg1 = (uint16_t*)malloc(sizeof(uint16_t) * (M * K + N * K));
+  uint16_t* hg2 = (uint16_t*)malloc(sizeof(uint16_t) * (M * K + N * K));
+  uint16_t* hdy = (uint16_t*)malloc(sizeof(uint16_t) * M * N);
+  if (!hx || !hw || !hq || !hs || !hy1 || !hy2 || !hg1 || !hg2 || !hdy) return 4;
   for (int i = 0; i < M * K; ++i) hx[i] = random_bf16(127);
   for (int i = 0; i < N * K; ++i) hw[i] = random_bf16(121);
+  for (int i = 0; i < M * N; ++i) hdy[i] = random_bf16(120);
 
-  void *dx, *dw, *dq, *ds, *dy1, *dy2, *ws;
+  void *dx, *dw, *dq, *ds, *dy1, *dy2, *ws, *ddy, *g1, *g2, *wst;
   const size_t ws_bytes = mx_linear_ws_bytes(M, N, K);
+  const size_t wst_bytes = mx_linear_train_ws_bytes(M, N, K);
   CHECK_CUDA(cudaMalloc(&dx, sizeof(uint16_t) * M * K));
   CHECK_CUDA(cudaMalloc(&dw, sizeof(uint16_t) * N * K));
   CHECK_CUDA(cudaMalloc(&dq, M * K));
@@ -94,6 +103,11 @@ int main(int argc, char** argv) {
   CHECK_CUDA(cudaMalloc(&dy1, sizeof(uint16_t) * M * N));
   CHECK_CUDA(cudaMalloc(&dy2, sizeof(uint16_t) * M * N));
   CHECK_CUDA(cudaMalloc(&ws, ws_bytes));
+  CHECK_CUDA(cudaMalloc(&wst, wst_bytes));
+  CHECK_CUDA(cudaMalloc(&ddy, sizeof(uint16_t) * M * N));
+  CHECK_CUDA(cudaMalloc(&g1, sizeof(uint16_t) * (M * K + N * K)));   /* dx then dw */
+  CHECK_CUDA(cudaMalloc(&g2, sizeof(uint16_t) * (M * K + N * K)));
+  CHECK_CUDA(cudaMemcpy(ddy, hdy, sizeof(uint16_t) * M * N, cudaMemcpyHostToDevice));
   CHECK_CUDA(cudaMemcpy(dx, hx, sizeof(uint16_t) * M * K, cudaMemcpyHostToDevice));
   CHECK_CUDA(cudaMemcpy(dw, hw, sizeof(uint16_t) * N * K, cudaMemcpyHostToDevice));
 
@@ -117,7 +131,25 @@ int main(int argc, char** argv) {
     return 6;
   }
 
-  /* 3. an invalid call is refused on the host */
+  /* 3. separate calls against the training pair: y, dx and dw bitwise equal */
+  uint16_t* g1dw = (uint16_t*)g1 + M * K;
+  uint16_t* g2dw = (uint16_t*)g2 + M * K;
+  CHECK_MX(mx_linear_fwd(dx, dw, M, N, K, NULL, 0, dy1, ws, ws_bytes, NULL));
+  CHECK_MX(mx_linear_bwd(ddy, dx, dw, M, N, K, NULL, 0, g1, g1dw, ws, ws_bytes, NULL));
+  CHECK_MX(mx_linear_fwd_train(dx, dw, M, N, K, NULL, 0, dy2, wst, wst_bytes, NULL));
+  CHECK_MX(mx_linear_bwd_after_fwd(ddy, dw, M, N, K, NULL, 0, g2, g2dw, wst, wst_bytes, NULL));
+  CHECK_MX(mx_device_error(NULL));
+  CHECK_CUDA(cudaMemcpy(hy1, dy1, sizeof(uint16_t) * M * N, cudaMemcpyDeviceToHost));
+  CHECK_CUDA(cudaMemcpy(hy2, dy2, sizeof(uint16_t) * M * N, cudaMemcpyDeviceToHost));
+  CHECK_CUDA(cudaMemcpy(hg1, g1, sizeof(uint16_t) * (M * K + N * K), cudaMemcpyDeviceToHost));
+  CHECK_CUDA(cudaMemcpy(hg2, g2, sizeof(uint16_t) * (M * K + N * K), cudaMemcpyDeviceToHost));
+  if (memcmp(hy1, hy2, sizeof(uint16_t) * M * N) != 0 ||
+      memcmp(hg1, hg2, sizeof(uint16_t) * (M * K + N * K)) != 0) {
+    fprintf(stderr, "linear: the training pair differs from the separate calls\n");
+    return 8;
+  }
+
+  /* 4. an invalid call is refused on the host */
   const mx_status bad = mx_cast_dim0(dx, M, 48, dq, ds, NULL);
   if (bad != MX_ERR_UNSUPPORTED || mx_last_error() == NULL || mx_last_error()[0] == '\0') {
     fprintf(stderr, "a 48-wide cast returned %d\n", (int)bad);
@@ -131,12 +163,19 @@ int main(int argc, char** argv) {
   cudaFree(dy1);
   cudaFree(dy2);
   cudaFree(ws);
+  cudaFree(wst);
+  cudaFree(ddy);
+  cudaFree(g1);
+  cudaFree(g2);
   free(hx);
   free(hw);
   free(hq);
   free(hs);
   free(hy1);
   free(hy2);
+  free(hg1);
+  free(hg2);
+  free(hdy);
   printf("ok\n");
   return 0;
 }

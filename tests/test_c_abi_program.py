@@ -5,7 +5,8 @@ Without a GPU: the program compiles as C99 with every warning an error and
 links against the library's exports. On a B200: it runs, casts a bf16 matrix
 rowwise (its codes and blocked scales are checked here bit for bit against the
 oracle), requires the linear forward with a workspace and without any
-allocation to agree bitwise, and requires a bad width to be refused.
+allocation to agree bitwise, the linear training pair to agree bitwise with the separate
+forward and backward calls, and requires a bad width to be refused.
 """
 import os
 import subprocess
