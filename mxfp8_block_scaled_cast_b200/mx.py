@@ -332,7 +332,10 @@ class WeightCache:
     ``clear_after_backward`` (default on): the MXFP8 linear's backward drops
     the weight's entry when it has finished, as the page's cache is cleared
     after backward (same page, Overview); a recompute forward inside the
-    backward (activation checkpointing) still hits.
+    backward (activation checkpointing) still hits. That holds for
+    non-reentrant checkpointing; the reentrant form recomputes on detached
+    aliases of the weights, new tensor objects to this cache, so there the
+    recompute re-quantizes (correct, not faster).
     """
 
     _serials = itertools.count(1)
@@ -721,21 +724,23 @@ class _LinearFn(torch.autograd.Function):
             return y
         ws = linear_workspace(M, N, K, x.device, train=True)
         mx_linear_fwd_train(x, w, cache, version, y, ws)
-        ctx.save_for_backward(w)        # autograd refuses the backward if w is updated in place meanwhile
-        ctx.cache, ctx.version, ctx.ws, ctx.M = cache, version, ws, M
+        # w: autograd refuses the backward if it is updated in place meanwhile; the
+        # workspace (x's codes) is saved the same way, so that activation
+        # checkpointing drops it after the forward and re-creates it by recompute
+        ctx.save_for_backward(w, ws)
+        ctx.cache, ctx.version, ctx.M = cache, version, M
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        w, = ctx.saved_tensors
+        w, ws = ctx.saved_tensors
         dy = _check_bf16(dy)
         N, K = w.shape
         dx = torch.empty(ctx.M, K, dtype=torch.bfloat16, device=w.device)
         dw = torch.empty(N, K, dtype=torch.bfloat16, device=w.device)
-        mx_linear_bwd_after_fwd(dy, w, ctx.cache, ctx.version, dx, dw, ctx.ws)
+        mx_linear_bwd_after_fwd(dy, w, ctx.cache, ctx.version, dx, dw, ws)
         if ctx.cache is not None and ctx.cache.clear_after_backward:
             ctx.cache.evict(w)
-        ctx.ws = None
         return dx, dw, None
 
 

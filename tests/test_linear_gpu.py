@@ -274,17 +274,61 @@ def test_training_pair_is_bitwise_the_separate_calls(mx, M, N, K, cached):
 
 def test_autograd_linear_runs_the_training_pair(mx):
     """mxfp8_linear under autograd: y, dX and dW bitwise those of the separate
-    calls, x not saved for the backward (only w is), and a forward without
-    gradients (mx_linear_fwd) gives the same y."""
+    calls, x not saved for the backward (w and the workspace holding x's codes
+    are), and a forward without gradients (mx_linear_fwd) gives the same y."""
     M, N, K = 256, 96, 576
     x, w, dy = _linear_inputs(M, N, K, seed=11)
     ref = _separate_calls(mx, x, w, dy)
     xg, wg = x.clone().requires_grad_(), w.clone().requires_grad_()
     y = mx.mxfp8_linear(xg, wg)
-    assert len(y.grad_fn.saved_tensors) == 1
+    saved = y.grad_fn.saved_tensors
+    assert len(saved) == 2 and saved[0] is wg and saved[1].dtype == torch.uint8
     y.backward(dy)
     assert torch.equal(y.detach(), ref[0])
     assert torch.equal(xg.grad, ref[1]) and torch.equal(wg.grad, ref[2])
     with torch.no_grad():
         assert torch.equal(mx.mxfp8_linear(x, w), ref[0])
     mx.mx_device_error()
+
+
+@pytest.mark.parametrize("use_reentrant", [False, True])
+def test_checkpointed_segment_with_the_cache_is_bitwise_the_plain_run(mx, use_reentrant):
+    """Full activation checkpointing ("Cache quantized weights for full AC",
+    prime-rl PR #3388, Overview: checkpoint grad parity; the cache is cleared
+    after backward so training stays bit-identical to an uncheckpointed run): a
+    segment of two MXFP8 linears around a GELU, under torch.utils.checkpoint with
+    a weight cache, gives the loss and every gradient bitwise equal to the same
+    segment run without checkpointing and without a cache, and the backward leaves
+    the cache empty; with non-reentrant checkpointing the recompute forward hits."""
+    from torch.utils.checkpoint import checkpoint
+    M, D, H = 256, 512, 768
+    x0 = S.normal_bf16((M, D), seed=21).cuda()
+    w1_0 = S.normal_bf16((H, D), 0.02, seed=22).cuda()
+    w2_0 = S.normal_bf16((D, H), 0.02, seed=23).cuda()
+
+    def segment(x, w1, w2, cache):
+        h = torch.nn.functional.gelu(mx.mxfp8_linear(x, w1, cache))
+        return mx.mxfp8_linear(h, w2, cache)
+
+    def run(ckpt, cache):
+        x, w1, w2 = (t.clone().requires_grad_() for t in (x0, w1_0, w2_0))
+        y = checkpoint(segment, x, w1, w2, cache, use_reentrant=use_reentrant) if ckpt else segment(x, w1, w2, cache)
+        loss = y.float().pow(2).sum()
+        loss.backward()
+        return loss.detach(), x.grad, w1.grad, w2.grad
+
+    ref = run(False, None)
+    cache = mx.WeightCache()
+    got = run(True, cache)
+    mx.mx_device_error()
+    for name, a, b in zip(("loss", "dx", "dw1", "dw2"), got, ref):
+        assert torch.equal(a, b), f"{name} under checkpointing (use_reentrant={use_reentrant})"
+    st = cache.stats()
+    if use_reentrant:
+        # the reentrant form recomputes on detached aliases of the weights: new tensor
+        # objects to the cache's per-object identity, so the recompute re-quantizes
+        # (two more misses) instead of risking a stale hit; the backward then hits
+        assert (st["misses"], st["hits"], st["entries"]) == (4, 2, 0), st
+    else:
+        assert st["misses"] == 2 and st["hits"] >= 2 and st["entries"] == 0, st
+    cache.close()
