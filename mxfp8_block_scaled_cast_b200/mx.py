@@ -677,20 +677,48 @@ class MXFP8GroupedMM:
 
 
 # ------------------------------------------------------------- autograd --
+def _flatten_saved(obj, tensors):
+    """(layout, tensors): the tensors of a nested tuple pulled out in order."""
+    if isinstance(obj, torch.Tensor):
+        tensors.append(obj)
+        return ("t", len(tensors) - 1)
+    if isinstance(obj, tuple):
+        return ("tuple", tuple(_flatten_saved(o, tensors) for o in obj))
+    return ("v", obj)
+
+
+def _unflatten_saved(layout, tensors):
+    kind, val = layout
+    if kind == "t":
+        return tensors[val]
+    if kind == "tuple":
+        return tuple(_unflatten_saved(v, tensors) for v in val)
+    return val
+
+
 class _GroupedMMFn(torch.autograd.Function):
-    """Autograd wrapper of MXFP8GroupedMM: forward and backward are its calls."""
+    """Autograd wrapper of MXFP8GroupedMM: forward and backward are its calls.
+    What the backward needs (x's columnwise codes, or the bf16 operands for the
+    high-precision arms, the weight's codes and the offsets) is saved with
+    save_for_backward, so that activation checkpointing drops it after the
+    forward and re-creates it by recompute."""
 
     @staticmethod
     def forward(ctx, x, w, offs, backward_override, wgrad_with_hp):
         op = MXFP8GroupedMM(backward_override=backward_override, wgrad_with_hp=wgrad_with_hp)
         y = op.forward(x, w, offs)
+        tensors = []
+        ctx.layout = _flatten_saved(op._saved, tensors)
+        op._saved = None
+        ctx.save_for_backward(*tensors)
         ctx.op = op
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        dx, dw = ctx.op.backward(dy)
-        ctx.op = None
+        op, ctx.op = ctx.op, None
+        op._saved = _unflatten_saved(ctx.layout, ctx.saved_tensors)
+        dx, dw = op.backward(dy)
         return dx, dw, None, None, None
 
 

@@ -92,3 +92,34 @@ def test_grouped_layer_backward_reads_the_forwards_codes_not_x(mx):
     assert torch.equal(y, y_ref)
     for name, a, b in zip(("dx", "dw"), got, ref):
         assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("use_reentrant", [False, True])
+@pytest.mark.parametrize("arm", [None, "high_precision", "dequantized"])
+def test_checkpointed_grouped_layer_is_bitwise_the_plain_run(mx, arm, use_reentrant):
+    """The grouped layer under torch.utils.checkpoint (its saved codes and operands
+    dropped after the forward and recomputed in the backward) gives the loss and
+    both gradients bitwise equal to the plain run, for each backward arm."""
+    from torch.utils.checkpoint import checkpoint
+    G, N, K = 4, 256, 384
+    sizes = [300, 0, 129, 595]
+    M = sum(sizes)
+    x0 = S.normal_bf16((M, K), seed=31, device="cuda")
+    w0 = S.normal_bf16((G, N, K), 0.02, seed=32, device="cuda")
+    offs = S.offsets_from_sizes(sizes).cuda()
+
+    def layer(a, b):
+        return mx.mxfp8_grouped_mm(a, b, offs, backward_override=arm)
+
+    def run(ckpt):
+        x, w = x0.clone().requires_grad_(), w0.clone().requires_grad_()
+        y = checkpoint(layer, x, w, use_reentrant=use_reentrant) if ckpt else layer(x, w)
+        loss = y.float().pow(2).sum()
+        loss.backward()
+        return loss.detach(), x.grad, w.grad
+
+    ref = run(False)
+    got = run(True)
+    mx.mx_device_error()
+    for name, a, b in zip(("loss", "dx", "dw"), got, ref):
+        assert torch.equal(a, b), f"{name} under checkpointing ({arm}, use_reentrant={use_reentrant})"
