@@ -412,7 +412,8 @@ MX_API mx_status mx_linear_bwd(const void* dy, const void* x, const void* w,
  * once the forward's work on `stream` is done.
  * ws: caller-owned, at least mx_linear_train_ws_bytes(M, N, K) bytes -- x's
  * columnwise cast, then the larger of x's rowwise and dy's casts, then w's
- * quantization; more than mx_linear_ws_bytes when K > 2N, because the forward
+ * quantization; more than mx_linear_ws_bytes when x's rowwise cast takes more
+ * bytes than dy's two casts (K > 2N, up to scale padding), because the forward
  * holds both casts of x at once. Size rules and errors as mx_linear_fwd and
  * mx_linear_bwd (a workspace below mx_linear_train_ws_bytes: MX_ERR_ARG). */
 MX_API size_t mx_linear_train_ws_bytes(int64_t M, int64_t N, int64_t K);
