@@ -38,7 +38,6 @@ import hashlib
 import json
 import os
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -89,8 +88,84 @@ def aggregate(step_ms_local, steps, world):
     return value, ms_per_step
 
 
+# The sampler runs in a process of its own: NVML readings stamped with the
+# system-wide monotonic clock by that process, so a busy host thread holding
+# the interpreter lock cannot thin them out. One per device, shared by every
+# measured region; each region keeps the readings stamped inside it.
+_SAMPLER_SRC = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+dev, period, deadline, path = sys.argv[1], float(sys.argv[2]), time.monotonic() + float(sys.argv[3]), sys.argv[4]
+try:
+    h, how = pynvml.nvmlDeviceGetHandleByUUID(dev), "uuid"
+except Exception:
+    h, how = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[5])), "index"
+with open(path, "a", buffering=1) as out:
+    out.write("# " + how + "\n")
+    while time.monotonic() < deadline:
+        try:
+            mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            out.write("%.6f %d %d\n" % (time.monotonic(), mhz, mask))
+        except Exception:
+            pass
+        time.sleep(period)
+"""
+_samplers = {}
+
+
+def start_clock_sampler(local, period_s=0.0005, lifetime_s=3600.0):
+    """Start (once) the NVML sampler process of CUDA device `local`; returns its
+    (output path, max SM MHz) or None without NVML. NVML does not see
+    CUDA_VISIBLE_DEVICES, so the device is named by its UUID (index as fallback)."""
+    if local in _samplers:
+        return _samplers[local]
+    import atexit
+    import subprocess
+    import tempfile
+    try:
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+        try:
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByIndex(local)
+        max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:
+        _samplers[local] = None
+        return None
+    fd, path = tempfile.mkstemp(prefix="mx_clocks_", suffix=".txt")
+    os.close(fd)
+    proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, uuid, str(period_s), str(lifetime_s), path,
+                             str(local)], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+
+    def _stop():
+        proc.terminate()
+        try:
+            proc.wait(timeout=5)
+        except Exception:
+            proc.kill()
+        try:
+            os.remove(path)
+        except OSError:
+            pass
+    atexit.register(_stop)
+    t_end = time.monotonic() + 20.0          # until its first reading is in
+    while time.monotonic() < t_end and proc.poll() is None:
+        with open(path) as fh:
+            if sum(1 for line in fh if not line.startswith("#")) > 0:
+                break
+        time.sleep(0.01)
+    _samplers[local] = (path, max_mhz)
+    return _samplers[local]
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML during a region."""
+    """SM clock and clock-event reasons of one device during a region (readings
+    of the sampler process whose stamps fall between entry and exit)."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
@@ -98,49 +173,39 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period_s=0.0005):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
-        self.period, self.index = period_s, index
-        self._stop = threading.Event()
-        self._thread = None
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nvml = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-        except Exception:
-            self.nvml = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
-                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if mask & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+    def __init__(self, local):
+        self.sampler = start_clock_sampler(local)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
-        if self.nvml is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._thread is not None:
-            self._thread.join()
+        self.t1 = time.monotonic()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        s = sorted(self.samples)
-        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(s)}
+        if self.sampler is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        path, max_mhz = self.sampler
+        t1 = self.t1 if self.t1 is not None else time.monotonic()
+        mhz, reasons, device = [], set(), None
+        with open(path) as fh:
+            for line in fh:
+                if line.startswith("#"):
+                    device = line[1:].strip()
+                    continue
+                parts = line.split()
+                if len(parts) != 3 or not (self.t0 <= float(parts[0]) <= t1):
+                    continue
+                mhz.append(int(parts[1]))
+                mask = int(parts[2])
+                reasons.update(n for n, bit in self.REASONS.items() if mask & bit and n != "gpu_idle")
+        out = {"sm_mhz": sorted(mhz)[len(mhz) // 2] if mhz else None, "sm_max_mhz": max_mhz,
+               "reasons": sorted(reasons), "samples": len(mhz)}
+        if device is not None:
+            out["nvml_device_by"] = device
+        return out
 
 
 def profile_traffic(name, source_files):
@@ -1067,6 +1132,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     mx.lib()
     dev = torch.device("cuda", local)
+    start_clock_sampler(local)          # running well before any timed region
     peaks, peak_src = load_peaks()
     step = MoEStep(mx, dev, seed=0)
 

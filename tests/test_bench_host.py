@@ -114,3 +114,39 @@ def test_peak_follows_the_length_of_the_timed_region_and_the_power_cap():
     # a measured file without a figure falls back to the recorded ones
     assert bench.select_peak(16.3, [], {})[1] == bench.FALLBACK_PEAKS["bf16_tflops"]
     assert bench.select_peak(250.0, [], {})[1] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+
+
+def test_clock_sampler_process_keeps_the_readings_inside_a_region(tmp_path):
+    """The NVML sampler runs as a process of its own (a fake NVML module here):
+    its readings carry their own monotonic stamps, and a region keeps exactly
+    the readings stamped inside it, with the clock-event reasons they flag
+    (gpu_idle left out) and how the device was found."""
+    import time
+    import bench
+    fake = tmp_path / "fake"
+    fake.mkdir()
+    (fake / "pynvml.py").write_text(
+        "NVML_CLOCK_SM = 0\n"
+        "def nvmlInit(): pass\n"
+        "def nvmlDeviceGetHandleByUUID(u): return u\n"
+        "def nvmlDeviceGetHandleByIndex(i): return i\n"
+        "def nvmlDeviceGetClockInfo(h, c): return 1800\n"
+        "def nvmlDeviceGetCurrentClocksEventReasons(h): return 0x5\n")      # gpu_idle | sw_power_cap
+    out = tmp_path / "clocks.txt"
+    out.write_text("")
+    env = dict(os.environ, PYTHONPATH=str(fake))
+    proc = subprocess.Popen([sys.executable, "-c", bench._SAMPLER_SRC, "GPU-0", "0.001", "2", str(out), "0"],
+                            env=env)
+    try:
+        time.sleep(0.5)
+        region = bench.ClockSampler.__new__(bench.ClockSampler)
+        region.sampler = (str(out), 1965)
+        with region:
+            time.sleep(0.2)
+    finally:
+        proc.wait(timeout=30)
+    s = region.summary()
+    assert s["samples"] >= 20 and s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["nvml_device_by"] == "uuid"
+    readings = sum(1 for line in open(out) if not line.startswith("#"))
+    assert readings > s["samples"]                      # the readings outside the region are left out
