@@ -591,9 +591,10 @@ class MXFP8GroupedMM:
     returns (dx, dw). In the MXFP8 backward x is cast rowwise and columnwise
     from one read in the forward (the fused grouped cast), and its columnwise
     codes -- one byte per element -- are kept for the wgrad instead of x
-    itself, so the backward casts dy alone. ``backward_override`` selects where the gradients come
-    from (ao "[moe training] Add backward_override to the MXFP8 grouped GEMM",
-    Design notes): None or "quantized" (alias) is the MXFP8 backward;
+    itself, so the backward casts dy alone. ``backward_override`` selects
+    where the gradients come from (ao "[moe training] Add backward_override to
+    the MXFP8 grouped GEMM", Design notes): None or "quantized" (alias) is the
+    MXFP8 backward;
     "high_precision" uses bf16 grouped GEMMs on the saved bf16 x and w;
     "dequantized" uses the same bf16 GEMMs on the forward's codes turned back
     into bf16 (the gradient of the function the quantized forward computes).
@@ -659,15 +660,16 @@ class MXFP8GroupedMM:
             xd = dequant_dim0_grouped(xq, xs, offs, M)
             wd = dequant_dim0(wq, wsf)
             return grouped_mm_bf16(dy, wd, offs), grouped_mm_bf16_wgrad(dy, xd, offs)
-        x, wq, wsd, offs, m_cap = saved
+        acts, wq, wsd, offs, m_cap = saved       # x (wgrad_with_hp) or (x's columnwise codes, scales, M, K)
         G, N, _ = wq.shape
         if self.wgrad_with_hp:
+            x = acts
             M, K = x.shape
             dq, ds = cast_dim0_grouped(dy, offs, m_cap)
             dx = torch.empty(M, K, dtype=torch.bfloat16, device=x.device)
             mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
             return dx, grouped_mm_bf16_wgrad(dy, x, offs)
-        xqt, xst, M, K = x
+        xqt, xst, M, K = acts
         dq, ds, dqt, dst = cast_2d_grouped(dy, offs, m_cap)
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=dy.device)
         mx_grouped_mm(dq, ds, wq, wsd, offs, G, MX_GROUPS_M_KN, dx, M, K, N, m_cap)
@@ -678,7 +680,7 @@ class MXFP8GroupedMM:
 
 # ------------------------------------------------------------- autograd --
 def _flatten_saved(obj, tensors):
-    """(layout, tensors): the tensors of a nested tuple pulled out in order."""
+    """The layout of a nested tuple; its tensors are appended to `tensors` in order."""
     if isinstance(obj, torch.Tensor):
         tensors.append(obj)
         return ("t", len(tensors) - 1)
