@@ -496,21 +496,24 @@ def gemm_only(mx, step, peaks, iters=100, runs=5):
         g.replay()
         torch.cuda.synchronize()
         ts = []
-        for _ in range(runs):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            g.replay()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b) / iters)
+        with ClockSampler(torch.cuda.current_device()) as ck:
+            for _ in range(runs):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) / iters)
         ts.sort()
         tf = step.gemm_flops / (ts[len(ts) // 2] * 1e-3) / 1e12
         out[name] = {"us_per_launch": round(ts[len(ts) // 2] * 1e3, 1), "tflops": round(tf, 1),
                      "frac_of_measured_sustained_fp8": round(tf / sustained, 3),
-                     "frac_of_measured_burst_fp8": round(tf / burst, 3), "frac_of_4500_spec": round(tf / 4500.0, 3)}
+                     "frac_of_measured_burst_fp8": round(tf / burst, 3), "frac_of_4500_spec": round(tf / 4500.0, 3),
+                     "clocks": ck.summary()}
         del g
     mx.mx_device_error()
-    out["method"] = (f"CUDA graph of {iters} back-to-back launches (power-capped), median of {runs} replays; "
+    out["method"] = (f"CUDA graph of {iters} back-to-back launches, median of {runs} replays (about 0.1 s "
+                     f"of load per GEMM: the sustained regime; `clocks` per GEMM); "
                      f"fp8 peaks = measured bf16 (sustained, burst) x {FP8_OVER_BF16}")
     return out
 
