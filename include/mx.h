@@ -19,7 +19,8 @@
  *     and the bf16 grouped GEMMs, dequantization and scale unswizzle of the
  *     backward-override arms (ao backward_override PR, Design notes);
  *   - the MXFP8 linear forward / dgrad / wgrad (ao PR #4705, "MXFP8Linear
- *     training paths") and a per-weight quantization cache keyed by the
+ *     training paths"), also as a training pair whose backward reuses the
+ *     forward's casts, and a per-weight quantization cache keyed by the
  *     weight's version counter ("Cache quantized weights for full AC",
  *     prime-rl PR #3388, Overview).
  *
