@@ -501,3 +501,36 @@ class MXFP8ExpertParallelMM:
         dy_recv = dispatch_bf16(dy.contiguous(), plan, self.a2a)
         dx_recv, dw = expert_backward(dy_recv, rq, rs, wq, wsd, plan)
         return return_grad(dx_recv, plan, self.a2a), dw
+
+
+class _ExpertParallelFn(torch.autograd.Function):
+    """Autograd wrapper of MXFP8ExpertParallelMM: forward and backward are the
+    layer's calls, collectives included (every rank runs them in the same
+    order). In the all-to-all mode the forward's state moves into the autograd
+    context, so several forwards (micro-batches) may precede their backwards,
+    in any order; direct mode keeps it in the layer, whose receive buffers hold
+    the codes the backward reads, and so refuses a second forward before the
+    backward."""
+
+    @staticmethod
+    def forward(ctx, x, w, send_counts, layer):
+        y = layer.forward(x, send_counts, w)
+        ctx.layer = layer
+        if not layer.direct:
+            ctx.state, layer._saved = layer._saved, None
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        layer, ctx.layer = ctx.layer, None
+        if not layer.direct:
+            layer._saved, ctx.state = ctx.state, None
+        dx, dw = layer.backward(dy)
+        return dx, dw, None, None
+
+
+def mxfp8_expert_parallel_mm(x, w, send_counts, layer):
+    """y = the expert-parallel MXFP8 MoE layer `layer` (an MXFP8ExpertParallelMM)
+    on x [M, K] (tokens ordered by global expert, send_counts tokens per global
+    expert) with this rank's experts w [E, N, K]; differentiable in x and w."""
+    return _ExpertParallelFn.apply(x, w, send_counts, layer)

@@ -310,3 +310,52 @@ def test_direct_dy_dispatch_equals_the_experts_own_cast(mx, W, E, N):
         assert torch.equal(bs[d], s.reshape(-1)), f"rowwise scales of rank {d}"
         assert torch.equal(bqt[d], qt.reshape(-1)), f"columnwise codes of rank {d}"
         assert torch.equal(bst[d], st.reshape(-1)), f"columnwise scales of rank {d}"
+
+
+def test_autograd_entry_over_a_one_rank_nccl_group(mx):
+    """mxfp8_expert_parallel_mm through autograd in both modes: y and the
+    gradients bitwise those of the layer's own forward and backward; in the
+    all-to-all mode two forwards (micro-batches) precede their backwards, run in
+    reverse order, and the weight's accumulated gradient is the sum of both."""
+    import torch.distributed as dist
+    from mxfp8_block_scaled_cast_b200 import ep
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        E, N, K = 4, 512, 256
+        counts = np.array([100, 0, 333, 129])
+        M = int(counts.sum())
+        x = S.normal_bf16((M, K), seed=60).cuda()
+        x2 = S.normal_bf16((M, K), seed=63).cuda()
+        w = S.normal_bf16((E, N, K), 0.02, seed=61).cuda()
+        dy = S.normal_bf16((M, N), 0.1, seed=62).cuda()
+        dy2 = S.normal_bf16((M, N), 0.1, seed=64).cuda()
+        ref = ep.MXFP8ExpertParallelMM()
+        y0 = ref.forward(x, counts, w)
+        dx0, dw0 = ref.backward(dy)
+        y2 = ref.forward(x2, counts, w)
+        dx2, dw2 = ref.backward(dy2)
+        for direct in (False, True):
+            layer = ep.MXFP8ExpertParallelMM(direct=direct)
+            xg, wg = x.clone().requires_grad_(), w.clone().requires_grad_()
+            y = ep.mxfp8_expert_parallel_mm(xg, wg, counts, layer)
+            y.backward(dy)
+            assert torch.equal(y.detach(), y0), f"y (direct={direct})"
+            assert torch.equal(xg.grad, dx0) and torch.equal(wg.grad, dw0), f"gradients (direct={direct})"
+        layer = ep.MXFP8ExpertParallelMM()
+        a, b = x.clone().requires_grad_(), x2.clone().requires_grad_()
+        wg = w.clone().requires_grad_()
+        ya = ep.mxfp8_expert_parallel_mm(a, wg, counts, layer)
+        yb = ep.mxfp8_expert_parallel_mm(b, wg, counts, layer)
+        yb.backward(dy2)
+        ya.backward(dy)
+        mx.mx_device_error()
+        assert torch.equal(ya.detach(), y0) and torch.equal(yb.detach(), y2)
+        assert torch.equal(a.grad, dx0) and torch.equal(b.grad, dx2)
+        assert torch.equal(wg.grad, dw2 + dw0)
+    finally:
+        dist.destroy_process_group()
