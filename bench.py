@@ -93,17 +93,18 @@ def aggregate(step_ms_local, steps, world):
 # the interpreter lock cannot thin them out. One per device, shared by every
 # measured region; each region keeps the readings stamped inside it.
 _SAMPLER_SRC = r"""
-import sys, time
+import os, sys, time
 import pynvml
 pynvml.nvmlInit()
 dev, period, deadline, path = sys.argv[1], float(sys.argv[2]), time.monotonic() + float(sys.argv[3]), sys.argv[4]
+parent = int(sys.argv[6])
 try:
     h, how = pynvml.nvmlDeviceGetHandleByUUID(dev), "uuid"
 except Exception:
     h, how = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[5])), "index"
 with open(path, "a", buffering=1) as out:
     out.write("# " + how + "\n")
-    while time.monotonic() < deadline:
+    while time.monotonic() < deadline and os.getppid() == parent:    # ends with its parent, however that ends
         try:
             mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
             mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
@@ -115,7 +116,7 @@ with open(path, "a", buffering=1) as out:
 _samplers = {}
 
 
-def start_clock_sampler(local, period_s=0.0005, lifetime_s=3600.0):
+def start_clock_sampler(local, period_s=0.0005, lifetime_s=1800.0):
     """Start (once) the NVML sampler process of CUDA device `local`; returns its
     (output path, max SM MHz) or None without NVML. NVML does not see
     CUDA_VISIBLE_DEVICES, so the device is named by its UUID (index as fallback)."""
@@ -140,7 +141,7 @@ def start_clock_sampler(local, period_s=0.0005, lifetime_s=3600.0):
     fd, path = tempfile.mkstemp(prefix="mx_clocks_", suffix=".txt")
     os.close(fd)
     proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, uuid, str(period_s), str(lifetime_s), path,
-                             str(local)], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+                             str(local), str(os.getpid())], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
 
     def _stop():
         proc.terminate()

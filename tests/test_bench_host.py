@@ -135,8 +135,8 @@ def test_clock_sampler_process_keeps_the_readings_inside_a_region(tmp_path):
     out = tmp_path / "clocks.txt"
     out.write_text("")
     env = dict(os.environ, PYTHONPATH=str(fake))
-    proc = subprocess.Popen([sys.executable, "-c", bench._SAMPLER_SRC, "GPU-0", "0.001", "2", str(out), "0"],
-                            env=env)
+    proc = subprocess.Popen([sys.executable, "-c", bench._SAMPLER_SRC, "GPU-0", "0.001", "2", str(out), "0",
+                             str(os.getpid())], env=env)
     try:
         time.sleep(0.5)
         region = bench.ClockSampler.__new__(bench.ClockSampler)
@@ -150,3 +150,26 @@ def test_clock_sampler_process_keeps_the_readings_inside_a_region(tmp_path):
     assert s["reasons"] == ["sw_power_cap"] and s["nvml_device_by"] == "uuid"
     readings = sum(1 for line in open(out) if not line.startswith("#"))
     assert readings > s["samples"]                      # the readings outside the region are left out
+
+
+def test_clock_sampler_process_ends_with_its_parent(tmp_path):
+    """A sampler whose parent is gone stops at once (a rank ended by a signal
+    runs no exit handlers), long before its own deadline."""
+    import time
+    import bench
+    fake = tmp_path / "fake"
+    fake.mkdir()
+    (fake / "pynvml.py").write_text(
+        "NVML_CLOCK_SM = 0\n"
+        "def nvmlInit(): pass\n"
+        "def nvmlDeviceGetHandleByUUID(u): return u\n"
+        "def nvmlDeviceGetClockInfo(h, c): return 1800\n"
+        "def nvmlDeviceGetCurrentClocksEventReasons(h): return 0\n")
+    out = tmp_path / "clocks.txt"
+    out.write_text("")
+    env = dict(os.environ, PYTHONPATH=str(fake))
+    t0 = time.monotonic()
+    proc = subprocess.Popen([sys.executable, "-c", bench._SAMPLER_SRC, "GPU-0", "0.001", "60", str(out), "0",
+                             "1"], env=env)           # parent id 1: not its parent, as after the parent died
+    proc.wait(timeout=30)
+    assert time.monotonic() - t0 < 30 and proc.returncode == 0
